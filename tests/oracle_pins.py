@@ -1,0 +1,312 @@
+"""Pins that tie the CPU oracle to facts that do not come from the oracle itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError when the oracle
+disagrees with the fact it pins.  ``tests/test_oracle_pins.py`` runs them on the real
+oracle; ``tests/test_oracle_mutants.py`` plants plausible mistakes in copies of the oracle's
+C source and checks that every mistake trips at least one pin.
+
+Sources (page title, section):
+  [E2D2 notes]  "Encoder-Decoder Diffusion Language Models for Efficient Training and
+                Inference" (paper notes): sec. 3 sampling algorithm, sec. 4 training
+                algorithm with its FLOPs table.
+  [BD3LM blog]  "Block Diffusion: Interpolating Between Autoregressive and Diffusion
+                Language Models": sec. 2 core insight (block size 1 = autoregressive,
+                block size = sequence length = full diffusion).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from block_discrete_diffusion_tcgen05_b200 import synth
+
+GOLDEN_PAIRS = __import__("pathlib").Path(__file__).resolve().parent / "golden" / "pair_counts.txt"
+
+
+def _rand(shape, seed, sigma=1.0):
+    return synth.normal_bf16(shape, seed, sigma).f32
+
+
+def _sdpa(q, k, v, scale, mask=None, causal=False):
+    """torch's own attention routine in float64 on the CPU (a library routine)."""
+    tq, tk, tv = (torch.from_numpy(np.asarray(x, dtype=np.float64)) for x in (q, k, v))
+    m = None if mask is None else torch.from_numpy(mask)
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=m,
+                                                           is_causal=causal, scale=scale)
+    return out.numpy()
+
+
+def _torch_lse(q, k, scale, mask):
+    """torch.logsumexp of the masked scaled scores (library routine)."""
+    tq, tk = (torch.from_numpy(np.asarray(x, dtype=np.float64)) for x in (q, k))
+    s = scale * torch.matmul(tq, tk.transpose(-1, -2))
+    s = s.masked_fill(~torch.from_numpy(mask), float("-inf"))
+    return torch.logsumexp(s, dim=-1).numpy()
+
+
+# ---------------------------------------------------------------------------------------
+# 1. Pair count: the FLOPs table of [E2D2 notes, sec. 4] charges an E2D2 encoder or decoder
+#    pass with (L^2 + L S) / 2 attended pairs (attention FLOPs 4 (N_E+N_D) D (L^2+LS)/2).
+# ---------------------------------------------------------------------------------------
+def pin_pair_count(orc, cases=((8, 1), (8, 2), (8, 8), (12, 3), (16, 4), (64, 8), (48, 16), (32, 32))):
+    for L, S in cases:
+        closed = (L * L + L * S) // 2
+        assert int(orc.mask_encoder(L, S).sum()) == closed, ("encoder", L, S)
+        assert int(orc.mask_decoder(L, S).sum()) == closed, ("decoder", L, S)
+
+
+def read_golden_pairs():
+    rows = []
+    for line in GOLDEN_PAIRS.read_text().splitlines():
+        line = line.split("#", 1)[0].strip()
+        if line:
+            L, S, pairs = (int(x) for x in line.split())
+            rows.append((L, S, pairs))
+    return rows
+
+
+def pin_golden_pairs(orc):
+    for L, S, pairs in read_golden_pairs():
+        assert int(orc.mask_encoder(L, S).sum()) == pairs, ("encoder", L, S)
+        assert int(orc.mask_decoder(L, S).sum()) == pairs, ("decoder", L, S)
+
+
+# ---------------------------------------------------------------------------------------
+# 2. Block size 1 is autoregressive ([BD3LM blog, sec. 2]): the encoder mask is the causal
+#    mask and the encoder output is torch's causal attention.
+# ---------------------------------------------------------------------------------------
+def pin_block_size_one_is_causal(orc):
+    L, d, B, H = 24, 16, 2, 2
+    assert np.array_equal(orc.mask_encoder(L, 1), np.tril(np.ones((L, L), dtype=bool)))
+    q, k, v = (_rand((B, H, L, d), 900 + t) for t in range(3))
+    scale = 0.31
+    out, lse = orc.encoder(q, k, v, S=1, scale=scale)
+    ref = _sdpa(q, k, v, scale, causal=True)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    causal = np.tril(np.ones((L, L), dtype=bool))
+    np.testing.assert_allclose(lse, _torch_lse(q, k, scale, causal), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
+# 3. Block size L is full diffusion ([BD3LM blog, sec. 2]): the encoder is bidirectional;
+#    the decoder sees no encoder key (no earlier block) and its whole own block, i.e. plain
+#    bidirectional attention over the decoder keys.
+# ---------------------------------------------------------------------------------------
+def pin_block_size_L_is_bidirectional(orc):
+    L, d, B, H = 20, 8, 1, 3
+    assert orc.mask_encoder(L, L).all()
+    md = orc.mask_decoder(L, L)
+    assert not md[:, :L].any() and md[:, L:].all()
+    q, k, v, ke, ve = (_rand((B, H, L, d), 910 + t) for t in range(5))
+    scale = 0.5
+    out, lse = orc.encoder(q, k, v, S=L, scale=scale)
+    np.testing.assert_allclose(out, _sdpa(q, k, v, scale), rtol=0, atol=1e-12)
+    full = np.ones((L, L), dtype=bool)
+    np.testing.assert_allclose(lse, _torch_lse(q, k, scale, full), rtol=0, atol=1e-12)
+    out, lse = orc.decoder_train(q, ke, ve, k, v, S=L, scale=scale)
+    np.testing.assert_allclose(out, _sdpa(q, k, v, scale), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, _torch_lse(q, k, scale, full), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
+# 4. Intermediate block sizes against torch's attention with a mask built here from the
+#    mask words of [E2D2 notes, sec. 4] (block ids compared with numpy broadcasting).
+# ---------------------------------------------------------------------------------------
+def _block_ids(L, S):
+    return np.arange(L) // S
+
+
+def pin_masked_against_torch(orc):
+    B, Hq, Hkv, L, S, d = 2, 4, 2, 24, 4, 8
+    G = Hq // Hkv
+    q = _rand((B, Hq, L, d), 920)
+    k, v, ke, ve = (_rand((B, Hkv, L, d), 921 + t) for t in range(4))
+    scale = 0.4
+    bid = _block_ids(L, S)
+    enc_mask = bid[None, :] <= bid[:, None]
+    kr, vr = np.repeat(k, G, axis=1), np.repeat(v, G, axis=1)
+    out, lse = orc.encoder(q, k, v, S=S, scale=scale)
+    np.testing.assert_allclose(out, _sdpa(q, kr, vr, scale, mask=enc_mask), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, _torch_lse(q, kr, scale, enc_mask), rtol=0, atol=1e-12)
+    # decoder: keys = [encoder keys | decoder keys]
+    dec_mask = np.concatenate([bid[None, :] < bid[:, None], bid[None, :] == bid[:, None]], axis=1)
+    kcat = np.concatenate([np.repeat(ke, G, 1), kr], axis=2)
+    vcat = np.concatenate([np.repeat(ve, G, 1), vr], axis=2)
+    out, lse = orc.decoder_train(q, ke, ve, k, v, S=S, scale=scale)
+    np.testing.assert_allclose(out, _sdpa(q, kcat, vcat, scale, mask=dec_mask), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, _torch_lse(q, kcat, scale, dec_mask), rtol=0, atol=1e-12)
+    # scale <= 0 selects the default softmax scale; torch's routine defaults to 1/sqrt(d).
+    out, _ = orc.encoder(q, k, v, S=S, scale=0.0)
+    np.testing.assert_allclose(out, _sdpa(q, kr, vr, None, mask=enc_mask), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
+# 5. Brute force on tiny inputs: allowed keys listed as index ranges (not compared element
+#    by element), scores and sums with math.fsum, one query at a time.
+# ---------------------------------------------------------------------------------------
+def _brute_row(qrow, keys, vals, scale):
+    scores = [scale * math.fsum(a * b for a, b in zip(qrow, kk)) for kk in keys]
+    m = max(scores)
+    w = [math.exp(s - m) for s in scores]
+    tot = math.fsum(w)
+    d = len(vals[0])
+    out = [math.fsum(wi * vv[c] for wi, vv in zip(w, vals)) / tot for c in range(d)]
+    return out, m + math.log(tot)
+
+
+def pin_brute_force(orc):
+    B, Hq, Hkv, L, S, d = 1, 2, 1, 12, 3, 4
+    q = _rand((B, Hq, L, d), 930).astype(np.float64)
+    k, v, ke, ve = (_rand((B, Hkv, L, d), 931 + t).astype(np.float64) for t in range(4))
+    scale = 0.7
+    out_e, lse_e = orc.encoder(q, k, v, S=S, scale=scale)
+    out_d, lse_d = orc.decoder_train(q, ke, ve, k, v, S=S, scale=scale)
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        for i in range(L):
+            b0 = (i // S) * S  # first position of the query's block
+            enc_keys = list(range(0, b0 + S))  # own block and every earlier block
+            o, l = _brute_row(q[0, h, i], [k[0, g, j] for j in enc_keys], [v[0, g, j] for j in enc_keys], scale)
+            np.testing.assert_allclose(out_e[0, h, i], o, rtol=0, atol=1e-12)
+            assert abs(lse_e[0, h, i] - l) < 1e-12
+            keys = [ke[0, g, j] for j in range(0, b0)] + [k[0, g, j] for j in range(b0, b0 + S)]
+            vals = [ve[0, g, j] for j in range(0, b0)] + [v[0, g, j] for j in range(b0, b0 + S)]
+            o, l = _brute_row(q[0, h, i], keys, vals, scale)
+            np.testing.assert_allclose(out_d[0, h, i], o, rtol=0, atol=1e-12)
+            assert abs(lse_d[0, h, i] - l) < 1e-12
+    # sampling step: every query sees the P prefix rows and the S own rows
+    P, cap = 5, 9
+    qs = _rand((B, Hq, S, d), 940).astype(np.float64)
+    kc, vc = (_rand((B, Hkv, cap, d), 941 + t).astype(np.float64) for t in range(2))
+    kb, vb = (_rand((B, Hkv, S, d), 943 + t).astype(np.float64) for t in range(2))
+    out_s, lse_s = orc.decoder_sample(qs, kc, vc, P, kb, vb, scale=scale)
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        keys = [kc[0, g, j] for j in range(P)] + [kb[0, g, j] for j in range(S)]
+        vals = [vc[0, g, j] for j in range(P)] + [vb[0, g, j] for j in range(S)]
+        for i in range(S):
+            o, l = _brute_row(qs[0, h, i], keys, vals, scale)
+            np.testing.assert_allclose(out_s[0, h, i], o, rtol=0, atol=1e-12)
+            assert abs(lse_s[0, h, i] - l) < 1e-12
+
+
+# ---------------------------------------------------------------------------------------
+# 6. Closed form with all-zero keys: every allowed score is 0, so lse_i = ln(n_i) and out_i
+#    is the mean of the allowed values.  n_i = (block(i) + 1) S for both train passes
+#    ([E2D2 notes, sec. 4]: own block plus every earlier block, from one side or the other)
+#    and P + S for the sampling step.
+# ---------------------------------------------------------------------------------------
+def pin_zero_keys_closed_form(orc):
+    B, H, L, S, d = 1, 2, 16, 4, 4
+    q = _rand((B, H, L, d), 950)
+    v, ve = _rand((B, H, L, d), 951), _rand((B, H, L, d), 952)
+    z = np.zeros((B, H, L, d), dtype=np.float32)
+    out, lse = orc.encoder(q, z, v, S=S)
+    for i in range(L):
+        n = (i // S + 1) * S
+        np.testing.assert_allclose(lse[:, :, i], math.log(n), rtol=0, atol=1e-13)
+        np.testing.assert_allclose(out[:, :, i], v[:, :, :n].astype(np.float64).mean(axis=2), rtol=0, atol=1e-12)
+    out, lse = orc.decoder_train(q, z, ve, z, v, S=S)
+    for i in range(L):
+        b0 = (i // S) * S
+        n = b0 + S
+        mean = (ve[:, :, :b0].astype(np.float64).sum(axis=2) + v[:, :, b0:b0 + S].astype(np.float64).sum(axis=2)) / n
+        np.testing.assert_allclose(lse[:, :, i], math.log(n), rtol=0, atol=1e-13)
+        np.testing.assert_allclose(out[:, :, i], mean, rtol=0, atol=1e-12)
+    P, cap = 7, 11
+    qs = _rand((B, H, S, d), 953)
+    vc, vb = _rand((B, H, cap, d), 954), _rand((B, H, S, d), 955)
+    out, lse = orc.decoder_sample(qs, np.zeros((B, H, cap, d), np.float32), vc, P,
+                                  np.zeros((B, H, S, d), np.float32), vb)
+    mean = (vc[:, :, :P].astype(np.float64).sum(axis=2) + vb.astype(np.float64).sum(axis=2)) / (P + S)
+    np.testing.assert_allclose(lse, math.log(P + S), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(out, np.repeat(mean[:, :, None, :], S, axis=2), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
+# 7. Invariants: constant values give that constant; GQA equals MHA with repeated kv heads.
+# ---------------------------------------------------------------------------------------
+def pin_constant_values(orc):
+    B, H, L, S, d = 1, 2, 16, 4, 8
+    q, k = _rand((B, H, L, d), 960), _rand((B, H, L, d), 961)
+    c = np.full((B, H, L, d), 0.375, dtype=np.float32)
+    out, _ = orc.encoder(q, k, c, S=S)
+    np.testing.assert_allclose(out, 0.375, rtol=0, atol=1e-14)
+    out, _ = orc.decoder_train(q, k, c, k, c, S=S)
+    np.testing.assert_allclose(out, 0.375, rtol=0, atol=1e-14)
+
+
+def pin_gqa_is_repeated_heads(orc):
+    B, Hq, Hkv, L, S, d = 1, 6, 2, 16, 4, 8
+    G = Hq // Hkv
+    q = _rand((B, Hq, L, d), 970)
+    k, v, ke, ve = (_rand((B, Hkv, L, d), 971 + t) for t in range(4))
+    rep = lambda t: np.repeat(t, G, axis=1)
+    a = orc.encoder(q, k, v, S=S)
+    b = orc.encoder(q, rep(k), rep(v), S=S)
+    np.testing.assert_array_equal(a[0], b[0])
+    a = orc.decoder_train(q, ke, ve, k, v, S=S)
+    b = orc.decoder_train(q, rep(ke), rep(ve), rep(k), rep(v), S=S)
+    np.testing.assert_array_equal(a[0], b[0])
+    P, cap = 6, 8
+    kc, vc = _rand((B, Hkv, cap, d), 975), _rand((B, Hkv, cap, d), 976)
+    qs = _rand((B, Hq, S, d), 977)
+    a = orc.decoder_sample(qs, kc, vc, P, k[:, :, :S], v[:, :, :S])
+    b = orc.decoder_sample(qs, rep(kc), rep(vc), P, rep(k[:, :, :S]), rep(v[:, :, :S]))
+    np.testing.assert_array_equal(a[0], b[0])
+
+
+# ---------------------------------------------------------------------------------------
+# 8. Sampling step == the matching rows of the training pass ([E2D2 notes, sec. 3 vs 4]):
+#    the noised block b with the encoder cache of blocks < b gives the decoder-train rows of
+#    block b; the encoder rows of block b are a sampling-shaped call over prefix [0, bS)
+#    plus the block itself.
+# ---------------------------------------------------------------------------------------
+def pin_sample_is_train_slice(orc):
+    B, Hq, Hkv, L, S, d = 2, 4, 2, 20, 5, 8
+    q = _rand((B, Hq, L, d), 980)
+    k, v, ke, ve = (_rand((B, Hkv, L, d), 981 + t) for t in range(4))
+    scale = 0.3
+    out_d, lse_d = orc.decoder_train(q, ke, ve, k, v, S=S, scale=scale)
+    out_e, lse_e = orc.encoder(q, k, v, S=S, scale=scale)
+    for blk in range(L // S):
+        r = slice(blk * S, blk * S + S)
+        o, l = orc.decoder_sample(q[:, :, r], ke, ve, blk * S, k[:, :, r], v[:, :, r], scale=scale)
+        np.testing.assert_allclose(o, out_d[:, :, r], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l, lse_d[:, :, r], rtol=0, atol=1e-13)
+        o, l = orc.decoder_sample(q[:, :, r], k, v, blk * S, k[:, :, r], v[:, :, r], scale=scale)
+        np.testing.assert_allclose(o, out_e[:, :, r], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l, lse_e[:, :, r], rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------
+# 9. KV-cache append is array concatenation ([E2D2 notes, sec. 3]: the cache grows by the
+#    decoded block); rows outside [P, P+S_new) are untouched.
+# ---------------------------------------------------------------------------------------
+def pin_append_is_concatenation(orc):
+    B, Hkv, cap, d = 2, 3, 12, 8
+    rng = np.random.default_rng(990)
+    kc = rng.integers(0, 65535, size=(B, Hkv, cap, d), dtype=np.uint16)
+    vc = rng.integers(0, 65535, size=(B, Hkv, cap, d), dtype=np.uint16)
+    P = 0
+    kc0, vc0 = kc.copy(), vc.copy()
+    pieces_k, pieces_v = [], []
+    for S_new in (3, 4, 2):
+        kn = rng.integers(0, 65535, size=(B, Hkv, S_new, d), dtype=np.uint16)
+        vn = rng.integers(0, 65535, size=(B, Hkv, S_new, d), dtype=np.uint16)
+        orc.kv_append(kc, vc, P, kn, vn)
+        pieces_k.append(kn)
+        pieces_v.append(vn)
+        P += S_new
+    np.testing.assert_array_equal(kc[:, :, :P], np.concatenate(pieces_k, axis=2))
+    np.testing.assert_array_equal(vc[:, :, :P], np.concatenate(pieces_v, axis=2))
+    np.testing.assert_array_equal(kc[:, :, P:], kc0[:, :, P:])
+    np.testing.assert_array_equal(vc[:, :, P:], vc0[:, :, P:])
+
+
+ALL_PINS = [pin_pair_count, pin_golden_pairs, pin_block_size_one_is_causal,
+            pin_block_size_L_is_bidirectional, pin_masked_against_torch, pin_brute_force,
+            pin_zero_keys_closed_form, pin_constant_values, pin_gqa_is_repeated_heads,
+            pin_sample_is_train_slice, pin_append_is_concatenation]
