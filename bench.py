@@ -1,0 +1,445 @@
+#!/usr/bin/env python3
+"""Benchmark of the E2D2 fused block-diffusion attention on B200.
+
+One step = one pass of the whole hot path on one batch of synthetic input:
+  * E2D2 train pass (B8 L1024 S16 H16 d64): encoder block-causal attention + decoder-train fused
+    self+cross attention over 2L keys,
+  * E2D2 sampling step (B32 P2048 S16 Hq16 Hkv8 d128, shared KV cache): decoder-sample
+    split-KV attention + KV-cache append of the block.
+Headline `value`: useful TFLOP/s of the train-mask calls (masked pairs excluded), whole job.
+`sample_step` carries the HBM GB/s of the sampling call.  Per-kernel times come from CUDA events
+on the launching stream inside the timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+`--impl reference` times the CPU oracle (the only reference that exists for this path) on a
+bounded sample of the same workload.  Multi-GPU: one process per GPU (torchrun); every rank runs
+the same per-GPU workload (weak scaling, no data-path collective), times are max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "useful TFLOP/s (train mask) and HBM GB/s (sample step), % of B200 roofline"
+PEAKS_FILE = ROOT / "MEASURED_PEAKS.json"
+TRAFFIC_FILE = ROOT / "profiles" / "dram_traffic.json"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    try:
+        p = json.loads(PEAKS_FILE.read_text())
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted((ROOT / "block_discrete_diffusion_tcgen05_b200" / "csrc").glob("*")):
+        h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    try:
+        t = json.loads(TRAFFIC_FILE.read_text())
+    except Exception:
+        return None
+    if t.get("source_hash") != kernel_source_hash():
+        return None
+    k = t.get("kernels", {}).get(kernel)
+    return None if k is None else k.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons (nvidia-smi) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._thr = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.05)
+
+    def __enter__(self):
+        self._thr = threading.Thread(target=self._run, daemon=True)
+        self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._thr.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for n, v in zip(names, s[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------------------------
+def make_inputs(torch, dev, rank: int):
+    from block_discrete_diffusion_tcgen05_b200 import synth, workloads
+
+    def t(shape, wl, tensor, sigma):
+        a = synth.normal_bf16(shape, synth.seed_for(wl, rank, tensor), sigma)
+        return synth.to_torch(a, dev)
+
+    tw, sw = workloads.TRAIN, workloads.SAMPLE
+    shp = (tw.batch, tw.q_heads, tw.L, tw.head_dim)
+    train = {n: t(shp, 2, n, tw.sigma) for n in ("q", "k", "v", "k_enc", "v_enc", "k_dec", "v_dec")}
+    cap = sw.P + sw.S
+    sample = {
+        "q": t((sw.batch, sw.q_heads, sw.S, sw.head_dim), 3, "q", sw.sigma),
+        "k_cache": t((sw.batch, sw.kv_heads, cap, sw.head_dim), 3, "k_cache", sw.sigma),
+        "v_cache": t((sw.batch, sw.kv_heads, cap, sw.head_dim), 3, "v_cache", sw.sigma),
+        "k_blk": t((sw.batch, sw.kv_heads, sw.S, sw.head_dim), 3, "k_new", sw.sigma),
+        "v_blk": t((sw.batch, sw.kv_heads, sw.S, sw.head_dim), 3, "v_new", sw.sigma),
+    }
+    return train, sample
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from block_discrete_diffusion_tcgen05_b200 import attn, workloads
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    tw, sw = workloads.TRAIN, workloads.SAMPLE
+    train, sample = make_inputs(torch, dev, rank)
+    S = tw.S
+    out_e = torch.empty_like(train["q"])
+    out_d = torch.empty_like(train["q"])
+    lse_e = torch.empty(train["q"].shape[:3], dtype=torch.float32, device=dev)
+    lse_d = torch.empty_like(lse_e)
+    out_s = torch.empty_like(sample["q"])
+    lse_s = torch.empty(sample["q"].shape[:3], dtype=torch.float32, device=dev)
+    ws = attn.sample_workspace(sample["q"], sample["k_cache"])
+    P = sw.P
+
+    def enc():
+        attn.encoder_blockcausal(train["q"], train["k"], train["v"], S, out=out_e, lse=lse_e)
+
+    def dec():
+        attn.decoder_train(train["q"], train["k_enc"], train["v_enc"], train["k_dec"], train["v_dec"], S,
+                           out=out_d, lse=lse_d)
+
+    def smp():
+        attn.decoder_sample(sample["q"], sample["k_cache"], sample["v_cache"], P, sample["k_blk"],
+                            sample["v_blk"], workspace=ws, out=out_s, lse=lse_s)
+
+    def app():
+        # The decoded block joins the cache at row P (the next step would read P + S rows;
+        # the benchmark keeps P fixed so every step is the same work).
+        attn.kv_cache_append(sample["k_cache"], sample["v_cache"], P, sample["k_blk"], sample["v_blk"])
+
+    kernels = [("encoder", enc), ("decoder_train", dec), ("decoder_sample", smp), ("kv_append", app)]
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        for _, f in kernels:
+            f()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+          for n, _ in kernels}
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_start.record(stream)
+        for i in range(K):
+            for n, f in kernels:
+                a, b = ev[n][i]
+                a.record(stream)
+                f()
+                b.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total_ms = t_start.elapsed_time(t_end)
+    per_kernel_ms = {n: sum(a.elapsed_time(b) for a, b in ev[n]) for n, _ in kernels}
+    launches = K * len(kernels)
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    total_ms = max_over_ranks(total_ms)
+    per_kernel_ms = {n: max_over_ranks(v) for n, v in per_kernel_ms.items()}
+
+    # ---- metrics -------------------------------------------------------------------------
+    peaks, peak_kind = load_peaks()
+    fl_train = workloads.useful_flops_train(tw)  # per call (encoder or decoder pass)
+    train_ms = per_kernel_ms["encoder"] + per_kernel_ms["decoder_train"]
+    value = (2 * fl_train * K * world) / (train_ms * 1e-3) / 1e12
+    by_enc = workloads.bytes_train(tw, decoder=False)
+    by_dec = workloads.bytes_train(tw, decoder=True)
+    by_smp = workloads.bytes_sample(sw)
+    smp_s = per_kernel_ms["decoder_sample"] * 1e-3
+    sample_gbs = by_smp * K * world / smp_s / 1e9
+
+    # dominant kernel by device time
+    dom = max(("encoder", "decoder_train", "decoder_sample"), key=lambda n: per_kernel_ms[n])
+    avg_s = per_kernel_ms[dom] * 1e-3 / K
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"])
+    ridge = tc_peak * 1e12 / (hbm_peak * 1e9)
+    if dom == "decoder_sample":
+        alg_bytes, alg_flops = by_smp, workloads.useful_flops_sample(sw)
+    else:
+        alg_bytes, alg_flops = (by_enc if dom == "encoder" else by_dec), fl_train
+    if alg_flops / alg_bytes >= ridge:
+        roof = {"bound": "tensor", "achieved": alg_flops / avg_s / 1e12, "peak": tc_peak, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": alg_bytes / avg_s / 1e9, "peak": hbm_peak, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == "measured" else "fallback"
+    roof["traffic"] = traffic_for(dom)
+    roof["avg_launch_us"] = avg_s * 1e6
+    roof["algorithmic"] = {"flops": alg_flops, "bytes": alg_bytes}
+
+    kern_detail = {}
+    for n, fl, by in (("encoder", fl_train, by_enc), ("decoder_train", fl_train, by_dec),
+                      ("decoder_sample", workloads.useful_flops_sample(sw), by_smp)):
+        s = per_kernel_ms[n] * 1e-3 / K
+        kern_detail[n] = {"avg_us": s * 1e6, "useful_tflops": fl / s / 1e12, "gbs": by / s / 1e9,
+                          "frac_tensor": fl / s / 1e12 / tc_peak, "frac_hbm": by / s / 1e9 / hbm_peak,
+                          "frac_attainable": (fl / s) / min(tc_peak * 1e12, fl / by * hbm_peak * 1e9)}
+    kern_detail["kv_append"] = {"avg_us": per_kernel_ms["kv_append"] * 1e3 / K}
+
+    # ---- e2e: the same train metric through the public API with host buffers --------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(torch, attn, workloads, train, dev, args, dist, world)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0, sigma^2) rounded to bf16)",
+        "config": {"workload": "E2D2 train pass B8 L1024 S16 H16 d64 (encoder + decoder-train) "
+                               "+ E2D2 sampling step B32 P2048 S16 Hq16 Hkv8 d128 (+ KV append)",
+                   "global_batch": 8 * world, "seq_len": 1024, "parallelism": f"dp{world} (replicas, no collective)",
+                   "l2": "not flushed: each step touches ~0.45 GB (> 126 MB L2), so every kernel's inputs are cold"},
+        "sample_step": {"value": sample_gbs, "unit": "GB/s", "frac_hbm": sample_gbs / world / hbm_peak,
+                        "avg_us": kern_detail["decoder_sample"]["avg_us"]},
+        "kernels": kern_detail,
+        "roofline": roof,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(torch, attn, workloads, train, dev, args, dist, world):
+    """Train metric end to end: per step, H2D of every input from pinned host memory, both
+    train-pass calls, D2H of both outputs and LSEs."""
+    host_in = {n: t.cpu().pin_memory() for n, t in train.items()}
+    dev_in = {n: torch.empty_like(t) for n, t in train.items()}
+    tw = workloads.TRAIN
+    S = tw.S
+    outs = [torch.empty_like(train["q"]) for _ in range(2)]
+    lses = [torch.empty(train["q"].shape[:3], dtype=torch.float32, device=dev) for _ in range(2)]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    host_lse = [torch.empty(l.shape, dtype=l.dtype).pin_memory() for l in lses]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for n in dev_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        attn.encoder_blockcausal(dev_in["q"], dev_in["k"], dev_in["v"], S, out=outs[0], lse=lses[0])
+        attn.decoder_train(dev_in["q"], dev_in["k_enc"], dev_in["v_enc"], dev_in["k_dec"], dev_in["v_dec"], S,
+                           out=outs[1], lse=lses[1])
+        for o, ho in zip(outs, host_out):
+            ho.copy_(o, non_blocking=True)
+        for l, hl in zip(lses, host_lse):
+            hl.copy_(l, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.e2e_steps, args.steps))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    fl = 2 * workloads.useful_flops_train(tw)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out + host_lse)
+    return {"value": fl * n * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n}
+
+
+# --------------------------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# --------------------------------------------------------------------------------------------
+def oracle_train_sample(budget_s: float):
+    """Times the oracle on a bounded sample of the train pass: all 16 heads of as many batch
+    entries as fit the budget (heads are independent, so useful FLOPs scale exactly)."""
+    import numpy as np
+
+    import oracle
+    from block_discrete_diffusion_tcgen05_b200 import synth, workloads
+
+    orc = oracle.default()
+    tw = workloads.TRAIN
+    shp = (1, tw.q_heads, tw.L, tw.head_dim)
+    gen = lambda n: synth.normal_bf16(shp, synth.seed_for(2, 0, n), tw.sigma).f32
+    q, k, v, ke, ve = (gen(n) for n in ("q", "k", "v", "k_enc", "v_enc"))
+    done_b, t_total = 0, 0.0
+    while done_b < tw.batch:
+        t0 = time.perf_counter()
+        orc.encoder(q, k, v, tw.S)
+        orc.decoder_train(q, ke, ve, k, v, tw.S)
+        t_total += time.perf_counter() - t0
+        done_b += 1
+        if t_total * (done_b + 1) / done_b > budget_s:
+            break
+    pairs = workloads.unmasked_pairs(tw.L, tw.S)
+    flops = 2 * 4 * tw.head_dim * tw.q_heads * done_b * pairs
+    return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"E2D2 train pass, encoder + decoder-train, {done_b} of {tw.batch} batch entries "
+                      f"x {tw.q_heads} heads (L1024 S16 d64), fp64, {t_total:.1f} s",
+            "seconds": t_total}
+
+
+def cpu_baseline(budget_s: float):
+    try:
+        return oracle_train_sample(budget_s)
+    except Exception as exc:  # the baseline is reported, never required
+        return {"value": None, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                "sample": f"failed: {exc}"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    t0 = time.perf_counter()
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_train_sample(args.ref_step_budget)
+        if i >= args.warmup:
+            per_step.append(r)
+    vals = [r["value"] for r in per_step]
+    value = statistics.mean(vals)
+    secs = sum(r["seconds"] for r in per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / max(1, len(per_step)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0, sigma^2) rounded to bf16)",
+        "config": {"workload": "E2D2 train pass B8 L1024 S16 H16 d64 (encoder + decoder-train), "
+                               "CPU oracle on a bounded sample", "global_batch": 8, "seq_len": 1024,
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": per_step[0]["cores"], "kind": "oracle",
+                         "sample": per_step[0]["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-step-budget", type=float, default=8.0, help="seconds of oracle work per reference step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"note: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,141 @@
+"""Python front-end of the E2D2 attention C ABI, taking torch tensors.
+
+Argument marshalling only: every step of the attention runs in the CUDA kernels of
+``libe2d2_attn.so``.  PyTorch provides device memory and the stream (the current stream of
+the tensors' device).  Names follow the C ABI (include/e2d2_attn.h)."""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _lib
+
+_BF16 = torch.bfloat16
+
+
+def _dims(batch, q_heads, kv_heads, head_dim, scale):
+    return _lib.Dims(batch, q_heads, kv_heads, head_dim, 0.0 if scale is None else float(scale))
+
+
+def _need(t: torch.Tensor, name: str, dtype=_BF16, ndim=4):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(t: torch.Tensor):
+    return ctypes_stream(torch.cuda.current_stream(t.device))
+
+
+def ctypes_stream(s: torch.cuda.Stream):
+    return s.cuda_stream
+
+
+def encoder_blockcausal(q, k, v, S: int, scale=None, out=None, lse=True):
+    """Block-causal encoder self-attention.  q [B,Hq,L,d], k/v [B,Hkv,L,d] (bf16, CUDA).
+    Returns (out [B,Hq,L,d] bf16, lse [B,Hq,L] fp32 or None)."""
+    lib = _lib.load()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, L, d) or v.shape != k.shape:
+        raise ValueError("k/v must be [B, Hkv, L, d] matching q")
+    out = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device) if lse is True else lse
+    st = lib.e2d2_attn_encoder_blockcausal(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                           None if lse_t is None or lse_t is False else lse_t.data_ptr(),
+                                           _dims(B, Hq, Hkv, d, scale), L, S, _stream(q))
+    _lib.check(st, "e2d2_attn_encoder_blockcausal")
+    return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
+
+
+def decoder_train(q, k_enc, v_enc, k_dec, v_dec, S: int, scale=None, out=None, lse=True):
+    """Decoder fused self+cross attention (training mode) over 2L keys."""
+    lib = _lib.load()
+    for t, n in ((q, "q"), (k_enc, "k_enc"), (v_enc, "v_enc"), (k_dec, "k_dec"), (v_dec, "v_dec")):
+        _need(t, n)
+    B, Hq, L, d = q.shape
+    Hkv = k_enc.shape[1]
+    for t in (k_enc, v_enc, k_dec, v_dec):
+        if t.shape != (B, Hkv, L, d):
+            raise ValueError("k_enc/v_enc/k_dec/v_dec must be [B, Hkv, L, d] matching q")
+    out = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device) if lse is True else lse
+    st = lib.e2d2_attn_decoder_train(q.data_ptr(), k_enc.data_ptr(), v_enc.data_ptr(), k_dec.data_ptr(),
+                                     v_dec.data_ptr(), out.data_ptr(),
+                                     None if lse_t is None or lse_t is False else lse_t.data_ptr(),
+                                     _dims(B, Hq, Hkv, d, scale), L, S, _stream(q))
+    _lib.check(st, "e2d2_attn_decoder_train")
+    return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
+
+
+def sample_workspace_bytes(batch, q_heads, kv_heads, head_dim, S, capacity) -> int:
+    lib = _lib.load()
+    return int(lib.e2d2_attn_decoder_sample_workspace(_dims(batch, q_heads, kv_heads, head_dim, None),
+                                                      S, capacity))
+
+
+def sample_workspace(q_blk: torch.Tensor, k_cache: torch.Tensor) -> torch.Tensor:
+    """A zero-filled workspace for decoder_sample with these shapes."""
+    B, Hq, S, d = q_blk.shape
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    n = sample_workspace_bytes(B, Hq, Hkv, d, S, cap)
+    return torch.zeros(n, dtype=torch.uint8, device=q_blk.device)
+
+
+def decoder_sample(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=None, scale=None,
+                   out=None, lse=True):
+    """Decoder sampling step over the cached prefix k_cache[:, :, :P] plus the own block."""
+    lib = _lib.load()
+    for t, n in ((q_blk, "q_blk"), (k_cache, "k_cache"), (v_cache, "v_cache"), (k_blk, "k_blk"),
+                 (v_blk, "v_blk")):
+        _need(t, n)
+    B, Hq, S, d = q_blk.shape
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, cap, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [B, Hkv, capacity, d]")
+    if k_blk.shape != (B, Hkv, S, d) or v_blk.shape != k_blk.shape:
+        raise ValueError("k_blk/v_blk must be [B, Hkv, S, d]")
+    ws = sample_workspace(q_blk, k_cache) if workspace is None else workspace
+    out = torch.empty_like(q_blk) if out is None else out
+    lse_t = torch.empty((B, Hq, S), dtype=torch.float32, device=q_blk.device) if lse is True else lse
+    st = lib.e2d2_attn_decoder_sample(q_blk.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cap, int(P),
+                                      k_blk.data_ptr(), v_blk.data_ptr(), out.data_ptr(),
+                                      None if lse_t is None or lse_t is False else lse_t.data_ptr(),
+                                      _dims(B, Hq, Hkv, d, scale), S, ws.data_ptr(),
+                                      ws.numel() * ws.element_size(), _stream(q_blk))
+    _lib.check(st, "e2d2_attn_decoder_sample")
+    return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
+
+
+def kv_cache_append(k_cache, v_cache, P: int, k_new, v_new):
+    """Writes k_new/v_new [B,Hkv,S_new,d] into rows P..P+S_new-1 of the caches; returns P+S_new."""
+    lib = _lib.load()
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (k_new, "k_new"), (v_new, "v_new")):
+        _need(t, n)
+    B, Hkv, cap, d = k_cache.shape
+    S_new = k_new.shape[2]
+    if k_new.shape != (B, Hkv, S_new, d) or v_new.shape != k_new.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    st = lib.e2d2_kv_cache_append(k_cache.data_ptr(), v_cache.data_ptr(), cap, int(P), k_new.data_ptr(),
+                                  v_new.data_ptr(), S_new, _dims(B, Hkv, Hkv, d, None), _stream(k_cache))
+    _lib.check(st, "e2d2_kv_cache_append")
+    return P + S_new
+
+
+def last_device_error(device=None) -> int:
+    lib = _lib.load()
+    return int(lib.e2d2_last_device_error(torch.cuda.current_stream(device).cuda_stream))
+
+
+def default_scale(head_dim: int) -> float:
+    return 1.0 / math.sqrt(head_dim)

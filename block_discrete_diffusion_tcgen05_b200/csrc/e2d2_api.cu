@@ -1,0 +1,359 @@
+// e2d2_api.cu -- host side of the C ABI declared in include/e2d2_attn.h: argument validation,
+// TMA tensor-map encoding, grid choice and kernel launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "e2d2_attn.h"
+#include "fmha_sm100.cuh"
+#include "kv_append.cuh"
+
+namespace e2d2 {
+
+__device__ unsigned int g_error_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool supported = false;
+    int sms = 0;
+    unsigned int* err = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+e2d2_status device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return E2D2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return E2D2_ERR_CUDA;
+        d.supported = (prop.major == 10);
+        d.sms = prop.multiProcessorCount;
+        void* sym = nullptr;
+        if (cudaGetSymbolAddress(&sym, g_error_word) != cudaSuccess) return E2D2_ERR_CUDA;
+        d.err = static_cast<unsigned int*>(sym);
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return E2D2_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        d.ready = true;
+    }
+    if (!d.supported) return E2D2_ERR_UNSUPPORTED;
+    *out = &d;
+    return E2D2_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+e2d2_status check_dims(const e2d2_dims& dm) {
+    if (dm.batch <= 0 || dm.q_heads <= 0 || dm.kv_heads <= 0 || dm.head_dim <= 0)
+        return E2D2_ERR_INVALID_ARG;
+    if (dm.q_heads % dm.kv_heads != 0) return E2D2_ERR_INVALID_ARG;
+    if (dm.head_dim != 32 && dm.head_dim != 64 && dm.head_dim != 128) return E2D2_ERR_UNSUPPORTED;
+    if (!std::isfinite(dm.scale)) return E2D2_ERR_INVALID_ARG;
+    return E2D2_OK;
+}
+
+float scale_log2(const e2d2_dims& dm) {
+    const double s = dm.scale > 0.f ? static_cast<double>(dm.scale) : 1.0 / std::sqrt((double)dm.head_dim);
+    return static_cast<float>(s * 1.4426950408889634);
+}
+
+// bf16 tensor [units][rows][D] (unit stride `unit_rows` rows), boxes of {min(D,64), box_rows, 1}.
+bool map_3d(CUtensorMap* m, const void* base, int D, long long rows, long long units,
+            long long unit_rows, int box_rows) {
+    const int rb = (D * 2 < 128) ? D * 2 : 128;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(units)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                             static_cast<cuuint64_t>(unit_rows) * D * 2};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(rb / 2), static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool map_2d(CUtensorMap* m, const void* base, int D, long long rows, int box_rows) {
+    const int rb = (D * 2 < 128) ? D * 2 : 128;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(rb / 2), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int MODE>
+e2d2_status launch_fmha(const FmhaParams& prm, int grid, cudaStream_t st) {
+    using SM = Smem<D, MODE>;
+    static_assert(SM::ALLOC <= 232448, "shared memory budget");
+    auto kern = fmha_sm100_kernel<D, MODE>;
+    // Ask for at least ~116 KB so that two CTAs never share an SM (each takes all of TMEM).
+    const int smem = SM::ALLOC > 118784 ? SM::ALLOC : 118784;
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return E2D2_ERR_CUDA;
+        configured_dev = dev;
+    }
+    kern<<<grid, kThreads, smem, st>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+}
+
+template <int MODE>
+e2d2_status dispatch_fmha(int D, const FmhaParams& prm, int grid, cudaStream_t st) {
+    switch (D) {
+        case 32: return launch_fmha<32, MODE>(prm, grid, st);
+        case 64: return launch_fmha<64, MODE>(prm, grid, st);
+        case 128: return launch_fmha<128, MODE>(prm, grid, st);
+        default: return E2D2_ERR_UNSUPPORTED;
+    }
+}
+
+constexpr long long kMaxI32 = 0x7fffffffLL;
+
+e2d2_status check_train_shape(const e2d2_dims& dm, int L, int S) {
+    if (L <= 0 || S <= 0) return E2D2_ERR_INVALID_ARG;
+    if (S > L || L % S != 0) return E2D2_ERR_SHAPE;
+    const long long rows = static_cast<long long>(dm.batch) * dm.q_heads * L;
+    if (rows > kMaxI32 / 8) return E2D2_ERR_SHAPE;
+    return E2D2_OK;
+}
+
+e2d2_status train_common(int mode, const void* q, const void* k0, const void* v0, const void* k1,
+                         const void* v1, void* out, float* lse, const e2d2_dims& dm, int L, int S,
+                         cudaStream_t st) {
+    e2d2_status s = check_dims(dm);
+    if (s != E2D2_OK) return s;
+    s = check_train_shape(dm, L, S);
+    if (s != E2D2_OK) return s;
+    if (!aligned16(q) || !aligned16(k0) || !aligned16(v0) || !aligned16(out) ||
+        (k1 && !aligned16(k1)) || (v1 && !aligned16(v1)) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return E2D2_ERR_ALIGNMENT;
+    DeviceInfo* di = nullptr;
+    s = device_info(&di);
+    if (s != E2D2_OK) return s;
+
+    const int D = dm.head_dim;
+    FmhaParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    const long long BHq = static_cast<long long>(dm.batch) * dm.q_heads;
+    const long long BHkv = static_cast<long long>(dm.batch) * dm.kv_heads;
+    bool ok = map_3d(&prm.tm_q, q, D, L, BHq, L, kBlockM) && map_3d(&prm.tm_o, out, D, L, BHq, L, kBlockM) &&
+              map_3d(&prm.tm_k0, k0, D, L, BHkv, L, kBlockN) && map_3d(&prm.tm_v0, v0, D, L, BHkv, L, kBlockN);
+    if (mode == kDecoderTrain)
+        ok = ok && map_3d(&prm.tm_k1, k1, D, L, BHkv, L, kBlockN) && map_3d(&prm.tm_v1, v1, D, L, BHkv, L, kBlockN);
+    if (!ok) return E2D2_ERR_CUDA;
+    prm.out = out;
+    prm.lse = lse;
+    prm.err = di->err;
+    prm.batch = dm.batch;
+    prm.q_heads = dm.q_heads;
+    prm.kv_heads = dm.kv_heads;
+    prm.group = dm.q_heads / dm.kv_heads;
+    prm.L = L;
+    prm.S = S;
+    prm.box1_rows = kBlockN;
+    prm.scale_log2 = scale_log2(dm);
+    prm.num_qtiles = (L + kBlockM - 1) / kBlockM;
+    prm.num_items = static_cast<int>(BHq * prm.num_qtiles);
+    const int grid = prm.num_items < di->sms ? prm.num_items : di->sms;
+    return mode == kEncoder ? dispatch_fmha<kEncoder>(D, prm, grid, st)
+                            : dispatch_fmha<kDecoderTrain>(D, prm, grid, st);
+}
+
+struct SampleLayout {
+    int rows_cap;
+    int slot_floats;
+    size_t bytes;
+};
+
+SampleLayout sample_layout(const e2d2_dims& dm, int S) {
+    SampleLayout w;
+    const long long rows = static_cast<long long>(dm.q_heads / dm.kv_heads) * S;
+    w.rows_cap = static_cast<int>(rows < kBlockM ? rows : kBlockM);
+    const long long f = static_cast<long long>(w.rows_cap) * (dm.head_dim + 2);
+    w.slot_floats = static_cast<int>((f + 63) / 64 * 64);
+    w.bytes = 1024 + static_cast<size_t>(2) * kSampleMaxCtas * w.slot_floats * sizeof(float);
+    return w;
+}
+
+}  // namespace
+}  // namespace e2d2
+
+using namespace e2d2;
+
+extern "C" {
+
+const char* e2d2_status_string(e2d2_status s) {
+    switch (s) {
+        case E2D2_OK: return "E2D2_OK";
+        case E2D2_ERR_INVALID_ARG: return "E2D2_ERR_INVALID_ARG";
+        case E2D2_ERR_UNSUPPORTED: return "E2D2_ERR_UNSUPPORTED";
+        case E2D2_ERR_SHAPE: return "E2D2_ERR_SHAPE";
+        case E2D2_ERR_ALIGNMENT: return "E2D2_ERR_ALIGNMENT";
+        case E2D2_ERR_CAPACITY: return "E2D2_ERR_CAPACITY";
+        case E2D2_ERR_WORKSPACE: return "E2D2_ERR_WORKSPACE";
+        case E2D2_ERR_CUDA: return "E2D2_ERR_CUDA";
+        case E2D2_ERR_TIMEOUT: return "E2D2_ERR_TIMEOUT";
+    }
+    return "E2D2_ERR_UNKNOWN";
+}
+
+int e2d2_version(void) { return 100; }
+
+e2d2_status e2d2_attn_encoder_blockcausal(const void* q, const void* k, const void* v, void* out,
+                                          float* lse, e2d2_dims dims, int L, int S,
+                                          cudaStream_t stream) {
+    if (!q || !k || !v || !out) return E2D2_ERR_INVALID_ARG;
+    return train_common(kEncoder, q, k, v, nullptr, nullptr, out, lse, dims, L, S, stream);
+}
+
+e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_enc, const void* v_enc,
+                                    const void* k_dec, const void* v_dec, void* out, float* lse,
+                                    e2d2_dims dims, int L, int S, cudaStream_t stream) {
+    if (!q_dec || !k_enc || !v_enc || !k_dec || !v_dec || !out) return E2D2_ERR_INVALID_ARG;
+    return train_common(kDecoderTrain, q_dec, k_enc, v_enc, k_dec, v_dec, out, lse, dims, L, S, stream);
+}
+
+size_t e2d2_attn_decoder_sample_workspace(e2d2_dims dims, int S, int capacity) {
+    if (check_dims(dims) != E2D2_OK || S <= 0 || capacity < 0) return 0;
+    return sample_layout(dims, S).bytes;
+}
+
+e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, const void* v_cache,
+                                     int capacity, int P, const void* k_blk, const void* v_blk,
+                                     void* out, float* lse, e2d2_dims dims, int S, void* workspace,
+                                     size_t ws_bytes, cudaStream_t stream) {
+    if (!q_blk || !k_cache || !v_cache || !k_blk || !v_blk || !out) return E2D2_ERR_INVALID_ARG;
+    e2d2_status s = check_dims(dims);
+    if (s != E2D2_OK) return s;
+    if (S <= 0 || capacity < 0 || P < 0) return E2D2_ERR_INVALID_ARG;
+    if (P > capacity) return E2D2_ERR_CAPACITY;
+    const long long rows = static_cast<long long>(dims.batch) * dims.q_heads * S;
+    if (rows > kMaxI32 / 8 || static_cast<long long>(capacity) * dims.batch * dims.kv_heads > kMaxI32)
+        return E2D2_ERR_SHAPE;
+    if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_blk) ||
+        !aligned16(v_blk) || !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return E2D2_ERR_ALIGNMENT;
+    const SampleLayout w = sample_layout(dims, S);
+    if (!workspace || ws_bytes < w.bytes) return E2D2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return E2D2_ERR_ALIGNMENT;
+    DeviceInfo* di = nullptr;
+    s = device_info(&di);
+    if (s != E2D2_OK) return s;
+
+    const int D = dims.head_dim;
+    const int G = dims.q_heads / dims.kv_heads;
+    FmhaParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    const long long BHkv = static_cast<long long>(dims.batch) * dims.kv_heads;
+    const int S16 = (S + 15) / 16 * 16;
+    const int box1 = S16 < kBlockN ? S16 : kBlockN;
+    bool ok = map_2d(&prm.tm_q, q_blk, D, rows, kBlockM) &&
+              map_3d(&prm.tm_k0, k_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
+              map_3d(&prm.tm_v0, v_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
+              map_3d(&prm.tm_k1, k_blk, D, S, BHkv, S, box1) && map_3d(&prm.tm_v1, v_blk, D, S, BHkv, S, box1);
+    if (!ok) return E2D2_ERR_CUDA;
+    prm.out = out;
+    prm.lse = lse;
+    prm.ws_tickets = static_cast<int*>(workspace);
+    prm.ws_partial = reinterpret_cast<float*>(static_cast<char*>(workspace) + 1024);
+    prm.err = di->err;
+    prm.batch = dims.batch;
+    prm.q_heads = dims.q_heads;
+    prm.kv_heads = dims.kv_heads;
+    prm.group = G;
+    prm.L = S;
+    prm.S = S;
+    prm.P = P;
+    prm.box1_rows = box1;
+    prm.scale_log2 = scale_log2(dims);
+    prm.rows_per_unit = G * S;
+    prm.num_qtiles = (G * S + kBlockM - 1) / kBlockM;
+    prm.tiles_per_unit = (S + kBlockN - 1) / kBlockN + (P + kBlockN - 1) / kBlockN;
+    prm.total_tiles = BHkv * prm.num_qtiles * static_cast<long long>(prm.tiles_per_unit);
+    prm.rows_cap = w.rows_cap;
+    prm.slot_floats = w.slot_floats;
+    long long grid = di->sms < kSampleMaxCtas ? di->sms : kSampleMaxCtas;
+    if (grid > prm.total_tiles) grid = prm.total_tiles;
+    return dispatch_fmha<kDecoderSample>(D, prm, static_cast<int>(grid), stream);
+}
+
+e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int P, const void* k_new,
+                                 const void* v_new, int S_new, e2d2_dims dims, cudaStream_t stream) {
+    if (!k_cache || !v_cache || !k_new || !v_new) return E2D2_ERR_INVALID_ARG;
+    e2d2_status s = check_dims(dims);
+    if (s != E2D2_OK) return s;
+    if (P < 0 || S_new < 0 || capacity < 0) return E2D2_ERR_INVALID_ARG;
+    if (static_cast<long long>(P) + S_new > capacity) return E2D2_ERR_CAPACITY;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new))
+        return E2D2_ERR_ALIGNMENT;
+    if (S_new == 0) return E2D2_OK;
+    DeviceInfo* di = nullptr;
+    s = device_info(&di);
+    if (s != E2D2_OK) return s;
+    AppendParams a;
+    a.cache[0] = static_cast<uint4*>(k_cache);
+    a.cache[1] = static_cast<uint4*>(v_cache);
+    a.src[0] = static_cast<const uint4*>(k_new);
+    a.src[1] = static_cast<const uint4*>(v_new);
+    a.capacity = capacity;
+    a.P = P;
+    a.S_new = S_new;
+    a.vec_per_row = dims.head_dim / 8;
+    a.units = dims.batch * dims.kv_heads;
+    const long long total = static_cast<long long>(a.units) * S_new * a.vec_per_row;
+    long long blocks = (total + 255) / 256;
+    const long long cap_blocks = static_cast<long long>(di->sms) * 8;
+    if (blocks > cap_blocks) blocks = cap_blocks;
+    kv_append_kernel<<<dim3(static_cast<unsigned>(blocks), 2), 256, 0, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+}
+
+e2d2_status e2d2_last_device_error(cudaStream_t stream) {
+    DeviceInfo* di = nullptr;
+    e2d2_status s = device_info(&di);
+    if (s != E2D2_OK) return s;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return E2D2_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return E2D2_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return E2D2_ERR_CUDA;
+        return E2D2_ERR_TIMEOUT;
+    }
+    return E2D2_OK;
+}
+
+}  // extern "C"

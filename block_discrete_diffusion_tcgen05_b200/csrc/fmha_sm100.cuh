@@ -1,0 +1,763 @@
+// fmha_sm100.cuh -- persistent, warp-specialised flash attention for B200 (sm_100a) that
+// computes the three E2D2 attention calls:
+//
+//   kEncoder        block-causal self-attention over clean tokens: query i sees keys j with
+//                   floor(j/S) <= floor(i/S)  ("Encoder-Decoder Diffusion Language Models for
+//                   Efficient Training and Inference", paper notes, sec. 4).
+//   kDecoderTrain   fused self+cross attention over 2L keys: encoder-side keys of the blocks
+//                   strictly before the query's block, decoder-side keys of its own block
+//                   (same page, sec. 2 and 4).
+//   kDecoderSample  sampling step: the S noised queries of one block (G = Hq/Hkv heads packed
+//                   into the rows of one tile) against the cached clean prefix (P keys) and
+//                   their own block (same page, sec. 3), split over CTAs stream-K style.
+//
+// Every row's allowed keys form, per key source, one interval [lo, hi), so the mask is
+// computed from tile indices and row numbers; key tiles outside every row's interval are
+// never loaded, and no mask matrix exists anywhere.
+//
+// CTA = 6 warps: warp 0 issues TMA loads, warp 1 owns tensor memory and issues tcgen05.mma,
+// warps 2..5 (one per TMEM lane quarter) run the online softmax and the epilogue.  One
+// 128-row query tile per work item; per key tile of up to 128 keys:
+//     S  = Q K^T        tcgen05.mma, A = Q (smem), B = K (smem, K-major)  -> TMEM (fp32)
+//     P  = exp2(S*c - m) softmax warps, written back over S as bf16      -> TMEM
+//     O += P V          tcgen05.mma, A = P (TMEM), B = V (smem, MN-major) -> TMEM (fp32)
+// S is double-buffered in TMEM so QK^T of tile j+1 overlaps the softmax of tile j; O is
+// double-buffered across work items so the epilogue of one item overlaps the next item.
+// The running max is only moved when it grows by more than 2^8 (log2 units), so O is
+// rescaled rarely; the final normalisation uses the same max and is exact.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx_sm100.cuh"
+
+namespace e2d2 {
+
+enum Mode : int { kEncoder = 0, kDecoderTrain = 1, kDecoderSample = 2 };
+
+constexpr int kBlockM = 128;            // query rows per tile (TMEM lanes)
+constexpr int kBlockN = 128;            // keys per tile
+constexpr int kThreads = 192;           // 6 warps
+constexpr int kSoftmaxThreads = 128;    // warps 2..5
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr int kSampleMaxCtas = 256;     // upper bound of the sampling grid (workspace sizing)
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
+
+// Bit set in the device error word when a bounded wait gives up.
+constexpr unsigned int kErrWaitTimeout = 1u;
+
+struct alignas(64) FmhaParams {
+    CUtensorMap tm_q;   // kEncoder/kDecoderTrain: 3D {D, L, B*Hq}; kDecoderSample: 2D {D, B*Hq*S}
+    CUtensorMap tm_k0;  // source 0: encoder self K | decoder-train encoder-side K | sample cache K
+    CUtensorMap tm_v0;
+    CUtensorMap tm_k1;  // source 1: decoder-train decoder-side K | sample own-block K
+    CUtensorMap tm_v1;
+    CUtensorMap tm_o;   // train modes: 3D {D, L, B*Hq} (TMA store)
+    void* out;          // kDecoderSample output, bf16 [B][Hq][S][D]
+    float* lse;         // nullable
+    float* ws_partial;  // kDecoderSample: split partial slots
+    int* ws_tickets;    // kDecoderSample: one ticket word per CTA
+    unsigned int* err;  // device error word
+    int batch, q_heads, kv_heads, group;
+    int L;              // train: sequence length
+    int S;              // block size
+    int P;              // sample: cached prefix length
+    int box1_rows;      // rows of one source-1 TMA box
+    float scale_log2;   // softmax scale * log2(e)
+    int num_items;      // train: (head, query tile) items
+    int num_qtiles;     // train: query tiles per head; sample: query tiles per (b, kv head)
+    int rows_per_unit;  // sample: G * S packed query rows per (b, kv head)
+    int tiles_per_unit; // sample: key tiles per unit
+    long long total_tiles;  // sample: units * tiles_per_unit
+    int slot_floats;    // sample: floats per partial slot
+    int rows_cap;       // sample: rows stored per partial slot
+};
+
+// A unit of work: one 128-row query tile against a contiguous range of its key tiles.
+struct Item {
+    int q_z;        // train: b*Hq + h (Q/O tensor-map z); sample: unit index
+    int kv_z;       // b*Hkv + g
+    int q_row0;     // train: first row within the head; sample: first packed row within the unit
+    int q_y;        // TMA y coordinate of the query tile
+    int out_row0;   // sample: first row of this tile in the [B*Hq*S] row space
+    int n1, a1;     // source-1 tiles (visited first), starting at key tile a1
+    int n0;         // source-0 tiles, starting at key tile 0
+    int t_begin, t_end;
+};
+
+template <int D>
+struct Cfg {
+    static constexpr int RB = (D * 2 < 128) ? D * 2 : 128;  // bytes per smem row of one chunk
+    static constexpr int NCH = D * 2 / RB;                   // column chunks per tile
+    static constexpr uint32_t SWZ = (RB == 128) ? 2u : 4u;   // 128-byte / 64-byte swizzle
+    static constexpr int CHUNK_BYTES = kBlockM * RB;
+    static constexpr int TILE_BYTES = kBlockM * D * 2;
+    static constexpr int NST = (D == 128) ? 2 : (D == 64 ? 4 : 6);
+    static constexpr int KSTEPS_PER_CHUNK = RB / 32;         // 16-element k steps per chunk
+};
+
+template <int D, int MODE>
+struct Smem {
+    using C = Cfg<D>;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + 2 * C::TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + C::NST * C::TILE_BYTES;
+    static constexpr int OFF_O = OFF_V + C::NST * C::TILE_BYTES;
+    static constexpr int O_BYTES = (MODE == kDecoderSample) ? 0 : C::TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_O + O_BYTES;
+    // barriers: k_full[NST], v_full[NST], kv_empty[NST], q_full[2], q_empty[2], s_full[2],
+    // p_full[2], o_free[2], pv_done, mma_drain
+    static constexpr int NBAR = 3 * C::NST + 2 * 5 + 2;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int BYTES = OFF_MISC + 64;
+    static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
+
+// Largest CTA c whose stream-K range [c*T/G, (c+1)*T/G) starts at or before tile x.
+__device__ __forceinline__ int owner_cta(long long x, long long T, int grid) {
+    return static_cast<int>(((x + 1) * grid - 1) / T);
+}
+__device__ __forceinline__ long long range_begin(int c, long long T, int grid) {
+    return (static_cast<long long>(c) * T) / grid;
+}
+
+// Iterates the work items of this CTA.  Every role walks the same sequence.
+template <int MODE>
+struct Scheduler {
+    const FmhaParams& p;
+    long long pos, end;  // sample: tile range of this CTA
+    int k;               // train: next item index
+
+    __device__ Scheduler(const FmhaParams& prm) : p(prm) {
+        if (MODE == kDecoderSample) {
+            pos = range_begin(blockIdx.x, p.total_tiles, gridDim.x);
+            end = range_begin(blockIdx.x + 1, p.total_tiles, gridDim.x);
+        } else {
+            k = blockIdx.x;
+        }
+    }
+
+    __device__ bool next(Item& it) {
+        if (MODE == kDecoderSample) {
+            if (pos >= end) return false;
+            const int Tu = p.tiles_per_unit;
+            const int u = static_cast<int>(pos / Tu);
+            const long long ubeg = static_cast<long long>(u) * Tu;
+            const long long seg_end = (end < ubeg + Tu) ? end : ubeg + Tu;
+            const int qt = u % p.num_qtiles;
+            const int kvz = u / p.num_qtiles;  // b*Hkv + g
+            const int b = kvz / p.kv_heads, g = kvz % p.kv_heads;
+            it.q_z = u;
+            it.kv_z = kvz;
+            it.q_row0 = qt * kBlockM;
+            it.out_row0 = (b * p.q_heads + g * p.group) * p.S + qt * kBlockM;
+            it.q_y = it.out_row0;
+            it.n1 = ceil_div_i(p.S, kBlockN);
+            it.a1 = 0;
+            it.n0 = ceil_div_i(p.P, kBlockN);
+            it.t_begin = static_cast<int>(pos - ubeg);
+            it.t_end = static_cast<int>(seg_end - ubeg);
+            pos = seg_end;
+            return true;
+        } else {
+            if (k >= p.num_items) return false;
+            const int BH = p.batch * p.q_heads;
+            const int qt = p.num_qtiles - 1 - k / BH;  // longest rows first
+            const int bh = k % BH;
+            k += gridDim.x;
+            const int b = bh / p.q_heads, h = bh % p.q_heads;
+            it.q_z = bh;
+            it.kv_z = b * p.kv_heads + h / p.group;
+            it.q_row0 = qt * kBlockM;
+            it.q_y = it.q_row0;
+            it.out_row0 = 0;
+            const int L = p.L, S = p.S;
+            const int q_last = min(L, it.q_row0 + kBlockM) - 1;
+            if (MODE == kEncoder) {
+                const int hi = min(L, (q_last / S + 1) * S);
+                it.n1 = 0;
+                it.a1 = 0;
+                it.n0 = ceil_div_i(hi, kBlockN);
+            } else {
+                const int own_lo = (it.q_row0 / S) * S;
+                const int own_hi = min(L, (q_last / S + 1) * S);
+                it.a1 = own_lo / kBlockN;
+                it.n1 = ceil_div_i(own_hi, kBlockN) - it.a1;
+                it.n0 = ceil_div_i((q_last / S) * S, kBlockN);
+            }
+            it.t_begin = 0;
+            it.t_end = it.n1 + it.n0;
+            return true;
+        }
+    }
+};
+
+// Virtual tile t of an item -> (source, key tile, keys in the tile rounded to 16, box rows).
+struct TileRef {
+    int src, kt, nk16, box_rows;
+};
+
+template <int MODE>
+__device__ __forceinline__ TileRef tile_of(const FmhaParams& p, const Item& it, int t) {
+    TileRef r;
+    if (t < it.n1) {
+        r.src = 1;
+        r.kt = it.a1 + t;
+        const int len = (MODE == kDecoderSample) ? p.S : p.L;
+        r.nk16 = round16(min(kBlockN, len - r.kt * kBlockN));
+        r.box_rows = p.box1_rows;
+    } else {
+        r.src = 0;
+        r.kt = t - it.n1;
+        const int len = (MODE == kDecoderSample) ? p.P : p.L;
+        r.nk16 = round16(min(kBlockN, len - r.kt * kBlockN));
+        r.box_rows = kBlockN;
+    }
+    return r;
+}
+
+// Bounded mbarrier wait.  Returns false (and flags the CTA and the device error word) if the
+// phase does not complete within kWaitTimeoutNs or another role already gave up.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned int* err) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((spin & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (ptx::globaltimer_ns() - t0 > kWaitTimeoutNs) {
+                *abort_flag = 1;
+                atomicOr(err, kErrWaitTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Warp-collective form of wait_bar: every lane returns the same answer, so the .sync.aligned
+// tcgen05 instructions that follow are always executed by the whole warp.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              unsigned int* err) {
+    const bool ok = wait_bar(bar, parity, abort_flag, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Byte offset of 16-byte unit `u` of row `r` inside one swizzled chunk (row pitch RB bytes).
+template <int RB>
+__device__ __forceinline__ uint32_t swz_offset(int r, int u) {
+    const uint32_t a = static_cast<uint32_t>(r * RB + u * 16);
+    constexpr uint32_t mask = (RB == 128) ? 7u : 3u;
+    return a ^ (((a >> 7) & mask) << 4);
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_constant__ FmhaParams p) {
+    using C = Cfg<D>;
+    using SM = Smem<D, MODE>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::OFF_BAR);
+    uint64_t* k_full = bars;
+    uint64_t* v_full = bars + C::NST;
+    uint64_t* kv_empty = bars + 2 * C::NST;
+    uint64_t* q_full = bars + 3 * C::NST;
+    uint64_t* q_empty = q_full + 2;
+    uint64_t* s_full = q_full + 4;
+    uint64_t* p_full = q_full + 6;
+    uint64_t* o_free = q_full + 8;
+    uint64_t* pv_done = q_full + 10;
+    uint64_t* mma_drain = q_full + 11;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);
+    volatile int* bcast = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 16);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NST; ++i) {
+            ptx::mbar_init(&k_full[i], 1);
+            ptx::mbar_init(&v_full[i], 1);
+            ptx::mbar_init(&kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&q_full[i], 1);
+            ptx::mbar_init(&q_empty[i], 1);
+            ptx::mbar_init(&s_full[i], 1);
+            ptx::mbar_init(&p_full[i], kSoftmaxThreads);
+            ptx::mbar_init(&o_free[i], kSoftmaxThreads);
+        }
+        ptx::mbar_init(pv_done, 1);
+        ptx::mbar_init(mma_drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_holder, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const uint32_t smem_base = ptx::smem_u32(smem);
+    const uint32_t sQ = smem_base + SM::OFF_Q;
+    const uint32_t sK = smem_base + SM::OFF_K;
+    const uint32_t sV = smem_base + SM::OFF_V;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            ptx::tma_prefetch_desc(&p.tm_q);
+            ptx::tma_prefetch_desc(&p.tm_k0);
+            ptx::tma_prefetch_desc(&p.tm_v0);
+            if (MODE != kEncoder) {
+                ptx::tma_prefetch_desc(&p.tm_k1);
+                ptx::tma_prefetch_desc(&p.tm_v1);
+            }
+            Scheduler<MODE> sched(p);
+            Item it;
+            uint32_t kv_iter = 0, item_idx = 0;
+            int last_round[C::NST];
+            for (int i = 0; i < C::NST; ++i) last_round[i] = -1;
+            int q_last_round[2] = {-1, -1};
+            bool ok = true;
+            while (ok && sched.next(it)) {
+                const int qb = item_idx & 1;
+                const uint32_t qround = item_idx >> 1;
+                ok = wait_bar(&q_empty[qb], (qround & 1) ^ 1, abort_flag, p.err);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(&q_full[qb], C::TILE_BYTES);
+                for (int ch = 0; ch < C::NCH; ++ch) {
+                    uint8_t* dst = smem + SM::OFF_Q + qb * C::TILE_BYTES + ch * C::CHUNK_BYTES;
+                    if (MODE == kDecoderSample)
+                        ptx::tma_load_2d(&p.tm_q, &q_full[qb], dst, ch * (C::RB / 2), it.q_y);
+                    else
+                        ptx::tma_load_3d(&p.tm_q, &q_full[qb], dst, ch * (C::RB / 2), it.q_y, it.q_z);
+                }
+                q_last_round[qb] = static_cast<int>(qround);
+                for (int t = it.t_begin; t < it.t_end && ok; ++t) {
+                    const int st = kv_iter % C::NST;
+                    const uint32_t round = kv_iter / C::NST;
+                    ok = wait_bar(&kv_empty[st], (round & 1) ^ 1, abort_flag, p.err);
+                    if (!ok) break;
+                    const TileRef tr = tile_of<MODE>(p, it, t);
+                    const CUtensorMap* mk = tr.src ? &p.tm_k1 : &p.tm_k0;
+                    const CUtensorMap* mv = tr.src ? &p.tm_v1 : &p.tm_v0;
+                    const uint32_t bytes = static_cast<uint32_t>(tr.box_rows) * D * 2;
+                    ptx::mbar_arrive_expect_tx(&k_full[st], bytes);
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        ptx::tma_load_3d(mk, &k_full[st],
+                                         smem + SM::OFF_K + st * C::TILE_BYTES + ch * C::CHUNK_BYTES,
+                                         ch * (C::RB / 2), tr.kt * kBlockN, it.kv_z);
+                    ptx::mbar_arrive_expect_tx(&v_full[st], bytes);
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        ptx::tma_load_3d(mv, &v_full[st],
+                                         smem + SM::OFF_V + st * C::TILE_BYTES + ch * C::CHUNK_BYTES,
+                                         ch * (C::RB / 2), tr.kt * kBlockN, it.kv_z);
+                    last_round[st] = static_cast<int>(round);
+                    ++kv_iter;
+                }
+                ++item_idx;
+            }
+            // Never leave with copies in flight: wait for the last load of every buffer.
+            for (int i = 0; i < C::NST; ++i) {
+                if (last_round[i] >= 0) {
+                    const uint32_t par = static_cast<uint32_t>(last_round[i]) & 1u;
+                    volatile int no_abort = 0;
+                    wait_bar(&k_full[i], par, &no_abort, p.err);
+                    wait_bar(&v_full[i], par, &no_abort, p.err);
+                }
+            }
+            for (int i = 0; i < 2; ++i) {
+                if (q_last_round[i] >= 0) {
+                    volatile int no_abort = 0;
+                    wait_bar(&q_full[i], static_cast<uint32_t>(q_last_round[i]) & 1u, &no_abort, p.err);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            Scheduler<MODE> sched(p);
+            Item it;
+            uint32_t kv_iter = 0, gtile = 0, item_idx = 0;
+            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBlockM, D, true);
+            // Pending P.V of the previous tile (issued after the next QK^T so that the tensor
+            // core computes S_{j+1} while the softmax warps work on tile j).
+            bool have_pv = false;
+            uint32_t pv_sb = 0, pv_st = 0, pv_round = 0, pv_g = 0, pv_ob = 0, pv_item = 0;
+            int pv_nk = 0;
+            bool pv_first = false;
+            bool ok = true;
+
+            auto issue_pv = [&]() -> bool {
+                if (!wait_bar(&p_full[pv_sb], (pv_g >> 1) & 1, abort_flag, p.err)) return false;
+                if (pv_first &&
+                    !wait_bar(&o_free[pv_ob], ((pv_item >> 1) & 1) ^ 1, abort_flag, p.err))
+                    return false;
+                if (!wait_bar(&v_full[pv_st], pv_round & 1, abort_flag, p.err)) return false;
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + 256 + pv_ob * D;
+                const uint32_t a_tmem = tmem_base + pv_sb * 128;
+                const uint32_t v_base = sV + pv_st * C::TILE_BYTES;
+                for (int ks = 0; ks < pv_nk / 16; ++ks) {
+                    const uint64_t bdesc =
+                        ptx::smem_desc(v_base + ks * 16 * C::RB, C::CHUNK_BYTES, 8 * C::RB, C::SWZ);
+                    ptx::mma_ts(d_tmem, a_tmem + ks * 8, bdesc, idesc_pv,
+                                (pv_first && ks == 0) ? 0u : 1u);
+                }
+                ptx::mma_commit(&kv_empty[pv_st]);
+                ptx::mma_commit(pv_done);
+                return true;
+            };
+
+            while (ok && sched.next(it)) {
+                const int qb = item_idx & 1;
+                ok = wait_bar(&q_full[qb], (item_idx >> 1) & 1, abort_flag, p.err);
+                if (!ok) break;
+                const uint32_t q_base = sQ + qb * C::TILE_BYTES;
+                if (it.t_end <= it.t_begin) ptx::mma_commit(&q_empty[qb]);
+                for (int t = it.t_begin; t < it.t_end; ++t) {
+                    const uint32_t st = kv_iter % C::NST;
+                    const uint32_t round = kv_iter / C::NST;
+                    ok = wait_bar(&k_full[st], round & 1, abort_flag, p.err);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const TileRef tr = tile_of<MODE>(p, it, t);
+                    const uint32_t sb = gtile & 1;
+                    const uint32_t idesc_qk = ptx::idesc_bf16_f32(kBlockM, tr.nk16, false);
+                    const uint32_t k_base = sK + st * C::TILE_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const int ch = ks / C::KSTEPS_PER_CHUNK;
+                        const uint32_t off = ch * C::CHUNK_BYTES + (ks % C::KSTEPS_PER_CHUNK) * 32;
+                        const uint64_t adesc = ptx::smem_desc(q_base + off, 16, 8 * C::RB, C::SWZ);
+                        const uint64_t bdesc = ptx::smem_desc(k_base + off, 16, 8 * C::RB, C::SWZ);
+                        ptx::mma_ss(tmem_base + sb * 128, adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit(&s_full[sb]);
+                    if (t == it.t_end - 1) ptx::mma_commit(&q_empty[qb]);
+                    if (have_pv) {
+                        ok = issue_pv();
+                        if (!ok) break;
+                    }
+                    have_pv = true;
+                    pv_sb = sb;
+                    pv_st = st;
+                    pv_round = round;
+                    pv_g = gtile;
+                    pv_ob = item_idx & 1;
+                    pv_item = item_idx;
+                    pv_nk = tr.nk16;
+                    pv_first = (t == it.t_begin);
+                    ++kv_iter;
+                    ++gtile;
+                }
+                ++item_idx;
+            }
+            if (ok && have_pv) issue_pv();
+            // Drain: every MMA issued by this thread completes before TMEM is released.
+            ptx::mma_commit(mma_drain);
+            volatile int no_abort = 0;
+            wait_bar(mma_drain, 0, &no_abort, p.err);
+        }
+    } else {
+        // ------------------------------------------------------------------ softmax warps
+        const int quarter = warp & 3;             // TMEM lane quarter of this warp
+        const int row = quarter * 32 + lane;      // row of the query tile
+        const int stid = threadIdx.x - 64;        // 0..127 within the softmax group
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const float sl2 = p.scale_log2;
+        Scheduler<MODE> sched(p);
+        Item it;
+        uint32_t gtile = 0, item_idx = 0;
+        bool ok = true;
+        while (ok && sched.next(it)) {
+            // Per-row key intervals [lo, hi) for source 0 and source 1.
+            int lo0, hi0, lo1, hi1;
+            bool row_valid;
+            if (MODE == kDecoderSample) {
+                row_valid = (it.q_row0 + row) < p.rows_per_unit;
+                lo0 = 0;
+                hi0 = p.P;
+                lo1 = 0;
+                hi1 = p.S;
+            } else {
+                const int i_raw = it.q_row0 + row;
+                row_valid = i_raw < p.L;
+                const int i = min(i_raw, p.L - 1);
+                const int b0 = (i / p.S) * p.S;
+                if (MODE == kEncoder) {
+                    lo0 = 0;
+                    hi0 = min(p.L, b0 + p.S);
+                    lo1 = 0;
+                    hi1 = 0;
+                } else {
+                    lo0 = 0;
+                    hi0 = b0;
+                    lo1 = b0;
+                    hi1 = min(p.L, b0 + p.S);
+                }
+            }
+            float m = -INFINITY, l = 0.f;
+            const uint32_t ob = item_idx & 1;
+            const uint32_t o_tmem = tmem_base + lane_off + 256 + ob * D;
+            for (int t = it.t_begin; t < it.t_end; ++t) {
+                const uint32_t sb = gtile & 1;
+                ok = wait_bar_warp(&s_full[sb], (gtile >> 1) & 1, abort_flag, p.err);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const TileRef tr = tile_of<MODE>(p, it, t);
+                const int k0 = tr.kt * kBlockN;
+                const int lo = tr.src ? lo1 : lo0;
+                const int hi = tr.src ? hi1 : hi0;
+                const int cmin = lo - k0;
+                const int cmax = min(hi - k0, tr.nk16);
+                const uint32_t s_tmem = tmem_base + lane_off + sb * 128;
+                uint32_t s_raw[kBlockN];
+                const int nchunks = tr.nk16 / 32 + ((tr.nk16 % 32) ? 1 : 0);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    if (cc < nchunks) ptx::tmem_ld32(s_tmem + cc * 32, &s_raw[cc * 32]);
+                }
+                ptx::tmem_wait_ld();
+                float s[kBlockN];
+#pragma unroll
+                for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(s_raw[c]);
+                float tmax = -INFINITY;
+                if (cmin <= 0 && cmax >= kBlockN) {
+#pragma unroll
+                    for (int c = 0; c < kBlockN; ++c) {
+                        s[c] *= sl2;
+                        tmax = fmaxf(tmax, s[c]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < kBlockN; ++c) {
+                        s[c] = (c >= cmin && c < cmax) ? s[c] * sl2 : -INFINITY;
+                        tmax = fmaxf(tmax, s[c]);
+                    }
+                }
+                const float m_new = fmaxf(m, tmax);
+                const bool first = (t == it.t_begin);
+                bool rescale = false;
+                float alpha = 1.f;
+                if (m_new > m + kRescaleThreshold) {
+                    alpha = ptx::ex2(m - m_new);
+                    rescale = !first;
+                    m = m_new;
+                    l *= alpha;
+                }
+                const float m_use = (m == -INFINITY) ? 0.f : m;
+                float rsum = 0.f;
+                uint32_t pk[kBlockN / 2];
+#pragma unroll
+                for (int c = 0; c < kBlockN; c += 2) {
+                    const float e0 = ptx::ex2(s[c] - m_use);
+                    const float e1 = ptx::ex2(s[c + 1] - m_use);
+                    rsum += e0 + e1;
+                    pk[c / 2] = ptx::pack_bf16x2(e0, e1);
+                }
+                l += rsum;
+                // P (bf16) goes over the first half of this S buffer.
+                ptx::tmem_st32(s_tmem, pk);
+                if (tr.nk16 > 64) ptx::tmem_st32(s_tmem + 32, pk + 32);
+                if (!first) {
+                    // O may only be touched once the previous P.V has landed.
+                    ok = wait_bar_warp(pv_done, (gtile - 1) & 1, abort_flag, p.err);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    // tcgen05.ld/st are warp-collective: the warp rescales if any row needs it.
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        const float f = rescale ? alpha : 1.f;
+#pragma unroll
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            uint32_t o[32];
+                            ptx::tmem_ld32(o_tmem + c0, o);
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+                            ptx::tmem_st32(o_tmem + c0, o);
+                        }
+                    }
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&p_full[sb]);
+                ++gtile;
+            }
+            if (!ok) break;
+            // ---------------------------------------------------------------- epilogue
+            ok = wait_bar_warp(pv_done, (gtile - 1) & 1, abort_flag, p.err);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            uint32_t o_raw[D];
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) ptx::tmem_ld32(o_tmem + c0, &o_raw[c0]);
+            ptx::tmem_wait_ld();
+            float o[D];
+#pragma unroll
+            for (int c = 0; c < D; ++c) o[c] = __uint_as_float(o_raw[c]);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&o_free[ob]);
+
+            if (MODE != kDecoderSample) {
+                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                // Stage the bf16 tile in the 128B/64B-swizzled layout of the output tensor map.
+                if (stid == 0) ptx::tma_store_wait_read_all();
+                ptx::named_barrier_sync(1, kSoftmaxThreads);
+                uint8_t* stage = smem + SM::OFF_O;
+#pragma unroll
+                for (int ch = 0; ch < C::NCH; ++ch) {
+#pragma unroll
+                    for (int u = 0; u < C::RB / 16; ++u) {
+                        const int c = ch * (C::RB / 2) + u * 8;
+                        uint4 w;
+                        w.x = ptx::pack_bf16x2(o[c + 0] * inv_l, o[c + 1] * inv_l);
+                        w.y = ptx::pack_bf16x2(o[c + 2] * inv_l, o[c + 3] * inv_l);
+                        w.z = ptx::pack_bf16x2(o[c + 4] * inv_l, o[c + 5] * inv_l);
+                        w.w = ptx::pack_bf16x2(o[c + 6] * inv_l, o[c + 7] * inv_l);
+                        *reinterpret_cast<uint4*>(stage + ch * C::CHUNK_BYTES + swz_offset<C::RB>(row, u)) = w;
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::named_barrier_sync(1, kSoftmaxThreads);
+                if (stid == 0) {
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        ptx::tma_store_3d(&p.tm_o, stage + ch * C::CHUNK_BYTES, ch * (C::RB / 2),
+                                          it.q_row0, it.q_z);
+                    ptx::tma_store_commit();
+                }
+                if (p.lse != nullptr && row_valid) {
+                    p.lse[static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row] =
+                        (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+                }
+            } else {
+                // ------------------------------------------------------------ sampling epilogue
+                const int Tu = p.tiles_per_unit;
+                const bool whole = (it.t_begin == 0 && it.t_end == Tu);
+                __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
+                if (whole) {
+                    if (row_valid) {
+                        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                        uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D);
+#pragma unroll
+                        for (int c = 0; c < D; c += 8) {
+                            uint4 w;
+                            w.x = ptx::pack_bf16x2(o[c + 0] * inv_l, o[c + 1] * inv_l);
+                            w.y = ptx::pack_bf16x2(o[c + 2] * inv_l, o[c + 3] * inv_l);
+                            w.z = ptx::pack_bf16x2(o[c + 4] * inv_l, o[c + 5] * inv_l);
+                            w.w = ptx::pack_bf16x2(o[c + 6] * inv_l, o[c + 7] * inv_l);
+                            dst[c / 8] = w;
+                        }
+                        if (p.lse != nullptr)
+                            p.lse[it.out_row0 + row] =
+                                (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+                    }
+                } else {
+                    // Split unit: publish (O, m, l) in this CTA's slot, take a ticket; the last
+                    // CTA of the unit merges every slot.
+                    const long long T = p.total_tiles;
+                    const int grid = gridDim.x;
+                    const long long ubeg = static_cast<long long>(it.q_z) * Tu;
+                    const int c_first = owner_cta(ubeg, T, grid);
+                    const int c_last = owner_cta(ubeg + Tu - 1, T, grid);
+                    auto slot_of = [&](int c) -> int {
+                        return (range_begin(c, T, grid) >= ubeg) ? 2 * c : 2 * c + 1;
+                    };
+                    float* slot = p.ws_partial + static_cast<size_t>(slot_of(blockIdx.x)) * p.slot_floats;
+                    if (row_valid && row < p.rows_cap) {
+                        float4* so = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D);
+#pragma unroll
+                        for (int c = 0; c < D; c += 4) so[c / 4] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+                        slot[p.rows_cap * D + row] = m;
+                        slot[p.rows_cap * D + p.rows_cap + row] = l;
+                    }
+                    __threadfence();
+                    ptx::named_barrier_sync(1, kSoftmaxThreads);
+                    if (stid == 0) {
+                        const int ticket = atomicAdd(&p.ws_tickets[c_first], 1);
+                        const int last = (ticket == c_last - c_first) ? 1 : 0;
+                        if (last) p.ws_tickets[c_first] = 0;
+                        *bcast = last;
+                    }
+                    ptx::named_barrier_sync(1, kSoftmaxThreads);
+                    const int is_last = *bcast;
+                    ptx::named_barrier_sync(1, kSoftmaxThreads);
+                    if (is_last) {
+                        __threadfence();
+                        if (row_valid && row < p.rows_cap) {
+                            float mmax = -INFINITY;
+                            for (int c = c_first; c <= c_last; ++c) {
+                                const float* sl = p.ws_partial + static_cast<size_t>(slot_of(c)) * p.slot_floats;
+                                mmax = fmaxf(mmax, __ldcg(sl + p.rows_cap * D + row));
+                            }
+                            const float muse = (mmax == -INFINITY) ? 0.f : mmax;
+                            float ltot = 0.f;
+                            for (int c = c_first; c <= c_last; ++c) {
+                                const float* sl = p.ws_partial + static_cast<size_t>(slot_of(c)) * p.slot_floats;
+                                ltot += ptx::ex2(__ldcg(sl + p.rows_cap * D + row) - muse) *
+                                        __ldcg(sl + p.rows_cap * D + p.rows_cap + row);
+                            }
+                            const float inv_l = (ltot > 0.f) ? 1.f / ltot : 0.f;
+                            uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D);
+#pragma unroll 1
+                            for (int c0 = 0; c0 < D; c0 += 32) {
+                                float acc[32];
+#pragma unroll
+                                for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+                                for (int c = c_first; c <= c_last; ++c) {
+                                    const float* sl = p.ws_partial + static_cast<size_t>(slot_of(c)) * p.slot_floats;
+                                    const float w = ptx::ex2(__ldcg(sl + p.rows_cap * D + row) - muse);
+                                    const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + c0);
+#pragma unroll
+                                    for (int c4 = 0; c4 < 8; ++c4) {
+                                        const float4 v = __ldcg(so + c4);
+                                        acc[4 * c4 + 0] += w * v.x;
+                                        acc[4 * c4 + 1] += w * v.y;
+                                        acc[4 * c4 + 2] += w * v.z;
+                                        acc[4 * c4 + 3] += w * v.w;
+                                    }
+                                }
+#pragma unroll
+                                for (int c = 0; c < 32; c += 8) {
+                                    uint4 w;
+                                    w.x = ptx::pack_bf16x2(acc[c + 0] * inv_l, acc[c + 1] * inv_l);
+                                    w.y = ptx::pack_bf16x2(acc[c + 2] * inv_l, acc[c + 3] * inv_l);
+                                    w.z = ptx::pack_bf16x2(acc[c + 4] * inv_l, acc[c + 5] * inv_l);
+                                    w.w = ptx::pack_bf16x2(acc[c + 6] * inv_l, acc[c + 7] * inv_l);
+                                    dst[(c0 + c) / 8] = w;
+                                }
+                            }
+                            if (p.lse != nullptr)
+                                p.lse[it.out_row0 + row] =
+                                    (ltot > 0.f) ? (mmax + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
+                        }
+                    }
+                }
+            }
+            ++item_idx;
+        }
+        if (MODE != kDecoderSample && stid == 0) ptx::tma_store_wait_all();
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace e2d2

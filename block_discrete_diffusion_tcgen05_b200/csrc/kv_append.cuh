@@ -1,0 +1,32 @@
+// kv_append.cuh -- KV-cache append: after a block is decoded the encoder absorbs it and each
+// layer's cache grows by that block ("Encoder-Decoder Diffusion Language Models for Efficient
+// Training and Inference", paper notes, sec. 3).  A pure copy, HBM-bound: 16-byte vector
+// loads and stores, grid-stride over the rows of K (blockIdx.y == 0) and V (blockIdx.y == 1).
+#pragma once
+
+#include <cstdint>
+
+namespace e2d2 {
+
+struct AppendParams {
+    uint4* cache[2];      // K, V caches [B*Hkv][capacity][D]
+    const uint4* src[2];  // new rows [B*Hkv][S_new][D]
+    int capacity, P, S_new, vec_per_row, units;
+};
+
+__global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams a) {
+    const int which = blockIdx.y;
+    uint4* __restrict__ dst = a.cache[which];
+    const uint4* __restrict__ src = a.src[which];
+    const long long per_unit = static_cast<long long>(a.S_new) * a.vec_per_row;
+    const long long total = per_unit * a.units;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long unit = i / per_unit;
+        const long long rem = i - unit * per_unit;  // (row, vec) inside the unit
+        const long long d = (unit * a.capacity + a.P) * a.vec_per_row + rem;
+        dst[d] = __ldg(src + i);
+    }
+}
+
+}  // namespace e2d2

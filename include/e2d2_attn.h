@@ -1,0 +1,142 @@
+/*
+ * e2d2_attn.h -- C ABI of the E2D2 fused block-diffusion attention for NVIDIA B200 (sm_100a).
+ *
+ * The operations are the attention calls of the E2D2 encoder-decoder block diffusion
+ * language model, as the pages describe them:
+ *   [E2D2 notes]  "Encoder-Decoder Diffusion Language Models for Efficient Training and
+ *                 Inference" (paper notes): sec. 2 "two connection variants" (last hidden
+ *                 state / shared KV cache; self- and cross-attention fused in one call),
+ *                 sec. 3 "sampling algorithm", sec. 4 "training algorithm" (block-causal
+ *                 encoder mask; decoder mask over 2L keys; FLOPs table).
+ *   [BD3LM blog]  "Block Diffusion: Interpolating Between Autoregressive and Diffusion
+ *                 Language Models", sec. 3 "block decomposition": position i is in block
+ *                 floor(i / S).
+ *
+ * Common conventions
+ *   - Every tensor is a plain device pointer to contiguous row-major memory, head_dim
+ *     innermost.  Q/K/V/O and KV caches are bfloat16; LSE is float32.  The caller owns all
+ *     memory; the library never allocates device memory.
+ *   - q, out: [batch][q_heads][len][head_dim]; k, v: [batch][kv_heads][len][head_dim];
+ *     KV cache: [batch][kv_heads][capacity][head_dim]; lse: [batch][q_heads][len].
+ *   - GQA: query head h reads kv head h / (q_heads / kv_heads).
+ *   - scale <= 0 selects 1/sqrt(head_dim).  lse is the natural-log log-sum-exp of the scaled
+ *     scores of each query row; pass NULL to skip it.
+ *   - Every call is enqueued on `stream` and never synchronises.  Argument errors are
+ *     reported before anything is launched; nothing is launched then.  E2D2_ERR_CUDA means a
+ *     launch or driver call failed.  A device-side wait that times out (bounded spin) sets a
+ *     device error word that e2d2_last_device_error() reads.
+ *   - Supported: head_dim in {32, 64, 128}; q_heads % kv_heads == 0; pointers 16-byte
+ *     aligned; lengths below 2^31 elements per dimension.
+ *   - The last-hidden-state and shared-KV-cache variants ([E2D2 notes, sec. 2]) are the same
+ *     calls: they differ only in which K/V the caller passes as the encoder side.
+ */
+#ifndef E2D2_ATTN_H_
+#define E2D2_ATTN_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define E2D2_API __attribute__((visibility("default")))
+#else
+#define E2D2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    E2D2_OK = 0,
+    E2D2_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad GQA ratio            */
+    E2D2_ERR_UNSUPPORTED = 2, /* head_dim not in {32, 64, 128}, or not an sm_100 device     */
+    E2D2_ERR_SHAPE = 3,       /* L % S != 0, S > L, or a dimension too large                 */
+    E2D2_ERR_ALIGNMENT = 4,   /* a pointer not 16-byte aligned                              */
+    E2D2_ERR_CAPACITY = 5,    /* P + S_new > capacity, or P > capacity                      */
+    E2D2_ERR_WORKSPACE = 6,   /* workspace missing or smaller than the _workspace query     */
+    E2D2_ERR_CUDA = 7,        /* a CUDA runtime / driver call failed                        */
+    E2D2_ERR_TIMEOUT = 8      /* a bounded device-side wait gave up (see e2d2_last_device_error) */
+} e2d2_status;
+
+typedef struct {
+    int batch;
+    int q_heads;
+    int kv_heads;
+    int head_dim;
+    float scale; /* <= 0: 1/sqrt(head_dim) */
+} e2d2_dims;
+
+/*
+ * Encoder block-causal self-attention over clean tokens ([E2D2 notes, sec. 4]): query i
+ * attends to every key j with floor(j/S) <= floor(i/S) (its own block, bidirectionally, and
+ * every earlier block).
+ *   q   [batch][q_heads][L][d]   k, v [batch][kv_heads][L][d]   out [batch][q_heads][L][d]
+ *   lse [batch][q_heads][L] or NULL.   Requires 1 <= S <= L and L % S == 0.
+ */
+E2D2_API e2d2_status e2d2_attn_encoder_blockcausal(const void* q, const void* k, const void* v, void* out,
+                                          float* lse, e2d2_dims dims, int L, int S,
+                                          cudaStream_t stream);
+
+/*
+ * Decoder fused self+cross attention, training mode ([E2D2 notes, sec. 2 and 4]): the L noised
+ * queries attend over 2L keys in one call -- the encoder-side keys k_enc/v_enc of the clean
+ * blocks strictly before the query's block, and the decoder-side keys k_dec/v_dec of the
+ * query's own block (bidirectional inside the block).
+ *   q_dec [batch][q_heads][L][d]; k_enc, v_enc, k_dec, v_dec [batch][kv_heads][L][d];
+ *   out [batch][q_heads][L][d]; lse [batch][q_heads][L] or NULL.  Requires L % S == 0.
+ */
+E2D2_API e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_enc, const void* v_enc,
+                                    const void* k_dec, const void* v_dec, void* out, float* lse,
+                                    e2d2_dims dims, int L, int S, cudaStream_t stream);
+
+/*
+ * Bytes of scratch workspace that e2d2_attn_decoder_sample needs for these dims and block
+ * size (split-KV partial results and per-split tickets).  Needs no GPU.  The caller
+ * allocates it once, zero-filled; every completed call leaves its ticket words at zero again,
+ * so the same workspace can be reused by later calls on the same stream.  Calls that may run
+ * at the same time (different streams) need different workspaces.  After E2D2_ERR_TIMEOUT
+ * the workspace must be zero-filled again.
+ */
+E2D2_API size_t e2d2_attn_decoder_sample_workspace(e2d2_dims dims, int S, int capacity);
+
+/*
+ * Decoder sampling step ([E2D2 notes, sec. 3]): the S noised queries of the block being
+ * denoised attend to the first P rows of the cached encoder KV (the clean prefix) and to
+ * the K/V of their own block, in one call.  Split-KV over the prefix; GQA rows packed.
+ *   q_blk [batch][q_heads][S][d]; k_cache, v_cache [batch][kv_heads][capacity][d] (rows
+ *   P..capacity-1 are never read); k_blk, v_blk [batch][kv_heads][S][d];
+ *   out [batch][q_heads][S][d]; lse [batch][q_heads][S] or NULL.
+ *   Requires 0 <= P <= capacity and ws_bytes >= e2d2_attn_decoder_sample_workspace().
+ */
+E2D2_API e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, const void* v_cache,
+                                     int capacity, int P, const void* k_blk, const void* v_blk,
+                                     void* out, float* lse, e2d2_dims dims, int S, void* workspace,
+                                     size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * KV-cache append ([E2D2 notes, sec. 3]: after a block is decoded the encoder absorbs it and
+ * the cache grows by that block): rows P..P+S_new-1 of every (batch, kv head) cache take the
+ * rows of k_new / v_new, bit for bit.  k_new, v_new [batch][kv_heads][S_new][d].  The cache
+ * length is tracked by the caller (P += S_new after E2D2_OK).  Requires P + S_new <= capacity.
+ */
+E2D2_API e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int P,
+                                 const void* k_new, const void* v_new, int S_new, e2d2_dims dims,
+                                 cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+E2D2_API const char* e2d2_status_string(e2d2_status status);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the current device:
+ * E2D2_OK, or E2D2_ERR_TIMEOUT if a bounded device-side wait gave up since the last read.
+ */
+E2D2_API e2d2_status e2d2_last_device_error(cudaStream_t stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+E2D2_API int e2d2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E2D2_ATTN_H_ */

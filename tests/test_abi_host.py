@@ -1,0 +1,105 @@
+"""Host-only checks of the C ABI (no GPU): the library loads, exports every function that
+include/e2d2_attn.h declares, and rejects bad arguments with the documented status before
+touching the GPU."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from block_discrete_diffusion_tcgen05_b200 import _lib, build
+
+ROOT = Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "e2d2_attn.h"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def header_functions():
+    text = HEADER.read_text()
+    return re.findall(r"E2D2_API\s+[\w\s\*]+?\b(e2d2_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(header_functions())
+    assert {"e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train", "e2d2_attn_decoder_sample",
+            "e2d2_kv_cache_append", "e2d2_attn_decoder_sample_workspace"} <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    assert set(_lib.EXPORTS) <= set(header_functions())
+
+
+def test_status_strings(lib):
+    for code, name in _lib.STATUS.items():
+        assert lib.e2d2_status_string(code).decode() == name
+    assert lib.e2d2_version() == 100
+
+
+DIMS = _lib.Dims(2, 4, 2, 64, 0.0)
+P16 = 0x10000  # fake 16-byte aligned addresses; validation must fail before any use
+
+
+def test_encoder_argument_errors(lib):
+    f = lib.e2d2_attn_encoder_blockcausal
+    assert f(None, P16, P16, P16, None, DIMS, 64, 8, None) == 1          # null q
+    assert f(P16, P16, P16, P16, None, _lib.Dims(2, 4, 2, 96, 0.0), 64, 8, None) == 2  # head_dim
+    assert f(P16, P16, P16, P16, None, _lib.Dims(2, 4, 3, 64, 0.0), 64, 8, None) == 1  # GQA ratio
+    assert f(P16, P16, P16, P16, None, _lib.Dims(0, 4, 2, 64, 0.0), 64, 8, None) == 1  # batch
+    assert f(P16, P16, P16, P16, None, DIMS, 60, 8, None) == 3           # S does not divide L
+    assert f(P16, P16, P16, P16, None, DIMS, 8, 16, None) == 3           # S > L
+    assert f(P16, P16, P16, P16, None, DIMS, 0, 8, None) == 1            # L = 0
+    assert f(P16 + 8, P16, P16, P16, None, DIMS, 64, 8, None) == 4       # misaligned q
+    assert f(P16, P16, P16, P16, P16 + 2, DIMS, 64, 8, None) == 4        # misaligned lse
+    assert f(P16, P16, P16, P16, None, _lib.Dims(2, 4, 2, 64, float("nan")), 64, 8, None) == 1
+
+
+def test_decoder_train_argument_errors(lib):
+    f = lib.e2d2_attn_decoder_train
+    assert f(P16, P16, P16, None, P16, P16, None, DIMS, 64, 8, None) == 1
+    assert f(P16, P16, P16, P16, P16 + 4, P16, None, DIMS, 64, 8, None) == 4
+    assert f(P16, P16, P16, P16, P16, P16, None, DIMS, 64, 7, None) == 3
+
+
+def test_sample_workspace_query_needs_no_gpu(lib):
+    n = lib.e2d2_attn_decoder_sample_workspace(_lib.Dims(32, 16, 8, 128, 0.0), 16, 2064)
+    assert n > 0
+    assert lib.e2d2_attn_decoder_sample_workspace(_lib.Dims(32, 16, 8, 96, 0.0), 16, 2064) == 0
+
+
+def test_sample_argument_errors(lib):
+    f = lib.e2d2_attn_decoder_sample
+    dm = _lib.Dims(2, 4, 2, 128, 0.0)
+    ws = lib.e2d2_attn_decoder_sample_workspace(dm, 16, 64)
+    assert f(P16, P16, P16, 64, 65, P16, P16, P16, None, dm, 16, P16, ws, None) == 5   # P > capacity
+    assert f(P16, P16, P16, 64, 32, P16, P16, P16, None, dm, 16, None, ws, None) == 6  # no workspace
+    assert f(P16, P16, P16, 64, 32, P16, P16, P16, None, dm, 16, P16, ws - 1, None) == 6
+    assert f(P16, P16, P16, 64, -1, P16, P16, P16, None, dm, 16, P16, ws, None) == 1
+    assert f(P16, P16, P16 + 8, 64, 32, P16, P16, P16, None, dm, 16, P16, ws, None) == 4
+    assert f(P16, P16, P16, 64, 32, P16, P16, None, None, dm, 16, P16, ws, None) == 1
+
+
+def test_append_argument_errors(lib):
+    f = lib.e2d2_kv_cache_append
+    dm = _lib.Dims(2, 2, 2, 64, 0.0)
+    assert f(P16, P16, 32, 30, P16, P16, 4, dm, None) == 5
+    assert f(P16, None, 32, 0, P16, P16, 4, dm, None) == 1
+    assert f(P16, P16, 32, 0, P16 + 2, P16, 4, dm, None) == 4
+    assert f(P16, P16, 32, 0, P16, P16, 0, dm, None) == 0  # nothing to copy: no launch
+
+
+def test_product_package_never_imports_the_oracle():
+    pkg = ROOT / "block_discrete_diffusion_tcgen05_b200"
+    for p in pkg.rglob("*.py"):
+        src = p.read_text()
+        assert "import oracle" not in src and "from oracle" not in src, p
+    for p in (ROOT / "oracle").rglob("*.py"):
+        src = p.read_text()
+        assert "import block_discrete_diffusion_tcgen05_b200" not in src, p
+        assert "from block_discrete_diffusion_tcgen05_b200" not in src, p
