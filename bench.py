@@ -120,13 +120,39 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------------------------
+# multi-rank plumbing (weak scaling: every rank runs the same per-GPU workload on its own
+# seeded inputs; no data-path collective; the only collectives are barriers and the max of
+# the timings)
+# --------------------------------------------------------------------------------------------
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """Max of a host float over all ranks (identity without a process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_ms: float, scale: float) -> float:
+    """Whole-job throughput: the units all ranks processed divided by the slowest rank's time."""
+    return units_per_rank_step * steps * world / (max_ms * 1e-3) / scale
+
+
+def rank_seed_layer(rank: int) -> int:
+    """Each rank draws its own inputs (the seed recipe's layer slot carries the rank)."""
+    return rank
+
+
+# --------------------------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------------------------
 def make_inputs(torch, dev, rank: int):
     from block_discrete_diffusion_tcgen05_b200 import synth, workloads
 
     def t(shape, wl, tensor, sigma):
-        a = synth.normal_bf16(shape, synth.seed_for(wl, rank, tensor), sigma)
+        a = synth.normal_bf16(shape, synth.seed_for(wl, rank_seed_layer(rank), tensor), sigma)
         return synth.to_torch(a, dev)
 
     tw, sw = workloads.TRAIN, workloads.SAMPLE
@@ -216,26 +242,19 @@ def run_ours(args, rank, world, local_rank):
     per_kernel_ms = {n: sum(a.elapsed_time(b) for a, b in ev[n]) for n, _ in kernels}
     launches = K * len(kernels)
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    total_ms = max_over_ranks(total_ms)
-    per_kernel_ms = {n: max_over_ranks(v) for n, v in per_kernel_ms.items()}
+    total_ms = max_over_ranks(total_ms, dist, dev)
+    per_kernel_ms = {n: max_over_ranks(v, dist, dev) for n, v in per_kernel_ms.items()}
 
     # ---- metrics -------------------------------------------------------------------------
     peaks, peak_kind = load_peaks()
     fl_train = workloads.useful_flops_train(tw)  # per call (encoder or decoder pass)
     train_ms = per_kernel_ms["encoder"] + per_kernel_ms["decoder_train"]
-    value = (2 * fl_train * K * world) / (train_ms * 1e-3) / 1e12
+    value = whole_job_rate(2 * fl_train, K, world, train_ms, 1e12)
     by_enc = workloads.bytes_train(tw, decoder=False)
     by_dec = workloads.bytes_train(tw, decoder=True)
     by_smp = workloads.bytes_sample(sw)
     smp_s = per_kernel_ms["decoder_sample"] * 1e-3
-    sample_gbs = by_smp * K * world / smp_s / 1e9
+    sample_gbs = whole_job_rate(by_smp, K, world, per_kernel_ms["decoder_sample"], 1e9)
 
     # dominant kernel by device time
     dom = max(("encoder", "decoder_train", "decoder_sample"), key=lambda n: per_kernel_ms[n])
@@ -335,48 +354,70 @@ def run_e2e(torch, attn, workloads, train, dev, args, dist, world):
         step()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b), dist, dev)
     fl = 2 * workloads.useful_flops_train(tw)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out + host_lse)
-    return {"value": fl * n * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+    return {"value": whole_job_rate(fl, n, world, ms, 1e12), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n}
 
 
 # --------------------------------------------------------------------------------------------
 # CPU oracle (baseline / reference arm)
 # --------------------------------------------------------------------------------------------
-def oracle_train_sample(budget_s: float):
-    """Times the oracle on a bounded sample of the train pass: all 16 heads of as many batch
-    entries as fit the budget (heads are independent, so useful FLOPs scale exactly)."""
-    import numpy as np
+_ORACLE_CACHE = {}
 
-    import oracle
-    from block_discrete_diffusion_tcgen05_b200 import synth, workloads
 
-    orc = oracle.default()
+def _oracle_inputs():
+    if "inputs" not in _ORACLE_CACHE:
+        import oracle
+        from block_discrete_diffusion_tcgen05_b200 import synth, workloads
+
+        tw = workloads.TRAIN
+        shp = (tw.batch, tw.q_heads, tw.L, tw.head_dim)
+        gen = lambda n: synth.normal_bf16(shp, synth.seed_for(2, 0, n), tw.sigma).f32
+        _ORACLE_CACHE["inputs"] = tuple(gen(n) for n in ("q", "k", "v", "k_enc", "v_enc"))
+        _ORACLE_CACHE["orc"] = oracle.default()
+    return _ORACLE_CACHE["orc"], _ORACLE_CACHE["inputs"]
+
+
+def _oracle_pass(orc, inputs, b0, nb, nh):
+    from block_discrete_diffusion_tcgen05_b200 import workloads
+
     tw = workloads.TRAIN
-    shp = (1, tw.q_heads, tw.L, tw.head_dim)
-    gen = lambda n: synth.normal_bf16(shp, synth.seed_for(2, 0, n), tw.sigma).f32
-    q, k, v, ke, ve = (gen(n) for n in ("q", "k", "v", "k_enc", "v_enc"))
-    done_b, t_total = 0, 0.0
-    while done_b < tw.batch:
-        t0 = time.perf_counter()
-        orc.encoder(q, k, v, tw.S)
-        orc.decoder_train(q, ke, ve, k, v, tw.S)
-        t_total += time.perf_counter() - t0
-        done_b += 1
-        if t_total * (done_b + 1) / done_b > budget_s:
-            break
+    q, k, v, ke, ve = (x[b0:b0 + nb, :nh] for x in inputs)
+    t0 = time.perf_counter()
+    orc.encoder(q, k, v, tw.S)
+    orc.decoder_train(q, ke, ve, k, v, tw.S)
+    return time.perf_counter() - t0
+
+
+def oracle_train_sample(budget_s: float):
+    """Times the CPU oracle on a bounded sample of the E2D2 train pass (encoder + decoder-train):
+    whole batch entries (16 heads each) while they fit the budget, else a subset of the heads of
+    one entry.  Heads are independent, so useful FLOPs scale exactly with the heads computed."""
+    from block_discrete_diffusion_tcgen05_b200 import workloads
+
+    tw = workloads.TRAIN
+    orc, inputs = _oracle_inputs()
+    if "t_batch" not in _ORACLE_CACHE:  # calibration: one batch entry, all heads
+        _ORACLE_CACHE["t_batch"] = _oracle_pass(orc, inputs, 0, 1, tw.q_heads)
+    t_batch = _ORACLE_CACHE["t_batch"]
+    heads_done, t_total, b = 0, 0.0, 0
+    if budget_s < t_batch:
+        nh = max(1, min(tw.q_heads, int(tw.q_heads * budget_s / t_batch)))
+        t_total = _oracle_pass(orc, inputs, 0, 1, nh)
+        heads_done = nh
+    else:
+        while t_total + t_batch <= budget_s or heads_done == 0:
+            t_total += _oracle_pass(orc, inputs, b % tw.batch, 1, tw.q_heads)
+            heads_done += tw.q_heads
+            b += 1
     pairs = workloads.unmasked_pairs(tw.L, tw.S)
-    flops = 2 * 4 * tw.head_dim * tw.q_heads * done_b * pairs
+    flops = 2 * 4 * tw.head_dim * heads_done * pairs
     return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
-            "sample": f"E2D2 train pass, encoder + decoder-train, {done_b} of {tw.batch} batch entries "
-                      f"x {tw.q_heads} heads (L1024 S16 d64), fp64, {t_total:.1f} s",
+            "sample": f"E2D2 train pass (encoder + decoder-train, L1024 S16 d64), {heads_done} (batch, head) "
+                      f"pairs of the workload's {tw.batch * tw.q_heads}, fp64, {t_total:.2f} s",
             "seconds": t_total}
 
 
@@ -393,8 +434,10 @@ def run_reference(args, rank, world):
         return
     t0 = time.perf_counter()
     per_step = []
+    # Keep the whole reference run to a few minutes whatever --steps/--warmup are.
+    step_budget = min(args.ref_step_budget, args.ref_total_budget / (args.warmup + args.steps))
     for i in range(args.warmup + args.steps):
-        r = oracle_train_sample(args.ref_step_budget)
+        r = oracle_train_sample(step_budget)
         if i >= args.warmup:
             per_step.append(r)
     vals = [r["value"] for r in per_step]
@@ -426,7 +469,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--ref-step-budget", type=float, default=8.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--ref-step-budget", type=float, default=8.0, help="max seconds of oracle work per reference step")
+    ap.add_argument("--ref-total-budget", type=float, default=150.0, help="seconds of oracle work for the whole reference run")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

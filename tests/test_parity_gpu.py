@@ -148,7 +148,7 @@ def test_outputs_fully_written_deterministic_and_bounded():
         res.append((out.clone(), lse.clone()))
     assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
     # sampling path
-    qs, kc, vc, kb, vb = H.sample_inputs(2, 8, 2, 16, 700, 800, 128, 1.0, 900)
+    qs, kc, vc, kb, vb = H.sample_inputs(2, 8, 2, 16, 800, 128, 1.0, 900)
     res = []
     for _ in range(2):
         o, l = attn.decoder_sample(qs[1], kc[1], vc[1], 700, kb[1], vb[1])
