@@ -51,10 +51,14 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_SOURCES = ("fmha_sm100.cuh", "ptx_sm100.cuh", "kv_append.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the device-code sources: ncu counters are only reported for the code they measured."""
     h = hashlib.sha256()
-    for p in sorted((ROOT / "block_discrete_diffusion_tcgen05_b200" / "csrc").glob("*")):
-        h.update(p.read_bytes())
+    for name in KERNEL_SOURCES:
+        h.update((ROOT / "block_discrete_diffusion_tcgen05_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()[:16]
 
 
