@@ -357,3 +357,69 @@ e2d2_status e2d2_last_device_error(cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Sampling step without any allocation: for callers that cannot allocate device memory.
+//
+// Some callers have no way to obtain a workspace: a serving engine that hands (nearly) all of
+// HBM to its own KV-cache pool at start-up and offers plugins no allocator, or a caller whose
+// hot path may not call cudaMalloc because that call can synchronise the device.  This entry
+// point takes the split-KV scratch from a file-scope device array instead.  The array
+// (kNoAllocScratchBytes) is reserved on every GPU that loads this library until the process
+// exits.  Every call shares it and it keeps the last call's contents: the per-CTA ticket words
+// are cleared (cudaMemsetAsync, which allocates nothing) before each launch, and the partial
+// slots are always written before they are read.  Calls that overlap on the GPU (different
+// streams, or different host threads on the same device) race on the array.
+// ---------------------------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = E2D2_SAMPLE_NOALLOC_MAX_BYTES;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+struct NoAllocScratch {
+    bool ready = false;
+    void* ptr = nullptr;  // device address of g_noalloc_scratch on this device
+};
+std::mutex g_noalloc_mutex;
+NoAllocScratch g_noalloc[kMaxDevices];
+
+// The host-side name of g_noalloc_scratch is only a stand-in; the device address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+e2d2_status noalloc_scratch(void** ptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return E2D2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    NoAllocScratch& s = g_noalloc[dev];
+    if (!s.ready) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return E2D2_ERR_CUDA;
+        s.ptr = p;
+        s.ready = true;
+    }
+    *ptr = s.ptr;
+    return E2D2_OK;
+}
+}  // namespace
+
+extern "C" {
+
+e2d2_status e2d2_attn_decoder_sample_noalloc(const void* q_blk, const void* k_cache, const void* v_cache,
+                                             int capacity, int P, const void* k_blk, const void* v_blk,
+                                             void* out, float* lse, e2d2_dims dims, int S,
+                                             cudaStream_t stream) {
+    if (!q_blk || !k_cache || !v_cache || !k_blk || !v_blk || !out) return E2D2_ERR_INVALID_ARG;
+    const e2d2_status sd = check_dims(dims);
+    if (sd != E2D2_OK) return sd;
+    if (S <= 0 || capacity < 0 || P < 0) return E2D2_ERR_INVALID_ARG;
+    const size_t need = e2d2_attn_decoder_sample_workspace(dims, S, capacity);
+    if (need == 0) return E2D2_ERR_INVALID_ARG;
+    if (need > kNoAllocScratchBytes) return E2D2_ERR_WORKSPACE;  // shape needs more than the array
+    void* scratch = nullptr;
+    e2d2_status s = noalloc_scratch(&scratch);
+    if (s != E2D2_OK) return s;
+    // Ticket words must start at zero; they occupy the first kSampleMaxCtas ints.
+    if (cudaMemsetAsync(scratch, 0, kSampleMaxCtas * sizeof(int), stream) != cudaSuccess) return E2D2_ERR_CUDA;
+    return e2d2_attn_decoder_sample(q_blk, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims, S,
+                                    scratch, kNoAllocScratchBytes, stream);
+}
+
+}  // extern "C"

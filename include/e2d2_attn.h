@@ -42,6 +42,9 @@
 #define E2D2_API
 #endif
 
+/* Size of the scratch array behind e2d2_attn_decoder_sample_noalloc (bytes). */
+#define E2D2_SAMPLE_NOALLOC_MAX_BYTES (((size_t)32) << 20)
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -112,6 +115,27 @@ E2D2_API e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_c
                                      int capacity, int P, const void* k_blk, const void* v_blk,
                                      void* out, float* lse, e2d2_dims dims, int S, void* workspace,
                                      size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Sampling step that allocates nothing: same arguments and result as e2d2_attn_decoder_sample
+ * minus the workspace.  The paper has no counterpart; this exists for callers that cannot
+ * allocate device memory (an engine that gives all of HBM to its own pool and no allocator to
+ * plugins, or a hot path that may not call cudaMalloc because it can synchronise the device).
+ * The split-KV scratch is a file-scope device array of E2D2_SAMPLE_NOALLOC_MAX_BYTES (32 MiB),
+ * reserved on every GPU that loads the library until the process exits.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     once per device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Shapes whose e2d2_attn_decoder_sample_workspace() exceeds the array are rejected with
+ *     E2D2_ERR_WORKSPACE before anything is launched.
+ *   - Every call shares the array: the ticket words are cleared (cudaMemsetAsync) on `stream`
+ *     before each launch.  Calls that overlap on the GPU race; serialise them (one stream).
+ *   - Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+E2D2_API e2d2_status e2d2_attn_decoder_sample_noalloc(const void* q_blk, const void* k_cache,
+                                             const void* v_cache, int capacity, int P,
+                                             const void* k_blk, const void* v_blk, void* out,
+                                             float* lse, e2d2_dims dims, int S, cudaStream_t stream);
 
 /*
  * KV-cache append ([E2D2 notes, sec. 3]: after a block is decoded the encoder absorbs it and
