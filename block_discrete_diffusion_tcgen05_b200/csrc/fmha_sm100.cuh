@@ -39,8 +39,8 @@ enum Mode : int { kEncoder = 0, kDecoderTrain = 1, kDecoderSample = 2 };
 
 constexpr int kBlockM = 128;            // query rows per tile (TMEM lanes)
 constexpr int kBlockN = 128;            // keys per tile
-constexpr int kThreads = 192;           // 6 warps
-constexpr int kSoftmaxThreads = 128;    // warps 2..5
+constexpr int kThreads = 320;           // 10 warps
+constexpr int kSoftmaxThreads = 256;    // warps 2..9
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kSampleMaxCtas = 256;     // upper bound of the sampling grid (workspace sizing)
@@ -106,12 +106,16 @@ struct Smem {
     static constexpr int OFF_K = OFF_Q + 2 * C::TILE_BYTES;
     static constexpr int OFF_V = OFF_K + C::NST * C::TILE_BYTES;
     static constexpr int OFF_O = OFF_V + C::NST * C::TILE_BYTES;
-    static constexpr int O_BYTES = (MODE == kDecoderSample) ? 0 : C::TILE_BYTES;
+    // Train calls stage the output tile for a TMA store, except at d = 128 where the shared
+    // memory is taken by the K/V ring; there rows are stored directly.
+    static constexpr bool STAGE_O = (MODE != kDecoderSample) && (D <= 64);
+    static constexpr int O_BYTES = STAGE_O ? C::TILE_BYTES : 0;
     static constexpr int OFF_BAR = OFF_O + O_BYTES;
     // barriers: k_full[NST], v_full[NST], kv_empty[NST], q_full[2], q_empty[2], s_full[2],
     // p_full[2], o_free[2], pv_done, mma_drain
     static constexpr int NBAR = 3 * C::NST + 2 * 5 + 2;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_RED = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;  // row-max / row-sum exchange
+    static constexpr int OFF_MISC = OFF_RED + 6 * kBlockM * 4;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
 };
@@ -255,6 +259,44 @@ __device__ __forceinline__ uint32_t swz_offset(int r, int u) {
     const uint32_t a = static_cast<uint32_t>(r * RB + u * 16);
     constexpr uint32_t mask = (RB == 128) ? 7u : 3u;
     return a ^ (((a >> 7) & mask) << 4);
+}
+
+// Loads N consecutive fp32 TMEM columns of this thread's lane (N in {16, 32, 64}).
+template <int N>
+__device__ __forceinline__ void load_tmem_cols(uint32_t taddr, float (&o)[N]) {
+    uint32_t r[N];
+    if constexpr (N == 16) {
+        ptx::tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+    } else {
+#pragma unroll
+        for (int c = 0; c < N; c += 32) ptx::tmem_ld32(taddr + c, &r[c]);
+    }
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < N; ++c) o[c] = __uint_as_float(r[c]);
+}
+
+// Multiplies N consecutive fp32 TMEM columns of this thread's lane by f.
+template <int N>
+__device__ __forceinline__ void rescale_tmem_cols(uint32_t taddr, float f) {
+    constexpr int W = N < 32 ? N : 32;
+#pragma unroll
+    for (int c0 = 0; c0 < N; c0 += W) {
+        uint32_t r[W];
+        if constexpr (W == 16) {
+            ptx::tmem_ld16(taddr + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
+        } else {
+            ptx::tmem_ld32(taddr + c0, r);
+        }
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < W; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
+        if constexpr (W == 16) {
+            ptx::tmem_st16(taddr + c0, r);
+        } else {
+            ptx::tmem_st32(taddr + c0, r);
+        }
+    }
 }
 
 template <int D, int MODE>
@@ -473,25 +515,35 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         }
     } else {
         // ------------------------------------------------------------------ softmax warps
-        const int quarter = warp & 3;             // TMEM lane quarter of this warp
-        const int row = quarter * 32 + lane;      // row of the query tile
-        const int stid = threadIdx.x - 64;        // 0..127 within the softmax group
+        // Eight warps.  Warps w and w+4 share TMEM lane quarter (w & 3) -- the same 32 query
+        // rows -- and split every S tile's key columns in two halves of 64; they exchange only
+        // their partial row maxima (shared memory, one pair barrier per tile).  Row sums stay
+        // per half until the epilogue.  Waits never break these loops: every warp takes every
+        // named barrier, so a wait that gives up (device error word set) cannot strand a partner.
+        const int sw = warp - 2;                     // 0..7
+        const int half = sw >> 2;                    // key-column half of this thread
+        const int quarter = warp & 3;                // TMEM lane quarter
+        const int row = quarter * 32 + lane;         // query row of the tile
+        const int stid = threadIdx.x - 64;           // 0..255 within the softmax group
+        const uint32_t pair_bar = 2 + quarter;       // named barrier of the two warps of a quarter
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        constexpr int DH = D / 2;                    // O columns owned by this thread
+        float* red = reinterpret_cast<float*>(smem + SM::OFF_RED);  // [2 parity][2 half][128]
+        float* lsh = red + 4 * kBlockM;                            // [2 half][128]
         const float sl2 = p.scale_log2;
         Scheduler<MODE> sched(p);
         Item it;
         uint32_t gtile = 0, item_idx = 0;
-        bool ok = true;
-        while (ok && sched.next(it)) {
-            // Per-row key intervals [lo, hi) for source 0 and source 1.
+        while (sched.next(it)) {
+            // Per-row key intervals [lo, hi) for source 0 and source 1 (empty for padded rows).
             int lo0, hi0, lo1, hi1;
             bool row_valid;
             if (MODE == kDecoderSample) {
                 row_valid = (it.q_row0 + row) < p.rows_per_unit;
                 lo0 = 0;
-                hi0 = p.P;
+                hi0 = row_valid ? p.P : 0;
                 lo1 = 0;
-                hi1 = p.S;
+                hi1 = row_valid ? p.S : 0;
             } else {
                 const int i_raw = it.q_row0 + row;
                 row_valid = i_raw < p.L;
@@ -499,23 +551,22 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 const int b0 = (i / p.S) * p.S;
                 if (MODE == kEncoder) {
                     lo0 = 0;
-                    hi0 = min(p.L, b0 + p.S);
+                    hi0 = row_valid ? min(p.L, b0 + p.S) : 0;
                     lo1 = 0;
                     hi1 = 0;
                 } else {
                     lo0 = 0;
-                    hi0 = b0;
+                    hi0 = row_valid ? b0 : 0;
                     lo1 = b0;
-                    hi1 = min(p.L, b0 + p.S);
+                    hi1 = row_valid ? min(p.L, b0 + p.S) : 0;
                 }
             }
-            float m = -INFINITY, l = 0.f;
+            float m = -INFINITY, l = 0.f;  // l: this half's partial row sum
             const uint32_t ob = item_idx & 1;
-            const uint32_t o_tmem = tmem_base + lane_off + 256 + ob * D;
+            const uint32_t o_tmem = tmem_base + lane_off + 256 + ob * D + half * DH;
             for (int t = it.t_begin; t < it.t_end; ++t) {
                 const uint32_t sb = gtile & 1;
-                ok = wait_bar_warp(&s_full[sb], (gtile >> 1) & 1, abort_flag, p.err);
-                if (!ok) break;
+                wait_bar_warp(&s_full[sb], (gtile >> 1) & 1, abort_flag, p.err);
                 ptx::tc_fence_after();
                 const TileRef tr = tile_of<MODE>(p, it, t);
                 const int k0 = tr.kt * kBlockN;
@@ -523,31 +574,49 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 const int hi = tr.src ? hi1 : hi0;
                 const int cmin = lo - k0;
                 const int cmax = min(hi - k0, tr.nk16);
+                const int nchunks = (tr.nk16 + 31) / 32;
                 const uint32_t s_tmem = tmem_base + lane_off + sb * 128;
-                uint32_t s_raw[kBlockN];
-                const int nchunks = tr.nk16 / 32 + ((tr.nk16 % 32) ? 1 : 0);
+                // This thread's chunks are a = 2*half + cc.  live: some row of the warp has an
+                // allowed key in the chunk (warp-uniform).
+                uint32_t live = 0;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    if (cc < nchunks) ptx::tmem_ld32(s_tmem + cc * 32, &s_raw[cc * 32]);
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int a = 2 * half + cc;
+                    const bool mine = (a < nchunks) && (cmin < 32 * a + 32) && (cmax > 32 * a);
+                    if (__any_sync(0xffffffffu, mine)) live |= 1u << cc;
                 }
+                uint32_t s_raw[64];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc)
+                    if (live & (1u << cc)) ptx::tmem_ld32(s_tmem + 32 * (2 * half + cc), &s_raw[32 * cc]);
                 ptx::tmem_wait_ld();
-                float s[kBlockN];
+                float s[64];
 #pragma unroll
-                for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(s_raw[c]);
-                float tmax = -INFINITY;
-                if (cmin <= 0 && cmax >= kBlockN) {
+                for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(s_raw[c]);
+                float cmx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < kBlockN; ++c) {
-                        s[c] *= sl2;
-                        tmax = fmaxf(tmax, s[c]);
-                    }
-                } else {
+                for (int cc = 0; cc < 2; ++cc) {
+                    if (live & (1u << cc)) {
+                        const int a = 2 * half + cc;
+                        const bool whole = (cmin <= 32 * a) && (cmax >= 32 * a + 32);
+                        if (!__all_sync(0xffffffffu, whole)) {
 #pragma unroll
-                    for (int c = 0; c < kBlockN; ++c) {
-                        s[c] = (c >= cmin && c < cmax) ? s[c] * sl2 : -INFINITY;
-                        tmax = fmaxf(tmax, s[c]);
+                            for (int c = 0; c < 32; ++c) {
+                                const int col = 32 * a + c;
+                                s[32 * cc + c] = (col >= cmin && col < cmax) ? s[32 * cc + c] : -INFINITY;
+                            }
+                        }
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2)
+                            cmx[cc] = ptx::fmax3(cmx[cc], s[32 * cc + c], s[32 * cc + c + 1]);
                     }
                 }
+                // Row maximum over both halves (raw scores), exchanged through shared memory.
+                const float pmax = fmaxf(cmx[0], cmx[1]);
+                float* rb = red + (gtile & 1) * 2 * kBlockM;
+                rb[half * kBlockM + row] = pmax;
+                ptx::named_barrier_sync(pair_bar, 64);
+                const float tmax = fmaxf(pmax, rb[(1 - half) * kBlockM + row]) * sl2;
                 const float m_new = fmaxf(m, tmax);
                 const bool first = (t == it.t_begin);
                 bool rescale = false;
@@ -558,38 +627,39 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     m = m_new;
                     l *= alpha;
                 }
-                const float m_use = (m == -INFINITY) ? 0.f : m;
-                float rsum = 0.f;
-                uint32_t pk[kBlockN / 2];
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                // P = exp2(s * scale*log2e - m) in bf16 over the first half of this S buffer:
+                // keys 32a..32a+31 -> TMEM columns 16a..16a+15.  Dead chunks are zeros.
+                float sums[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < kBlockN; c += 2) {
-                    const float e0 = ptx::ex2(s[c] - m_use);
-                    const float e1 = ptx::ex2(s[c + 1] - m_use);
-                    rsum += e0 + e1;
-                    pk[c / 2] = ptx::pack_bf16x2(e0, e1);
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int a = 2 * half + cc;
+                    if (a < nchunks) {
+                        uint32_t pk[16];
+                        if (live & (1u << cc)) {
+#pragma unroll
+                            for (int c = 0; c < 32; c += 2) {
+                                const float e0 = ptx::ex2(fmaf(s[32 * cc + c], sl2, neg_m));
+                                const float e1 = ptx::ex2(fmaf(s[32 * cc + c + 1], sl2, neg_m));
+                                sums[(c >> 1) & 3] += e0 + e1;
+                                pk[c / 2] = ptx::pack_bf16x2(e0, e1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                        }
+                        ptx::tmem_st16(s_tmem + 16 * a, pk);
+                    }
                 }
-                l += rsum;
-                // P (bf16) goes over the first half of this S buffer.
-                ptx::tmem_st32(s_tmem, pk);
-                if (tr.nk16 > 64) ptx::tmem_st32(s_tmem + 32, pk + 32);
+                l += (sums[0] + sums[1]) + (sums[2] + sums[3]);
                 if (!first) {
                     // O may only be touched once the previous P.V has landed.
-                    ok = wait_bar_warp(pv_done, (gtile - 1) & 1, abort_flag, p.err);
-                    if (!ok) break;
+                    wait_bar_warp(pv_done, (gtile - 1) & 1, abort_flag, p.err);
                     ptx::tc_fence_after();
                     // tcgen05.ld/st are warp-collective: the warp rescales if any row needs it.
                     if (__any_sync(0xffffffffu, rescale)) {
                         const float f = rescale ? alpha : 1.f;
-#pragma unroll
-                        for (int c0 = 0; c0 < D; c0 += 32) {
-                            uint32_t o[32];
-                            ptx::tmem_ld32(o_tmem + c0, o);
-                            ptx::tmem_wait_ld();
-#pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-                            ptx::tmem_st32(o_tmem + c0, o);
-                        }
+                        rescale_tmem_cols<DH>(o_tmem, f);
                     }
                 }
                 ptx::tmem_wait_st();
@@ -597,39 +667,53 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 ptx::mbar_arrive(&p_full[sb]);
                 ++gtile;
             }
-            if (!ok) break;
             // ---------------------------------------------------------------- epilogue
-            ok = wait_bar_warp(pv_done, (gtile - 1) & 1, abort_flag, p.err);
-            if (!ok) break;
+            wait_bar_warp(pv_done, (gtile - 1) & 1, abort_flag, p.err);
             ptx::tc_fence_after();
-            uint32_t o_raw[D];
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) ptx::tmem_ld32(o_tmem + c0, &o_raw[c0]);
-            ptx::tmem_wait_ld();
-            float o[D];
-#pragma unroll
-            for (int c = 0; c < D; ++c) o[c] = __uint_as_float(o_raw[c]);
+            float o[DH];
+            load_tmem_cols<DH>(o_tmem, o);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&o_free[ob]);
+            // Row sum over both halves.
+            lsh[half * kBlockM + row] = l;
+            ptx::named_barrier_sync(pair_bar, 64);
+            const float l_tot = l + lsh[(1 - half) * kBlockM + row];
+            const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+            const float lse_val = (l_tot > 0.f) ? (m + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
 
-            if (MODE != kDecoderSample) {
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-                // Stage the bf16 tile in the 128B/64B-swizzled layout of the output tensor map.
-                if (stid == 0) ptx::tma_store_wait_read_all();
-                ptx::named_barrier_sync(1, kSoftmaxThreads);
-                uint8_t* stage = smem + SM::OFF_O;
+            if (MODE != kDecoderSample && !SM::STAGE_O) {
+                if (row_valid) {
+                    __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
+                    uint4* dst = reinterpret_cast<uint4*>(
+                        outp + (static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row) * D + half * DH);
 #pragma unroll
-                for (int ch = 0; ch < C::NCH; ++ch) {
-#pragma unroll
-                    for (int u = 0; u < C::RB / 16; ++u) {
-                        const int c = ch * (C::RB / 2) + u * 8;
+                    for (int c = 0; c < DH; c += 8) {
                         uint4 w;
                         w.x = ptx::pack_bf16x2(o[c + 0] * inv_l, o[c + 1] * inv_l);
                         w.y = ptx::pack_bf16x2(o[c + 2] * inv_l, o[c + 3] * inv_l);
                         w.z = ptx::pack_bf16x2(o[c + 4] * inv_l, o[c + 5] * inv_l);
                         w.w = ptx::pack_bf16x2(o[c + 6] * inv_l, o[c + 7] * inv_l);
-                        *reinterpret_cast<uint4*>(stage + ch * C::CHUNK_BYTES + swz_offset<C::RB>(row, u)) = w;
+                        dst[c / 8] = w;
                     }
+                    if (p.lse != nullptr && half == 0)
+                        p.lse[static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row] = lse_val;
+                }
+            } else if (MODE != kDecoderSample) {
+                // Stage the bf16 tile in the swizzled layout of the output tensor map.
+                if (stid == 0) ptx::tma_store_wait_read_all();
+                ptx::named_barrier_sync(1, kSoftmaxThreads);
+                uint8_t* stage = smem + SM::OFF_O;
+#pragma unroll
+                for (int g = 0; g < DH / 8; ++g) {
+                    const int unit = half * (DH / 8) + g;  // 16-byte unit of the D-column row
+                    const int ch = unit / (C::RB / 16);
+                    const int u = unit % (C::RB / 16);
+                    uint4 w;
+                    w.x = ptx::pack_bf16x2(o[8 * g + 0] * inv_l, o[8 * g + 1] * inv_l);
+                    w.y = ptx::pack_bf16x2(o[8 * g + 2] * inv_l, o[8 * g + 3] * inv_l);
+                    w.z = ptx::pack_bf16x2(o[8 * g + 4] * inv_l, o[8 * g + 5] * inv_l);
+                    w.w = ptx::pack_bf16x2(o[8 * g + 6] * inv_l, o[8 * g + 7] * inv_l);
+                    *reinterpret_cast<uint4*>(stage + ch * C::CHUNK_BYTES + swz_offset<C::RB>(row, u)) = w;
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::named_barrier_sync(1, kSoftmaxThreads);
@@ -639,10 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                                           it.q_row0, it.q_z);
                     ptx::tma_store_commit();
                 }
-                if (p.lse != nullptr && row_valid) {
-                    p.lse[static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row] =
-                        (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-                }
+                if (p.lse != nullptr && row_valid && half == 0)
+                    p.lse[static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row] = lse_val;
             } else {
                 // ------------------------------------------------------------ sampling epilogue
                 const int Tu = p.tiles_per_unit;
@@ -650,10 +732,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
                 if (whole) {
                     if (row_valid) {
-                        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-                        uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D);
+                        uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D + half * DH);
 #pragma unroll
-                        for (int c = 0; c < D; c += 8) {
+                        for (int c = 0; c < DH; c += 8) {
                             uint4 w;
                             w.x = ptx::pack_bf16x2(o[c + 0] * inv_l, o[c + 1] * inv_l);
                             w.y = ptx::pack_bf16x2(o[c + 2] * inv_l, o[c + 3] * inv_l);
@@ -661,9 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                             w.w = ptx::pack_bf16x2(o[c + 6] * inv_l, o[c + 7] * inv_l);
                             dst[c / 8] = w;
                         }
-                        if (p.lse != nullptr)
-                            p.lse[it.out_row0 + row] =
-                                (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+                        if (p.lse != nullptr && half == 0) p.lse[it.out_row0 + row] = lse_val;
                     }
                 } else {
                     // Split unit: publish (O, m, l) in this CTA's slot, take a ticket; the last
@@ -678,11 +757,13 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     };
                     float* slot = p.ws_partial + static_cast<size_t>(slot_of(blockIdx.x)) * p.slot_floats;
                     if (row_valid && row < p.rows_cap) {
-                        float4* so = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D);
+                        float4* so = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + half * DH);
 #pragma unroll
-                        for (int c = 0; c < D; c += 4) so[c / 4] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-                        slot[p.rows_cap * D + row] = m;
-                        slot[p.rows_cap * D + p.rows_cap + row] = l;
+                        for (int c = 0; c < DH; c += 4) so[c / 4] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+                        if (half == 0) {
+                            slot[p.rows_cap * D + row] = m;
+                            slot[p.rows_cap * D + p.rows_cap + row] = l_tot;
+                        }
                     }
                     __threadfence();
                     ptx::named_barrier_sync(1, kSoftmaxThreads);
@@ -710,19 +791,20 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                                 ltot += ptx::ex2(__ldcg(sl + p.rows_cap * D + row) - muse) *
                                         __ldcg(sl + p.rows_cap * D + p.rows_cap + row);
                             }
-                            const float inv_l = (ltot > 0.f) ? 1.f / ltot : 0.f;
-                            uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D);
+                            const float inv = (ltot > 0.f) ? 1.f / ltot : 0.f;
+                            uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D + half * DH);
+                            constexpr int CW = DH < 32 ? DH : 32;
 #pragma unroll 1
-                            for (int c0 = 0; c0 < D; c0 += 32) {
-                                float acc[32];
+                            for (int c0 = 0; c0 < DH; c0 += CW) {
+                                float acc[CW];
 #pragma unroll
-                                for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+                                for (int c = 0; c < CW; ++c) acc[c] = 0.f;
                                 for (int c = c_first; c <= c_last; ++c) {
                                     const float* sl = p.ws_partial + static_cast<size_t>(slot_of(c)) * p.slot_floats;
                                     const float w = ptx::ex2(__ldcg(sl + p.rows_cap * D + row) - muse);
-                                    const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + c0);
+                                    const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + half * DH + c0);
 #pragma unroll
-                                    for (int c4 = 0; c4 < 8; ++c4) {
+                                    for (int c4 = 0; c4 < CW / 4; ++c4) {
                                         const float4 v = __ldcg(so + c4);
                                         acc[4 * c4 + 0] += w * v.x;
                                         acc[4 * c4 + 1] += w * v.y;
@@ -731,16 +813,16 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                                     }
                                 }
 #pragma unroll
-                                for (int c = 0; c < 32; c += 8) {
+                                for (int c = 0; c < CW; c += 8) {
                                     uint4 w;
-                                    w.x = ptx::pack_bf16x2(acc[c + 0] * inv_l, acc[c + 1] * inv_l);
-                                    w.y = ptx::pack_bf16x2(acc[c + 2] * inv_l, acc[c + 3] * inv_l);
-                                    w.z = ptx::pack_bf16x2(acc[c + 4] * inv_l, acc[c + 5] * inv_l);
-                                    w.w = ptx::pack_bf16x2(acc[c + 6] * inv_l, acc[c + 7] * inv_l);
+                                    w.x = ptx::pack_bf16x2(acc[c + 0] * inv, acc[c + 1] * inv);
+                                    w.y = ptx::pack_bf16x2(acc[c + 2] * inv, acc[c + 3] * inv);
+                                    w.z = ptx::pack_bf16x2(acc[c + 4] * inv, acc[c + 5] * inv);
+                                    w.w = ptx::pack_bf16x2(acc[c + 6] * inv, acc[c + 7] * inv);
                                     dst[(c0 + c) / 8] = w;
                                 }
                             }
-                            if (p.lse != nullptr)
+                            if (p.lse != nullptr && half == 0)
                                 p.lse[it.out_row0 + row] =
                                     (ltot > 0.f) ? (mmax + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
                         }
@@ -749,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             }
             ++item_idx;
         }
-        if (MODE != kDecoderSample && stid == 0) ptx::tma_store_wait_all();
+        if (SM::STAGE_O && stid == 0) ptx::tma_store_wait_all();
     }
 
     ptx::tc_fence_before();
