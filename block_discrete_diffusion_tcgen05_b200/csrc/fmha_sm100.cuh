@@ -15,16 +15,22 @@
 // computed from tile indices and row numbers; key tiles outside every row's interval are
 // never loaded, and no mask matrix exists anywhere.
 //
-// CTA = 6 warps: warp 0 issues TMA loads, warp 1 owns tensor memory and issues tcgen05.mma,
-// warps 2..5 (one per TMEM lane quarter) run the online softmax and the epilogue.  One
-// 128-row query tile per work item; per key tile of up to 128 keys:
-//     S  = Q K^T        tcgen05.mma, A = Q (smem), B = K (smem, K-major)  -> TMEM (fp32)
-//     P  = exp2(S*c - m) softmax warps, written back over S as bf16      -> TMEM
-//     O += P V          tcgen05.mma, A = P (TMEM), B = V (smem, MN-major) -> TMEM (fp32)
-// S is double-buffered in TMEM so QK^T of tile j+1 overlaps the softmax of tile j; O is
-// double-buffered across work items so the epilogue of one item overlaps the next item.
-// The running max is only moved when it grows by more than 2^8 (log2 units), so O is
-// rescaled rarely; the final normalisation uses the same max and is exact.
+// CTA = 10 warps: warp 0 issues TMA loads, warp 1 owns tensor memory and issues tcgen05.mma,
+// warps 2..9 run the online softmax and the epilogue.  One 128-row query tile per work item;
+// per key tile of up to 128 keys:
+//     S   = Q K^T          tcgen05.mma, A = Q (smem), B = K (smem, K-major)  -> TMEM (fp32)
+//     P   = exp2(S*c - m)  softmax warps, written back over S as bf16      -> TMEM
+//     O_h += P_h V_h       tcgen05.mma, A = P (TMEM), B = V (smem, MN-major) -> TMEM (fp32)
+// The key columns of every tile are split in two halves h (keys 0-63 and 64-127).  Each half
+// has its own softmax warps (the two warps on one TMEM lane quarter: same rows, different
+// keys), its own running max m_h and sum l_h, and its own accumulator O_h; the halves are
+// merged once, in the epilogue (O = sum_h 2^(m_h - M) O_h / sum_h 2^(m_h - M) l_h).  So the
+// two warps never wait for each other inside the key loop, and the tensor core gets two
+// independent P.V accumulation chains to interleave.
+// S is double-buffered in TMEM so QK^T of tile j+1 overlaps the softmax of tile j; at
+// head_dim <= 64 the O pair is double-buffered across work items as well.  A running max is
+// only moved when it grows by more than 2^8 (log2 units), so O is rescaled rarely; the final
+// normalisation uses the same max and is exact.
 #pragma once
 
 #include <cstdint>
@@ -90,6 +96,7 @@ struct Item {
 
 template <int D>
 struct Cfg {
+    static constexpr int NOB = (D <= 64) ? 2 : 1;             // O accumulator sets in TMEM
     static constexpr int RB = (D * 2 < 128) ? D * 2 : 128;  // bytes per smem row of one chunk
     static constexpr int NCH = D * 2 / RB;                   // column chunks per tile
     static constexpr uint32_t SWZ = (RB == 128) ? 2u : 4u;   // 128-byte / 64-byte swizzle
@@ -112,10 +119,10 @@ struct Smem {
     static constexpr int O_BYTES = STAGE_O ? C::TILE_BYTES : 0;
     static constexpr int OFF_BAR = OFF_O + O_BYTES;
     // barriers: k_full[NST], v_full[NST], kv_empty[NST], q_full[2], q_empty[2], s_full[2],
-    // p_full[2], o_free[2], pv_done, mma_drain
-    static constexpr int NBAR = 3 * C::NST + 2 * 5 + 2;
-    static constexpr int OFF_RED = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;  // row-max / row-sum exchange
-    static constexpr int OFF_MISC = OFF_RED + 6 * kBlockM * 4;
+    // p_full[2 S buffers][2 halves], o_free[2], pv_done[2 halves], mma_drain
+    static constexpr int NBAR = 3 * C::NST + 2 + 2 + 2 + 4 + 2 + 2 + 1;
+    static constexpr int OFF_RED = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;  // per-half (m, l) exchange
+    static constexpr int OFF_MISC = OFF_RED + 4 * kBlockM * 4;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
 };
@@ -261,9 +268,53 @@ __device__ __forceinline__ uint32_t swz_offset(int r, int u) {
     return a ^ (((a >> 7) & mask) << 4);
 }
 
+// Issues the two P.V chains of one key tile: O[ob][h] += P[sb][keys of half h] . V[st][same keys]
+// (A = P read from TMEM, B = V MN-major in shared memory), interleaved so the tensor core always
+// has an independent accumulation to work on.  Waits for both halves' P (p_full), for the O set
+// to be free (first tile of an item), and for V.  State is passed by value (nothing in local
+// memory).  started[h]: chain h already holds a partial sum in this item.
+template <class C>
+__device__ __forceinline__ bool issue_pv(uint64_t* p_full, uint64_t* o_free, uint64_t* v_full,
+                                         uint64_t* kv_empty, uint64_t* pv_done, volatile int* abort_flag,
+                                         unsigned int* err, uint32_t tmem_base, uint32_t sV, uint64_t vdesc,
+                                         uint32_t idesc_pv, uint32_t sb, uint32_t st, uint32_t round,
+                                         uint32_t g, uint32_t ob, uint32_t item, uint32_t nk, bool first,
+                                         int D, bool (&started)[2], bool leader) {
+    if (!wait_bar_warp(&p_full[2 * sb + 0], (g >> 1) & 1, abort_flag, err)) return false;
+    if (!wait_bar_warp(&p_full[2 * sb + 1], (g >> 1) & 1, abort_flag, err)) return false;
+    if (first && !wait_bar_warp(&o_free[ob], ((item / C::NOB) & 1) ^ 1, abort_flag, err)) return false;
+    if (!wait_bar_warp(&v_full[st], round & 1, abort_flag, err)) return false;
+    ptx::tc_fence_after();
+    const uint32_t a_tmem = tmem_base + sb * 128;
+    const uint32_t v_base = sV + st * C::TILE_BYTES;
+    const uint32_t nks = nk / 16;  // 16-key steps in this tile; half h owns steps [4h, 4h+4)
+    if (leader) {
+#pragma unroll
+        for (uint32_t i = 0; i < 4; ++i) {
+#pragma unroll
+            for (uint32_t h = 0; h < 2; ++h) {
+                const uint32_t ks = 4 * h + i;
+                if (ks < nks) {
+                    const uint32_t d_tmem = tmem_base + 256 + (ob * 2 + h) * D;
+                    // P of half h sits in the first 32 of that half's own 64 S columns.
+                    ptx::mma_ts(d_tmem, a_tmem + 64 * h + i * 8, vdesc | ((v_base + ks * 16 * C::RB) >> 4),
+                                idesc_pv, (started[h] || i > 0) ? 1u : 0u);
+                }
+            }
+        }
+        ptx::mma_commit(&pv_done[0]);
+        ptx::mma_commit(&pv_done[1]);
+        ptx::mma_commit(&kv_empty[st]);
+    }
+    __syncwarp();
+    if (nks > 0) started[0] = true;
+    if (nks > 4) started[1] = true;
+    return true;
+}
+
 // Loads N consecutive fp32 TMEM columns of this thread's lane (N in {16, 32, 64}).
 template <int N>
-__device__ __forceinline__ void load_tmem_cols(uint32_t taddr, float (&o)[N]) {
+__device__ __forceinline__ void load_tmem_cols(uint32_t taddr, float* o) {
     uint32_t r[N];
     if constexpr (N == 16) {
         ptx::tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
@@ -272,6 +323,7 @@ __device__ __forceinline__ void load_tmem_cols(uint32_t taddr, float (&o)[N]) {
         for (int c = 0; c < N; c += 32) ptx::tmem_ld32(taddr + c, &r[c]);
     }
     ptx::tmem_wait_ld();
+    ptx::reg_fence<N>(r);
 #pragma unroll
     for (int c = 0; c < N; ++c) o[c] = __uint_as_float(r[c]);
 }
@@ -289,6 +341,7 @@ __device__ __forceinline__ void rescale_tmem_cols(uint32_t taddr, float f) {
             ptx::tmem_ld32(taddr + c0, r);
         }
         ptx::tmem_wait_ld();
+        ptx::reg_fence<W>(r);
 #pragma unroll
         for (int c = 0; c < W; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * f);
         if constexpr (W == 16) {
@@ -297,6 +350,15 @@ __device__ __forceinline__ void rescale_tmem_cols(uint32_t taddr, float f) {
             ptx::tmem_st32(taddr + c0, r);
         }
     }
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float* v, float scale) {
+    uint4 w;
+    w.x = ptx::pack_bf16x2(v[0] * scale, v[1] * scale);
+    w.y = ptx::pack_bf16x2(v[2] * scale, v[3] * scale);
+    w.z = ptx::pack_bf16x2(v[4] * scale, v[5] * scale);
+    w.w = ptx::pack_bf16x2(v[6] * scale, v[7] * scale);
+    return w;
 }
 
 template <int D, int MODE>
@@ -313,10 +375,10 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
     uint64_t* q_full = bars + 3 * C::NST;
     uint64_t* q_empty = q_full + 2;
     uint64_t* s_full = q_full + 4;
-    uint64_t* p_full = q_full + 6;
-    uint64_t* o_free = q_full + 8;
-    uint64_t* pv_done = q_full + 10;
-    uint64_t* mma_drain = q_full + 11;
+    uint64_t* p_full = q_full + 6;    // [sb][half]
+    uint64_t* o_free = q_full + 10;   // [ob]
+    uint64_t* pv_done = q_full + 12;  // [half]
+    uint64_t* mma_drain = q_full + 14;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);
     volatile int* bcast = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 16);
@@ -334,10 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             ptx::mbar_init(&q_full[i], 1);
             ptx::mbar_init(&q_empty[i], 1);
             ptx::mbar_init(&s_full[i], 1);
-            ptx::mbar_init(&p_full[i], kSoftmaxThreads);
             ptx::mbar_init(&o_free[i], kSoftmaxThreads);
+            ptx::mbar_init(&pv_done[i], 1);
         }
-        ptx::mbar_init(pv_done, 1);
+        for (int i = 0; i < 4; ++i) ptx::mbar_init(&p_full[i], kSoftmaxThreads / 2);
         ptx::mbar_init(mma_drain, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -358,7 +420,10 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+        // The whole warp walks the schedule (warp-uniform control flow); one elected lane
+        // issues the copies.
+        const bool leader = ptx::elect_one();
+        if (leader) {
             ptx::tma_prefetch_desc(&p.tm_q);
             ptx::tma_prefetch_desc(&p.tm_k0);
             ptx::tma_prefetch_desc(&p.tm_v0);
@@ -366,18 +431,18 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 ptx::tma_prefetch_desc(&p.tm_k1);
                 ptx::tma_prefetch_desc(&p.tm_v1);
             }
-            Scheduler<MODE> sched(p);
-            Item it;
-            uint32_t kv_iter = 0, item_idx = 0;
-            int last_round[C::NST];
-            for (int i = 0; i < C::NST; ++i) last_round[i] = -1;
-            int q_last_round[2] = {-1, -1};
-            bool ok = true;
-            while (ok && sched.next(it)) {
-                const int qb = item_idx & 1;
-                const uint32_t qround = item_idx >> 1;
-                ok = wait_bar(&q_empty[qb], (qround & 1) ^ 1, abort_flag, p.err);
-                if (!ok) break;
+        }
+        __syncwarp();
+        Scheduler<MODE> sched(p);
+        Item it;
+        uint32_t kv_iter = 0, item_idx = 0;
+        bool ok = true;
+        while (ok && sched.next(it)) {
+            const int qb = item_idx & 1;
+            const uint32_t qround = item_idx >> 1;
+            ok = wait_bar_warp(&q_empty[qb], (qround & 1) ^ 1, abort_flag, p.err);
+            if (!ok) break;
+            if (leader) {
                 ptx::mbar_arrive_expect_tx(&q_full[qb], C::TILE_BYTES);
                 for (int ch = 0; ch < C::NCH; ++ch) {
                     uint8_t* dst = smem + SM::OFF_Q + qb * C::TILE_BYTES + ch * C::CHUNK_BYTES;
@@ -386,13 +451,16 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     else
                         ptx::tma_load_3d(&p.tm_q, &q_full[qb], dst, ch * (C::RB / 2), it.q_y, it.q_z);
                 }
-                q_last_round[qb] = static_cast<int>(qround);
-                for (int t = it.t_begin; t < it.t_end && ok; ++t) {
-                    const int st = kv_iter % C::NST;
-                    const uint32_t round = kv_iter / C::NST;
-                    ok = wait_bar(&kv_empty[st], (round & 1) ^ 1, abort_flag, p.err);
-                    if (!ok) break;
-                    const TileRef tr = tile_of<MODE>(p, it, t);
+            }
+            __syncwarp();
+            ++item_idx;
+            for (int t = it.t_begin; t < it.t_end; ++t) {
+                const int st = kv_iter % C::NST;
+                const uint32_t round = kv_iter / C::NST;
+                ok = wait_bar_warp(&kv_empty[st], (round & 1) ^ 1, abort_flag, p.err);
+                if (!ok) break;
+                const TileRef tr = tile_of<MODE>(p, it, t);
+                if (leader) {
                     const CUtensorMap* mk = tr.src ? &p.tm_k1 : &p.tm_k0;
                     const CUtensorMap* mv = tr.src ? &p.tm_v1 : &p.tm_v0;
                     const uint32_t bytes = static_cast<uint32_t>(tr.box_rows) * D * 2;
@@ -406,130 +474,114 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         ptx::tma_load_3d(mv, &v_full[st],
                                          smem + SM::OFF_V + st * C::TILE_BYTES + ch * C::CHUNK_BYTES,
                                          ch * (C::RB / 2), tr.kt * kBlockN, it.kv_z);
-                    last_round[st] = static_cast<int>(round);
-                    ++kv_iter;
                 }
-                ++item_idx;
-            }
-            // Never leave with copies in flight: wait for the last load of every buffer.
-            for (int i = 0; i < C::NST; ++i) {
-                if (last_round[i] >= 0) {
-                    const uint32_t par = static_cast<uint32_t>(last_round[i]) & 1u;
-                    volatile int no_abort = 0;
-                    wait_bar(&k_full[i], par, &no_abort, p.err);
-                    wait_bar(&v_full[i], par, &no_abort, p.err);
-                }
-            }
-            for (int i = 0; i < 2; ++i) {
-                if (q_last_round[i] >= 0) {
-                    volatile int no_abort = 0;
-                    wait_bar(&q_full[i], static_cast<uint32_t>(q_last_round[i]) & 1u, &no_abort, p.err);
-                }
+                __syncwarp();
+                ++kv_iter;
             }
         }
+        // Never leave with copies in flight: wait for the last load of every buffer (the last
+        // NST K/V loads and the last two Q loads).
+        volatile int no_abort = 0;
+        const uint32_t first_live = kv_iter > static_cast<uint32_t>(C::NST) ? kv_iter - C::NST : 0u;
+        for (uint32_t i = first_live; i < kv_iter; ++i) {
+            wait_bar_warp(&k_full[i % C::NST], (i / C::NST) & 1u, &no_abort, p.err);
+            wait_bar_warp(&v_full[i % C::NST], (i / C::NST) & 1u, &no_abort, p.err);
+        }
+        for (uint32_t i = item_idx > 2u ? item_idx - 2u : 0u; i < item_idx; ++i)
+            wait_bar_warp(&q_full[i & 1u], (i >> 1) & 1u, &no_abort, p.err);
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            Scheduler<MODE> sched(p);
-            Item it;
-            uint32_t kv_iter = 0, gtile = 0, item_idx = 0;
-            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBlockM, D, true);
-            // Pending P.V of the previous tile (issued after the next QK^T so that the tensor
-            // core computes S_{j+1} while the softmax warps work on tile j).
-            bool have_pv = false;
-            uint32_t pv_sb = 0, pv_st = 0, pv_round = 0, pv_g = 0, pv_ob = 0, pv_item = 0;
-            int pv_nk = 0;
-            bool pv_first = false;
-            bool ok = true;
-
-            auto issue_pv = [&]() -> bool {
-                if (!wait_bar(&p_full[pv_sb], (pv_g >> 1) & 1, abort_flag, p.err)) return false;
-                if (pv_first &&
-                    !wait_bar(&o_free[pv_ob], ((pv_item >> 1) & 1) ^ 1, abort_flag, p.err))
-                    return false;
-                if (!wait_bar(&v_full[pv_st], pv_round & 1, abort_flag, p.err)) return false;
-                ptx::tc_fence_after();
-                const uint32_t d_tmem = tmem_base + 256 + pv_ob * D;
-                const uint32_t a_tmem = tmem_base + pv_sb * 128;
-                const uint32_t v_base = sV + pv_st * C::TILE_BYTES;
-                for (int ks = 0; ks < pv_nk / 16; ++ks) {
-                    const uint64_t bdesc =
-                        ptx::smem_desc(v_base + ks * 16 * C::RB, C::CHUNK_BYTES, 8 * C::RB, C::SWZ);
-                    ptx::mma_ts(d_tmem, a_tmem + ks * 8, bdesc, idesc_pv,
-                                (pv_first && ks == 0) ? 0u : 1u);
-                }
-                ptx::mma_commit(&kv_empty[pv_st]);
-                ptx::mma_commit(pv_done);
-                return true;
-            };
-
-            while (ok && sched.next(it)) {
-                const int qb = item_idx & 1;
-                ok = wait_bar(&q_full[qb], (item_idx >> 1) & 1, abort_flag, p.err);
+        // The whole warp walks the schedule, so descriptors and TMEM addresses are warp-uniform;
+        // one elected lane issues tcgen05.mma / tcgen05.commit.
+        const bool leader = ptx::elect_one();
+        Scheduler<MODE> sched(p);
+        Item it;
+        uint32_t kv_iter = 0, gtile = 0, item_idx = 0;
+        // Descriptor bits without the start address (added per MMA).
+        const uint64_t kdesc = ptx::smem_desc(0, 16, 8 * C::RB, C::SWZ);             // Q, K: K-major
+        const uint64_t vdesc = ptx::smem_desc(0, C::CHUNK_BYTES, 8 * C::RB, C::SWZ);  // V: MN-major
+        constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBlockM, D, true);
+        // The P.V of tile j is issued after the QK^T of tile j+1, so the tensor core computes
+        // S_{j+1} while the softmax warps work on tile j.
+        bool have_pv = false, pv_first = false;
+        bool started[2] = {false, false};  // chains of the item the pending P.V belongs to
+        uint32_t pv_sb = 0, pv_st = 0, pv_round = 0, pv_g = 0, pv_ob = 0, pv_item = 0, pv_nk = 0;
+        bool ok = true;
+        while (ok && sched.next(it)) {
+            const int qb = item_idx & 1;
+            ok = wait_bar_warp(&q_full[qb], (item_idx >> 1) & 1, abort_flag, p.err);
+            if (!ok) break;
+            const uint32_t q_base = sQ + qb * C::TILE_BYTES;
+            if (it.t_end <= it.t_begin && leader) ptx::mma_commit(&q_empty[qb]);
+            for (int t = it.t_begin; t < it.t_end; ++t) {
+                const uint32_t st = kv_iter % C::NST;
+                const uint32_t round = kv_iter / C::NST;
+                ok = wait_bar_warp(&k_full[st], round & 1, abort_flag, p.err);
                 if (!ok) break;
-                const uint32_t q_base = sQ + qb * C::TILE_BYTES;
-                if (it.t_end <= it.t_begin) ptx::mma_commit(&q_empty[qb]);
-                for (int t = it.t_begin; t < it.t_end; ++t) {
-                    const uint32_t st = kv_iter % C::NST;
-                    const uint32_t round = kv_iter / C::NST;
-                    ok = wait_bar(&k_full[st], round & 1, abort_flag, p.err);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                    const TileRef tr = tile_of<MODE>(p, it, t);
-                    const uint32_t sb = gtile & 1;
-                    const uint32_t idesc_qk = ptx::idesc_bf16_f32(kBlockM, tr.nk16, false);
-                    const uint32_t k_base = sK + st * C::TILE_BYTES;
+                ptx::tc_fence_after();
+                const TileRef tr = tile_of<MODE>(p, it, t);
+                const uint32_t sb = gtile & 1;
+                const uint32_t idesc_qk = ptx::idesc_bf16_f32(kBlockM, tr.nk16, false);
+                const uint32_t k_base = sK + st * C::TILE_BYTES;
+                if (leader) {
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
-                        const int ch = ks / C::KSTEPS_PER_CHUNK;
-                        const uint32_t off = ch * C::CHUNK_BYTES + (ks % C::KSTEPS_PER_CHUNK) * 32;
-                        const uint64_t adesc = ptx::smem_desc(q_base + off, 16, 8 * C::RB, C::SWZ);
-                        const uint64_t bdesc = ptx::smem_desc(k_base + off, 16, 8 * C::RB, C::SWZ);
-                        ptx::mma_ss(tmem_base + sb * 128, adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+                        const uint32_t off = (ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
+                                             (ks % C::KSTEPS_PER_CHUNK) * 32;
+                        ptx::mma_ss(tmem_base + sb * 128, kdesc | ((q_base + off) >> 4),
+                                    kdesc | ((k_base + off) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
                     }
                     ptx::mma_commit(&s_full[sb]);
                     if (t == it.t_end - 1) ptx::mma_commit(&q_empty[qb]);
-                    if (have_pv) {
-                        ok = issue_pv();
-                        if (!ok) break;
-                    }
-                    have_pv = true;
-                    pv_sb = sb;
-                    pv_st = st;
-                    pv_round = round;
-                    pv_g = gtile;
-                    pv_ob = item_idx & 1;
-                    pv_item = item_idx;
-                    pv_nk = tr.nk16;
-                    pv_first = (t == it.t_begin);
-                    ++kv_iter;
-                    ++gtile;
                 }
-                ++item_idx;
+                __syncwarp();
+                if (have_pv) {
+                    ok = issue_pv<C>(p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err, tmem_base, sV,
+                                     vdesc, idesc_pv, pv_sb, pv_st, pv_round, pv_g, pv_ob, pv_item, pv_nk,
+                                     pv_first, D, started, leader);
+                    if (!ok) break;
+                }
+                // started[] follows the item of the pending P.V: a new item starts both chains afresh.
+                if (t == it.t_begin) started[0] = started[1] = false;
+                have_pv = true;
+                pv_sb = sb;
+                pv_st = st;
+                pv_round = round;
+                pv_g = gtile;
+                pv_ob = item_idx % C::NOB;
+                pv_item = item_idx;
+                pv_nk = tr.nk16;
+                pv_first = (t == it.t_begin);
+                ++kv_iter;
+                ++gtile;
             }
-            if (ok && have_pv) issue_pv();
-            // Drain: every MMA issued by this thread completes before TMEM is released.
-            ptx::mma_commit(mma_drain);
-            volatile int no_abort = 0;
-            wait_bar(mma_drain, 0, &no_abort, p.err);
+            ++item_idx;
         }
+        if (ok && have_pv)
+            issue_pv<C>(p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err, tmem_base, sV, vdesc,
+                        idesc_pv, pv_sb, pv_st, pv_round, pv_g, pv_ob, pv_item, pv_nk, pv_first, D, started,
+                        leader);
+        // Drain: every MMA issued by this warp completes before TMEM is released.
+        if (leader) ptx::mma_commit(mma_drain);
+        __syncwarp();
+        volatile int no_abort = 0;
+        wait_bar_warp(mma_drain, 0, &no_abort, p.err);
     } else {
         // ------------------------------------------------------------------ softmax warps
         // Eight warps.  Warps w and w+4 share TMEM lane quarter (w & 3) -- the same 32 query
-        // rows -- and split every S tile's key columns in two halves of 64; they exchange only
-        // their partial row maxima (shared memory, one pair barrier per tile).  Row sums stay
-        // per half until the epilogue.  Waits never break these loops: every warp takes every
-        // named barrier, so a wait that gives up (device error word set) cannot strand a partner.
+        // rows -- and own the two key halves of every S tile (keys 0-63 / 64-127) with their
+        // own running max, sum and O accumulator.  They meet only in the epilogue.  Waits never
+        // break these loops: every warp takes every named barrier, so a wait that gives up
+        // (device error word set) cannot strand another warp.
         const int sw = warp - 2;                     // 0..7
-        const int half = sw >> 2;                    // key-column half of this thread
+        const int half = sw >> 2;                    // key half of this thread
         const int quarter = warp & 3;                // TMEM lane quarter
         const int row = quarter * 32 + lane;         // query row of the tile
         const int stid = threadIdx.x - 64;           // 0..255 within the softmax group
         const uint32_t pair_bar = 2 + quarter;       // named barrier of the two warps of a quarter
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        constexpr int DH = D / 2;                    // O columns owned by this thread
-        float* red = reinterpret_cast<float*>(smem + SM::OFF_RED);  // [2 parity][2 half][128]
-        float* lsh = red + 4 * kBlockM;                            // [2 half][128]
+        constexpr int DH = D / 2;                    // output columns written by this thread
+        float* xch = reinterpret_cast<float*>(smem + SM::OFF_RED);  // [m|l][half][128]
         const float sl2 = p.scale_log2;
         Scheduler<MODE> sched(p);
         Item it;
@@ -561,9 +613,10 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     hi1 = row_valid ? min(p.L, b0 + p.S) : 0;
                 }
             }
-            float m = -INFINITY, l = 0.f;  // l: this half's partial row sum
-            const uint32_t ob = item_idx & 1;
-            const uint32_t o_tmem = tmem_base + lane_off + 256 + ob * D + half * DH;
+            float m = -INFINITY, l = 0.f;  // this half's running max (log2 units) and sum
+            const uint32_t ob = item_idx % C::NOB;
+            const uint32_t o_base = tmem_base + lane_off + 256 + ob * 2 * D;  // O[ob][0]; O[ob][1] at +D
+            const uint32_t o_mine = o_base + half * D;
             for (int t = it.t_begin; t < it.t_end; ++t) {
                 const uint32_t sb = gtile & 1;
                 wait_bar_warp(&s_full[sb], (gtile >> 1) & 1, abort_flag, p.err);
@@ -590,6 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 for (int cc = 0; cc < 2; ++cc)
                     if (live & (1u << cc)) ptx::tmem_ld32(s_tmem + 32 * (2 * half + cc), &s_raw[32 * cc]);
                 ptx::tmem_wait_ld();
+                ptx::reg_fence<64>(s_raw);
                 float s[64];
 #pragma unroll
                 for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(s_raw[c]);
@@ -611,13 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                             cmx[cc] = ptx::fmax3(cmx[cc], s[32 * cc + c], s[32 * cc + c + 1]);
                     }
                 }
-                // Row maximum over both halves (raw scores), exchanged through shared memory.
-                const float pmax = fmaxf(cmx[0], cmx[1]);
-                float* rb = red + (gtile & 1) * 2 * kBlockM;
-                rb[half * kBlockM + row] = pmax;
-                ptx::named_barrier_sync(pair_bar, 64);
-                const float tmax = fmaxf(pmax, rb[(1 - half) * kBlockM + row]) * sl2;
-                const float m_new = fmaxf(m, tmax);
+                const float m_new = fmaxf(m, fmaxf(cmx[0], cmx[1]) * sl2);
                 const bool first = (t == it.t_begin);
                 bool rescale = false;
                 float alpha = 1.f;
@@ -628,8 +676,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     l *= alpha;
                 }
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                // P = exp2(s * scale*log2e - m) in bf16 over the first half of this S buffer:
-                // keys 32a..32a+31 -> TMEM columns 16a..16a+15.  Dead chunks are zeros.
+                // P = exp2(s * scale*log2e - m) in bf16, written over this half's own S columns
+                // (which no other warp reads): keys 64h + 32cc .. +31 -> TMEM columns
+                // 64h + 16cc .. +15.  Dead chunks are zeros.
                 float sums[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
@@ -648,184 +697,180 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
 #pragma unroll
                             for (int c = 0; c < 16; ++c) pk[c] = 0u;
                         }
-                        ptx::tmem_st16(s_tmem + 16 * a, pk);
+                        ptx::tmem_st16(s_tmem + 64 * half + 16 * cc, pk);
                     }
                 }
                 l += (sums[0] + sums[1]) + (sums[2] + sums[3]);
                 if (!first) {
-                    // O may only be touched once the previous P.V has landed.
-                    wait_bar_warp(pv_done, (gtile - 1) & 1, abort_flag, p.err);
+                    // This half's O may only be touched once its previous P.V has landed.
+                    wait_bar_warp(&pv_done[half], (gtile - 1) & 1, abort_flag, p.err);
                     ptx::tc_fence_after();
                     // tcgen05.ld/st are warp-collective: the warp rescales if any row needs it.
-                    if (__any_sync(0xffffffffu, rescale)) {
-                        const float f = rescale ? alpha : 1.f;
-                        rescale_tmem_cols<DH>(o_tmem, f);
-                    }
+                    if (__any_sync(0xffffffffu, rescale)) rescale_tmem_cols<D>(o_mine, rescale ? alpha : 1.f);
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(&p_full[sb]);
+                ptx::mbar_arrive(&p_full[2 * sb + half]);
                 ++gtile;
             }
             // ---------------------------------------------------------------- epilogue
-            wait_bar_warp(pv_done, (gtile - 1) & 1, abort_flag, p.err);
-            ptx::tc_fence_after();
-            float o[DH];
-            load_tmem_cols<DH>(o_tmem, o);
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&o_free[ob]);
-            // Row sum over both halves.
-            lsh[half * kBlockM + row] = l;
+            // Merge the two halves: exchange (m, l) with the partner warp of this quarter.
+            xch[half * kBlockM + row] = m;
+            xch[(2 + half) * kBlockM + row] = l;
             ptx::named_barrier_sync(pair_bar, 64);
-            const float l_tot = l + lsh[(1 - half) * kBlockM + row];
+            const float m_o = xch[(1 - half) * kBlockM + row];
+            const float l_o = xch[(3 - half) * kBlockM + row];
+            ptx::named_barrier_sync(pair_bar, 64);  // partner done reading before the next write
+            const float m_a = half == 0 ? m : m_o, l_a = half == 0 ? l : l_o;
+            const float m_b = half == 0 ? m_o : m, l_b = half == 0 ? l_o : l;
+            const float mx = fmaxf(m_a, m_b);
+            const float w_a = (l_a > 0.f) ? ptx::ex2(m_a - mx) : 0.f;
+            const float w_b = (l_b > 0.f) ? ptx::ex2(m_b - mx) : 0.f;
+            const float l_tot = l_a * w_a + l_b * w_b;
             const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
-            const float lse_val = (l_tot > 0.f) ? (m + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+            const float lse_val = (l_tot > 0.f) ? (mx + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+            // Both chains' last P.V must have landed (this thread reads its columns of both).
+            wait_bar_warp(&pv_done[0], (gtile - 1) & 1, abort_flag, p.err);
+            wait_bar_warp(&pv_done[1], (gtile - 1) & 1, abort_flag, p.err);
+            ptx::tc_fence_after();
 
-            if (MODE != kDecoderSample && !SM::STAGE_O) {
-                if (row_valid) {
-                    __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
-                    uint4* dst = reinterpret_cast<uint4*>(
-                        outp + (static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row) * D + half * DH);
-#pragma unroll
-                    for (int c = 0; c < DH; c += 8) {
-                        uint4 w;
-                        w.x = ptx::pack_bf16x2(o[c + 0] * inv_l, o[c + 1] * inv_l);
-                        w.y = ptx::pack_bf16x2(o[c + 2] * inv_l, o[c + 3] * inv_l);
-                        w.z = ptx::pack_bf16x2(o[c + 4] * inv_l, o[c + 5] * inv_l);
-                        w.w = ptx::pack_bf16x2(o[c + 6] * inv_l, o[c + 7] * inv_l);
-                        dst[c / 8] = w;
-                    }
-                    if (p.lse != nullptr && half == 0)
-                        p.lse[static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row] = lse_val;
-                }
-            } else if (MODE != kDecoderSample) {
-                // Stage the bf16 tile in the swizzled layout of the output tensor map.
+            constexpr int CW = DH < 32 ? DH : 32;   // columns merged per step
+            __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
+            const int Tu = p.tiles_per_unit;
+            const bool whole = (MODE != kDecoderSample) || (it.t_begin == 0 && it.t_end == Tu);
+            float* slot = nullptr;
+            int c_first = 0, c_last = 0;
+            long long ubeg = 0;
+            if (MODE == kDecoderSample && !whole) {
+                ubeg = static_cast<long long>(it.q_z) * Tu;
+                c_first = owner_cta(ubeg, p.total_tiles, gridDim.x);
+                c_last = owner_cta(ubeg + Tu - 1, p.total_tiles, gridDim.x);
+                const int my_slot = (range_begin(blockIdx.x, p.total_tiles, gridDim.x) >= ubeg) ? 2 * blockIdx.x
+                                                                                                : 2 * blockIdx.x + 1;
+                slot = p.ws_partial + static_cast<size_t>(my_slot) * p.slot_floats;
+            }
+            uint8_t* stage = smem + SM::OFF_O;
+            if (SM::STAGE_O) {
                 if (stid == 0) ptx::tma_store_wait_read_all();
                 ptx::named_barrier_sync(1, kSoftmaxThreads);
-                uint8_t* stage = smem + SM::OFF_O;
+            }
 #pragma unroll
-                for (int g = 0; g < DH / 8; ++g) {
-                    const int unit = half * (DH / 8) + g;  // 16-byte unit of the D-column row
-                    const int ch = unit / (C::RB / 16);
-                    const int u = unit % (C::RB / 16);
-                    uint4 w;
-                    w.x = ptx::pack_bf16x2(o[8 * g + 0] * inv_l, o[8 * g + 1] * inv_l);
-                    w.y = ptx::pack_bf16x2(o[8 * g + 2] * inv_l, o[8 * g + 3] * inv_l);
-                    w.z = ptx::pack_bf16x2(o[8 * g + 4] * inv_l, o[8 * g + 5] * inv_l);
-                    w.w = ptx::pack_bf16x2(o[8 * g + 6] * inv_l, o[8 * g + 7] * inv_l);
-                    *reinterpret_cast<uint4*>(stage + ch * C::CHUNK_BYTES + swz_offset<C::RB>(row, u)) = w;
+            for (int c0 = 0; c0 < DH; c0 += CW) {
+                float oa[CW], obv[CW], o[CW];
+                load_tmem_cols<CW>(o_base + half * DH + c0, oa);
+                load_tmem_cols<CW>(o_base + D + half * DH + c0, obv);
+#pragma unroll
+                for (int c = 0; c < CW; ++c)
+                    o[c] = (w_a > 0.f ? oa[c] * w_a : 0.f) + (w_b > 0.f ? obv[c] * w_b : 0.f);
+                const int col = half * DH + c0;  // first output column of this step
+                if (SM::STAGE_O) {
+                    // bf16 tile in the swizzled layout of the output tensor map
+#pragma unroll
+                    for (int g = 0; g < CW / 8; ++g) {
+                        const int unit = (col + 8 * g) / 8;
+                        const int ch = unit / (C::RB / 16);
+                        const int u = unit % (C::RB / 16);
+                        *reinterpret_cast<uint4*>(stage + ch * C::CHUNK_BYTES + swz_offset<C::RB>(row, u)) =
+                            pack8_bf16(&o[8 * g], inv_l);
+                    }
+                } else if (MODE != kDecoderSample || whole) {
+                    if (row_valid) {
+                        const size_t r = (MODE == kDecoderSample)
+                                             ? static_cast<size_t>(it.out_row0 + row)
+                                             : static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row;
+                        uint4* dst = reinterpret_cast<uint4*>(outp + r * D + col);
+#pragma unroll
+                        for (int c = 0; c < CW; c += 8) dst[c / 8] = pack8_bf16(&o[c], inv_l);
+                    }
+                } else if (row_valid && row < p.rows_cap) {
+                    float4* so = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + col);
+#pragma unroll
+                    for (int c = 0; c < CW; c += 4) so[c / 4] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
                 }
-                ptx::fence_proxy_async_smem();
-                ptx::named_barrier_sync(1, kSoftmaxThreads);
-                if (stid == 0) {
-                    for (int ch = 0; ch < C::NCH; ++ch)
-                        ptx::tma_store_3d(&p.tm_o, stage + ch * C::CHUNK_BYTES, ch * (C::RB / 2),
-                                          it.q_row0, it.q_z);
-                    ptx::tma_store_commit();
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&o_free[ob]);
+
+            if (MODE != kDecoderSample) {
+                if (SM::STAGE_O) {
+                    ptx::fence_proxy_async_smem();
+                    ptx::named_barrier_sync(1, kSoftmaxThreads);
+                    if (stid == 0) {
+                        for (int ch = 0; ch < C::NCH; ++ch)
+                            ptx::tma_store_3d(&p.tm_o, stage + ch * C::CHUNK_BYTES, ch * (C::RB / 2),
+                                              it.q_row0, it.q_z);
+                        ptx::tma_store_commit();
+                    }
                 }
                 if (p.lse != nullptr && row_valid && half == 0)
                     p.lse[static_cast<size_t>(it.q_z) * p.L + it.q_row0 + row] = lse_val;
+            } else if (whole) {
+                if (p.lse != nullptr && row_valid && half == 0) p.lse[it.out_row0 + row] = lse_val;
             } else {
-                // ------------------------------------------------------------ sampling epilogue
-                const int Tu = p.tiles_per_unit;
-                const bool whole = (it.t_begin == 0 && it.t_end == Tu);
-                __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
-                if (whole) {
-                    if (row_valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D + half * DH);
-#pragma unroll
-                        for (int c = 0; c < DH; c += 8) {
-                            uint4 w;
-                            w.x = ptx::pack_bf16x2(o[c + 0] * inv_l, o[c + 1] * inv_l);
-                            w.y = ptx::pack_bf16x2(o[c + 2] * inv_l, o[c + 3] * inv_l);
-                            w.z = ptx::pack_bf16x2(o[c + 4] * inv_l, o[c + 5] * inv_l);
-                            w.w = ptx::pack_bf16x2(o[c + 6] * inv_l, o[c + 7] * inv_l);
-                            dst[c / 8] = w;
-                        }
-                        if (p.lse != nullptr && half == 0) p.lse[it.out_row0 + row] = lse_val;
-                    }
-                } else {
-                    // Split unit: publish (O, m, l) in this CTA's slot, take a ticket; the last
-                    // CTA of the unit merges every slot.
-                    const long long T = p.total_tiles;
-                    const int grid = gridDim.x;
-                    const long long ubeg = static_cast<long long>(it.q_z) * Tu;
-                    const int c_first = owner_cta(ubeg, T, grid);
-                    const int c_last = owner_cta(ubeg + Tu - 1, T, grid);
-                    auto slot_of = [&](int c) -> int {
-                        return (range_begin(c, T, grid) >= ubeg) ? 2 * c : 2 * c + 1;
-                    };
-                    float* slot = p.ws_partial + static_cast<size_t>(slot_of(blockIdx.x)) * p.slot_floats;
-                    if (row_valid && row < p.rows_cap) {
-                        float4* so = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + half * DH);
-#pragma unroll
-                        for (int c = 0; c < DH; c += 4) so[c / 4] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-                        if (half == 0) {
-                            slot[p.rows_cap * D + row] = m;
-                            slot[p.rows_cap * D + p.rows_cap + row] = l_tot;
-                        }
-                    }
+                // Split unit: (O, m, l) of this CTA is in its slot; take a ticket; the last CTA of
+                // the unit merges every slot.
+                if (row_valid && row < p.rows_cap && half == 0) {
+                    slot[p.rows_cap * D + row] = mx;
+                    slot[p.rows_cap * D + p.rows_cap + row] = l_tot;
+                }
+                __threadfence();
+                ptx::named_barrier_sync(1, kSoftmaxThreads);
+                if (stid == 0) {
+                    const int ticket = atomicAdd(&p.ws_tickets[c_first], 1);
+                    const int last = (ticket == c_last - c_first) ? 1 : 0;
+                    if (last) p.ws_tickets[c_first] = 0;
+                    *bcast = last;
+                }
+                ptx::named_barrier_sync(1, kSoftmaxThreads);
+                const int is_last = *bcast;
+                ptx::named_barrier_sync(1, kSoftmaxThreads);
+                if (is_last) {
                     __threadfence();
-                    ptx::named_barrier_sync(1, kSoftmaxThreads);
-                    if (stid == 0) {
-                        const int ticket = atomicAdd(&p.ws_tickets[c_first], 1);
-                        const int last = (ticket == c_last - c_first) ? 1 : 0;
-                        if (last) p.ws_tickets[c_first] = 0;
-                        *bcast = last;
-                    }
-                    ptx::named_barrier_sync(1, kSoftmaxThreads);
-                    const int is_last = *bcast;
-                    ptx::named_barrier_sync(1, kSoftmaxThreads);
-                    if (is_last) {
-                        __threadfence();
-                        if (row_valid && row < p.rows_cap) {
-                            float mmax = -INFINITY;
-                            for (int c = c_first; c <= c_last; ++c) {
-                                const float* sl = p.ws_partial + static_cast<size_t>(slot_of(c)) * p.slot_floats;
-                                mmax = fmaxf(mmax, __ldcg(sl + p.rows_cap * D + row));
-                            }
-                            const float muse = (mmax == -INFINITY) ? 0.f : mmax;
-                            float ltot = 0.f;
-                            for (int c = c_first; c <= c_last; ++c) {
-                                const float* sl = p.ws_partial + static_cast<size_t>(slot_of(c)) * p.slot_floats;
-                                ltot += ptx::ex2(__ldcg(sl + p.rows_cap * D + row) - muse) *
-                                        __ldcg(sl + p.rows_cap * D + p.rows_cap + row);
-                            }
-                            const float inv = (ltot > 0.f) ? 1.f / ltot : 0.f;
-                            uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D + half * DH);
-                            constexpr int CW = DH < 32 ? DH : 32;
-#pragma unroll 1
-                            for (int c0 = 0; c0 < DH; c0 += CW) {
-                                float acc[CW];
-#pragma unroll
-                                for (int c = 0; c < CW; ++c) acc[c] = 0.f;
-                                for (int c = c_first; c <= c_last; ++c) {
-                                    const float* sl = p.ws_partial + static_cast<size_t>(slot_of(c)) * p.slot_floats;
-                                    const float w = ptx::ex2(__ldcg(sl + p.rows_cap * D + row) - muse);
-                                    const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + half * DH + c0);
-#pragma unroll
-                                    for (int c4 = 0; c4 < CW / 4; ++c4) {
-                                        const float4 v = __ldcg(so + c4);
-                                        acc[4 * c4 + 0] += w * v.x;
-                                        acc[4 * c4 + 1] += w * v.y;
-                                        acc[4 * c4 + 2] += w * v.z;
-                                        acc[4 * c4 + 3] += w * v.w;
-                                    }
-                                }
-#pragma unroll
-                                for (int c = 0; c < CW; c += 8) {
-                                    uint4 w;
-                                    w.x = ptx::pack_bf16x2(acc[c + 0] * inv, acc[c + 1] * inv);
-                                    w.y = ptx::pack_bf16x2(acc[c + 2] * inv, acc[c + 3] * inv);
-                                    w.z = ptx::pack_bf16x2(acc[c + 4] * inv, acc[c + 5] * inv);
-                                    w.w = ptx::pack_bf16x2(acc[c + 6] * inv, acc[c + 7] * inv);
-                                    dst[(c0 + c) / 8] = w;
-                                }
-                            }
-                            if (p.lse != nullptr && half == 0)
-                                p.lse[it.out_row0 + row] =
-                                    (ltot > 0.f) ? (mmax + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
+                    if (row_valid && row < p.rows_cap) {
+                        const long long T = p.total_tiles;
+                        const int grid = gridDim.x;
+                        auto slot_ptr = [&](int c) -> const float* {
+                            const int si = (range_begin(c, T, grid) >= ubeg) ? 2 * c : 2 * c + 1;
+                            return p.ws_partial + static_cast<size_t>(si) * p.slot_floats;
+                        };
+                        float mmax = -INFINITY;
+                        for (int c = c_first; c <= c_last; ++c)
+                            mmax = fmaxf(mmax, __ldcg(slot_ptr(c) + p.rows_cap * D + row));
+                        const float muse = (mmax == -INFINITY) ? 0.f : mmax;
+                        float ltot = 0.f;
+                        for (int c = c_first; c <= c_last; ++c) {
+                            const float* sl = slot_ptr(c);
+                            const float mw = __ldcg(sl + p.rows_cap * D + row);
+                            if (mw != -INFINITY) ltot += ptx::ex2(mw - muse) * __ldcg(sl + p.rows_cap * D + p.rows_cap + row);
                         }
+                        const float inv = (ltot > 0.f) ? 1.f / ltot : 0.f;
+                        uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D + half * DH);
+#pragma unroll 1
+                        for (int c0 = 0; c0 < DH; c0 += CW) {
+                            float acc[CW];
+#pragma unroll
+                            for (int c = 0; c < CW; ++c) acc[c] = 0.f;
+                            for (int c = c_first; c <= c_last; ++c) {
+                                const float* sl = slot_ptr(c);
+                                const float mw = __ldcg(sl + p.rows_cap * D + row);
+                                if (mw == -INFINITY) continue;
+                                const float w = ptx::ex2(mw - muse);
+                                const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + half * DH + c0);
+#pragma unroll
+                                for (int c4 = 0; c4 < CW / 4; ++c4) {
+                                    const float4 v = __ldcg(so + c4);
+                                    acc[4 * c4 + 0] += w * v.x;
+                                    acc[4 * c4 + 1] += w * v.y;
+                                    acc[4 * c4 + 2] += w * v.z;
+                                    acc[4 * c4 + 3] += w * v.w;
+                                }
+                            }
+#pragma unroll
+                            for (int c = 0; c < CW; c += 8) dst[(c0 + c) / 8] = pack8_bf16(&acc[c], inv);
+                        }
+                        if (p.lse != nullptr && half == 0)
+                            p.lse[it.out_row0 + row] =
+                                (ltot > 0.f) ? (mmax + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
                     }
                 }
             }
