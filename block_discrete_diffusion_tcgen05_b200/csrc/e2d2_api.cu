@@ -185,7 +185,7 @@ e2d2_status train_common(int mode, const void* q, const void* k0, const void* v0
     prm.S = S;
     prm.box1_rows = kBlockN;
     prm.scale_log2 = scale_log2(dm);
-    prm.num_qtiles = (L + kBlockM - 1) / kBlockM;
+    prm.num_qtiles = (L + 2 * kBlockM - 1) / (2 * kBlockM);  // work items take pairs of query tiles
     prm.num_items = static_cast<int>(BHq * prm.num_qtiles);
     const int grid = prm.num_items < di->sms ? prm.num_items : di->sms;
     return mode == kEncoder ? dispatch_fmha<kEncoder>(D, prm, grid, st)
