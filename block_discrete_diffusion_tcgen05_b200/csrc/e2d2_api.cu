@@ -280,7 +280,12 @@ e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, con
     const long long BHkv = static_cast<long long>(dims.batch) * dims.kv_heads;
     const int S16 = (S + 15) / 16 * 16;
     const int box1 = S16 < kBlockN ? S16 : kBlockN;
-    bool ok = map_2d(&prm.tm_q, q_blk, D, rows, kBlockM) &&
+    // Packed query rows per TMEM lane quarter.  The kernel can spread a short packed tile over the
+    // four lane quarters (q_chunk < 32); on B200 that measured slower for the sampling shapes (four
+    // warps then issue full-width TMEM loads and instruction streams for a quarter of the rows
+    // each), so rows stay contiguous.
+    const int q_chunk = kBlockM / 4;
+    bool ok = map_2d(&prm.tm_q, q_blk, D, rows, q_chunk) &&
               map_3d(&prm.tm_k0, k_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
               map_3d(&prm.tm_v0, v_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
               map_3d(&prm.tm_k1, k_blk, D, S, BHkv, S, box1) && map_3d(&prm.tm_v1, v_blk, D, S, BHkv, S, box1);
@@ -304,6 +309,7 @@ e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, con
     prm.tiles_per_unit = (S + kBlockN - 1) / kBlockN + (P + kBlockN - 1) / kBlockN;
     prm.total_tiles = BHkv * prm.num_qtiles * static_cast<long long>(prm.tiles_per_unit);
     prm.rows_cap = w.rows_cap;
+    prm.q_chunk = q_chunk;
     prm.slot_floats = w.slot_floats;
     long long grid = di->sms < kSampleMaxCtas ? di->sms : kSampleMaxCtas;
     if (grid > prm.total_tiles) grid = prm.total_tiles;

@@ -83,6 +83,7 @@ struct alignas(64) FmhaParams {
     long long total_tiles;  // sample: units * tiles_per_unit
     int slot_floats;    // sample: floats per partial slot
     int rows_cap;       // sample: rows stored per partial slot
+    int q_chunk;        // sample: packed query rows per TMEM lane quarter (multiple of 8, <= 32)
 };
 
 template <int D, int MODE>
@@ -143,7 +144,23 @@ struct Item {
     int n1, a1;     // source-1 tiles (visited first), starting at key tile a1
     int n0;         // source-0 tiles, starting at key tile 0
     int t_begin, t_end;
+    // What each query tile needs of that stream: source-1 key tiles [a1q, e1q), source-0 key
+    // tiles [0, n0q).  Other tiles are skipped for that query tile (no MMA, no softmax).
+    int a1q[2], e1q[2], n0q[2];
 };
+
+// Key tile t of the item's stream is needed by query tile q.
+__device__ __forceinline__ bool tile_needed(const Item& it, int q, int t) {
+    // select, not index: q may be a runtime value and the arrays must stay in registers
+    const int a1q = q ? it.a1q[1] : it.a1q[0];
+    const int e1q = q ? it.e1q[1] : it.e1q[0];
+    const int n0q = q ? it.n0q[1] : it.n0q[0];
+    if (t < it.n1) {
+        const int kt = it.a1 + t;
+        return kt >= a1q && kt < e1q;
+    }
+    return (t - it.n1) < n0q;
+}
 
 // Key-tile ranges a block of query rows [r0, r_last] needs (train calls).
 template <int MODE>
@@ -194,6 +211,9 @@ struct Scheduler {
             it.n1 = ceil_div_i(p.S, kBlockN);
             it.a1 = 0;
             it.n0 = ceil_div_i(p.P, kBlockN);
+            it.a1q[0] = it.a1q[1] = 0;
+            it.e1q[0] = it.e1q[1] = it.n1;
+            it.n0q[0] = it.n0q[1] = it.n0;
             it.t_begin = static_cast<int>(pos - ubeg);
             it.t_end = static_cast<int>(seg_end - ubeg);
             pos = seg_end;
@@ -212,10 +232,22 @@ struct Scheduler {
             it.q_y = it.q_row0;
             it.out_row0 = 0;
             it.nact = (it.q_row0 + kBlockM < L) ? 2 : 1;
-            // Key tiles: the union of what the active query tiles need.
-            const int r_last = min(L, it.q_row0 + it.nact * kBlockM) - 1;
-            int a1, e1, n0;
-            train_ranges<MODE>(L, S, it.q_row0, r_last, a1, e1, n0);
+            // Key tiles: each active query tile's ranges, and their union (the stream).
+            int a1 = 1 << 30, e1 = 0, n0 = 0;
+            for (int q = 0; q < 2; ++q) {
+                const int r0 = it.q_row0 + q * kBlockM;
+                if (q < it.nact) {
+                    train_ranges<MODE>(L, S, r0, min(L, r0 + kBlockM) - 1, it.a1q[q], it.e1q[q], it.n0q[q]);
+                    if (it.e1q[q] > it.a1q[q]) {
+                        a1 = min(a1, it.a1q[q]);
+                        e1 = max(e1, it.e1q[q]);
+                    }
+                    n0 = max(n0, it.n0q[q]);
+                } else {
+                    it.a1q[q] = it.e1q[q] = it.n0q[q] = 0;
+                }
+            }
+            if (e1 == 0) a1 = 0;
             it.a1 = a1;
             it.n1 = e1 - a1;
             it.n0 = n0;
@@ -297,7 +329,6 @@ struct PendingPV {
     uint32_t qt;       // per-query-tile tile counter (p_full parity)
     uint32_t qi;       // per-query-tile item counter (o_free parity, O buffer)
     uint32_t nk;       // keys in the tile (multiple of 16)
-    uint32_t extra;    // additional kv_empty arrivals (query tiles inactive in this item)
 };
 
 // Issues O[q] (+)= P[q] . V[st] (A = P from TMEM, B = V MN-major in shared memory) once the
@@ -323,7 +354,7 @@ __device__ __forceinline__ bool issue_pv(int q, const PendingPV& pv, uint64_t* p
             ptx::mma_ts(d_tmem, a_tmem + p_col(ks), vdesc | ((v_base + ks * 16 * C::RB) >> 4), idesc_pv,
                         (pv.first && ks == 0) ? 0u : 1u);
         ptx::mma_commit(&pv_done[q]);
-        for (uint32_t i = 0; i <= pv.extra; ++i) ptx::mma_commit(&kv_empty[pv.st]);
+        ptx::mma_commit(&kv_empty[pv.st]);
     }
     __syncwarp();
     return true;
@@ -379,8 +410,9 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v, float scale) {
 
 // Loads the 128 S columns of this thread's row (one TMEM round trip), applies the row's key
 // interval [cmin, cmax) (tile-relative) and sets chunks without any allowed key in the warp to
-// -inf.  The loads are unconditional so that s has a single definition (no spills).
-__device__ __forceinline__ void load_s_row(uint32_t s_tmem, uint32_t live, int cmin, int cmax, float (&s)[128]) {
+// -inf.  The loads are unconditional so that s has a single definition (no spills).  Returns the
+// chunks in which every row of the warp has all 32 keys (no -inf there).
+__device__ __forceinline__ uint32_t load_s_row(uint32_t s_tmem, uint32_t live, int cmin, int cmax, float (&s)[128]) {
     uint32_t raw[128];
 #pragma unroll
     for (int a = 0; a < 4; ++a) ptx::tmem_ld32(s_tmem + 32 * a, &raw[32 * a]);
@@ -388,6 +420,7 @@ __device__ __forceinline__ void load_s_row(uint32_t s_tmem, uint32_t live, int c
     ptx::reg_fence<128>(raw);
 #pragma unroll
     for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c]);
+    uint32_t whole_bits = 0;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
         if (!(live & (1u << a))) {
@@ -401,15 +434,18 @@ __device__ __forceinline__ void load_s_row(uint32_t s_tmem, uint32_t live, int c
                     const int col = 32 * a + c;
                     s[32 * a + c] = (col >= cmin && col < cmax) ? s[32 * a + c] : -INFINITY;
                 }
+            } else {
+                whole_bits |= 1u << a;
             }
         }
     }
+    return whole_bits;
 }
 
 // P = exp2(s * sl2 + neg_m) for the live chunks, packed to bf16 and stored over S (keys 32a..
 // 32a+31 -> columns 16a..16a+15); dead chunks below nchunks store zeros.  Returns the row sum.
-__device__ __forceinline__ float exp_store_row(uint32_t s_tmem, uint32_t live, int nchunks, const float (&s)[128],
-                                               float sl2, float neg_m) {
+__device__ __forceinline__ float exp_store_row(uint32_t s_tmem, uint32_t live, uint32_t whole, int nchunks,
+                                               const float (&s)[128], float sl2, float neg_m) {
     float sums[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
@@ -531,16 +567,25 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             ok = wait_bar_warp(&q_empty[qb], (qround & 1) ^ 1, abort_flag, p.err);
             if (!ok) break;
             if (leader) {
-                ptx::mbar_arrive_expect_tx(&q_full[qb], NQ * C::TILE_BYTES);
-                for (int q = 0; q < NQ; ++q)
-                    for (int ch = 0; ch < C::NCH; ++ch) {
-                        uint8_t* dst = smem + SM::OFF_Q + (qb * NQ + q) * C::TILE_BYTES + ch * C::CHUNK_BYTES;
-                        if (MODE == kDecoderSample)
-                            ptx::tma_load_2d(&p.tm_q, &q_full[qb], dst, ch * (C::RB / 2), it.q_y);
-                        else
+                if (MODE == kDecoderSample) {
+                    // The packed rows are spread over the four TMEM lane quarters: rows
+                    // [k*q_chunk, (k+1)*q_chunk) go to tile rows 32k.. so that every softmax warp
+                    // gets a share of them.
+                    ptx::mbar_arrive_expect_tx(&q_full[qb], 4u * p.q_chunk * D * 2);
+                    for (int k = 0; k < 4; ++k)
+                        for (int ch = 0; ch < C::NCH; ++ch) {
+                            uint8_t* dst = smem + SM::OFF_Q + qb * C::TILE_BYTES + ch * C::CHUNK_BYTES + 32 * k * C::RB;
+                            ptx::tma_load_2d(&p.tm_q, &q_full[qb], dst, ch * (C::RB / 2), it.q_y + k * p.q_chunk);
+                        }
+                } else {
+                    ptx::mbar_arrive_expect_tx(&q_full[qb], NQ * C::TILE_BYTES);
+                    for (int q = 0; q < NQ; ++q)
+                        for (int ch = 0; ch < C::NCH; ++ch) {
+                            uint8_t* dst = smem + SM::OFF_Q + (qb * NQ + q) * C::TILE_BYTES + ch * C::CHUNK_BYTES;
                             ptx::tma_load_3d(&p.tm_q, &q_full[qb], dst, ch * (C::RB / 2), it.q_y + q * kBlockM,
                                              it.q_z);
-                    }
+                        }
+                }
             }
             __syncwarp();
             ++item_idx;
@@ -613,10 +658,22 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     pend[q].have = false;
                 }
             if (!ok) break;
-            if (it.t_end <= it.t_begin && leader) ptx::mma_commit(&q_empty[qb]);
+            bool seen[NQ];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) seen[q] = false;
             for (int t = it.t_begin; t < it.t_end && ok; ++t) {
                 const uint32_t st = kv_iter % C::NST;
                 const uint32_t round = kv_iter / C::NST;
+                // A P.V still pending on this stage (its query tile skipped the tiles since)
+                // must be issued now: the stage is reloaded only after it.
+#pragma unroll
+                for (int q = 0; q < NQ; ++q)
+                    if (ok && pend[q].have && pend[q].st == st) {
+                        ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
+                                         tmem_base, sV, vdesc, idesc_pv, D, leader);
+                        pend[q].have = false;
+                    }
+                if (!ok) break;
                 ok = wait_bar_warp(&k_full[st], round & 1, abort_flag, p.err);
                 if (!ok) break;
                 ptx::tc_fence_after();
@@ -625,7 +682,12 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 const uint32_t k_base = sK + st * C::TILE_BYTES;
 #pragma unroll
                 for (int q = 0; q < NQ; ++q) {
-                    if (q >= it.nact) continue;
+                    if (q >= it.nact || !tile_needed(it, q, t)) {
+                        // This query tile does not use the stage: its kv_empty share is free now.
+                        if (leader) ptx::mbar_arrive(&kv_empty[st]);
+                        __syncwarp();
+                        continue;
+                    }
                     const uint32_t sbuf = qtile[q] % NSB;
                     // With one S buffer per query tile, the pending P.V (reading P over S) must be
                     // issued before S is overwritten; with two, S first keeps the tensor core busy.
@@ -644,7 +706,6 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                                         kdesc | ((k_base + off) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
                         }
                         ptx::mma_commit(&s_full[q * NSB + sbuf]);
-                        if (t == it.t_end - 1 && q == it.nact - 1) ptx::mma_commit(&q_empty[qb]);
                     }
                     __syncwarp();
                     if (NSB == 2 && pend[q].have) {
@@ -653,13 +714,13 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         if (!ok) break;
                     }
                     pend[q].have = true;
-                    pend[q].first = (t == it.t_begin);
+                    pend[q].first = !seen[q];
+                    seen[q] = true;
                     pend[q].st = st;
                     pend[q].round = round;
                     pend[q].qt = qtile[q];
                     pend[q].qi = qitem[q];
                     pend[q].nk = tr.nk16;
-                    pend[q].extra = (q == it.nact - 1) ? static_cast<uint32_t>(NQ - it.nact) : 0u;
                     ++qtile[q];
                 }
                 ++kv_iter;
@@ -667,6 +728,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
 #pragma unroll
             for (int q = 0; q < NQ; ++q)
                 if (q < it.nact) ++qitem[q];
+            // Q of this item is free once every QK^T issued so far has completed.
+            if (leader) ptx::mma_commit(&q_empty[qb]);
+            __syncwarp();
             ++item_idx;
         }
 #pragma unroll
@@ -707,9 +771,13 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 // Per-row key intervals [lo, hi) for source 0 and source 1 (empty for padded rows).
                 int lo0, hi0, lo1, hi1;
                 bool row_valid;
-                const int qrow = it.q_row0 + q * kBlockM + row;  // row within the head / packed unit
+                // Row of this lane within the head (train) or within the packed tile (sample: lane
+                // quarter k holds packed rows k*q_chunk ..).
+                const int prow = (MODE == kDecoderSample) ? (lane < p.q_chunk ? quarter * p.q_chunk + lane : kBlockM)
+                                                          : row;
+                const int qrow = it.q_row0 + q * kBlockM + prow;
                 if (MODE == kDecoderSample) {
-                    row_valid = qrow < p.rows_per_unit;
+                    row_valid = prow < kBlockM && qrow < p.rows_per_unit;
                     lo0 = 0;
                     hi0 = row_valid ? p.P : 0;
                     lo1 = 0;
@@ -733,7 +801,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of this row
                 const uint32_t ob = qitem % NOB;
                 const uint32_t o_tmem = tmem_base + lane_off + 256 + (ob * NQ + q) * D;
+                bool first = true;
                 for (int t = it.t_begin; t < it.t_end; ++t) {
+                    if (!tile_needed(it, q, t)) continue;
                     const uint32_t sbuf = qtile % NSB;
                     wait_bar_warp(&s_full[q * NSB + sbuf], (qtile / NSB) & 1, abort_flag, p.err);
                     ptx::tc_fence_after();
@@ -753,7 +823,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         if (__any_sync(0xffffffffu, mine)) live |= 1u << a;
                     }
                     float s[128];
-                    load_s_row(s_tmem, live, cmin, cmax, s);
+                    const uint32_t whole = load_s_row(s_tmem, live, cmin, cmax, s);
                     float cmx[4];
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
@@ -763,7 +833,6 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     }
                     const float mx = ptx::fmax3(cmx[0], cmx[1], fmaxf(cmx[2], cmx[3]));
                     const float m_new = fmaxf(m, mx * sl2);
-                    const bool first = (t == it.t_begin);
                     bool rescale = false;
                     float alpha = 1.f;
                     if (m_new > m + kRescaleThreshold) {
@@ -773,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         l *= alpha;
                     }
                     const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                    l += exp_store_row(s_tmem, live, nchunks, s, sl2, neg_m);
+                    l += exp_store_row(s_tmem, live, whole, nchunks, s, sl2, neg_m);
                     if (!first) {
                         // O may only be touched once the previous P.V has landed.
                         wait_bar_warp(&pv_done[q], (qtile - 1) & 1, abort_flag, p.err);
@@ -785,6 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     ptx::tc_fence_before();
                     ptx::mbar_arrive(&p_full[q * NSB + sbuf]);
                     ++qtile;
+                    first = false;
                 }
                 // ------------------------------------------------------------ epilogue
                 wait_bar_warp(&pv_done[q], (qtile - 1) & 1, abort_flag, p.err);
@@ -828,14 +898,14 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         }
                     } else if (whole) {
                         if (row_valid) {
-                            const size_t r = (MODE == kDecoderSample) ? static_cast<size_t>(it.out_row0 + row)
+                            const size_t r = (MODE == kDecoderSample) ? static_cast<size_t>(it.out_row0 + prow)
                                                                       : static_cast<size_t>(it.q_z) * p.L + qrow;
                             uint4* dst = reinterpret_cast<uint4*>(outp + r * D + c0);
 #pragma unroll
                             for (int c = 0; c < CW; c += 8) dst[c / 8] = pack8_bf16(&o[c], inv_l);
                         }
-                    } else if (row_valid && row < p.rows_cap) {
-                        float4* so = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + c0);
+                    } else if (row_valid && prow < p.rows_cap) {
+                        float4* so = reinterpret_cast<float4*>(slot + static_cast<size_t>(prow) * D + c0);
 #pragma unroll
                         for (int c = 0; c < CW; c += 4) so[c / 4] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
                     }
@@ -856,13 +926,13 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     }
                     if (p.lse != nullptr && row_valid) p.lse[static_cast<size_t>(it.q_z) * p.L + qrow] = lse_val;
                 } else if (whole) {
-                    if (p.lse != nullptr && row_valid) p.lse[it.out_row0 + row] = lse_val;
+                    if (p.lse != nullptr && row_valid) p.lse[it.out_row0 + prow] = lse_val;
                 } else {
                     // Split unit: (O, m, l) of this CTA is in its slot; take a ticket; the last CTA
                     // of the unit merges every slot.
-                    if (row_valid && row < p.rows_cap) {
-                        slot[p.rows_cap * D + row] = m;
-                        slot[p.rows_cap * D + p.rows_cap + row] = l;
+                    if (row_valid && prow < p.rows_cap) {
+                        slot[p.rows_cap * D + prow] = m;
+                        slot[p.rows_cap * D + p.rows_cap + prow] = l;
                     }
                     __threadfence();
                     ptx::named_barrier_sync(wg_bar, 128);
@@ -877,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     ptx::named_barrier_sync(wg_bar, 128);
                     if (is_last) {
                         __threadfence();
-                        if (row_valid && row < p.rows_cap) {
+                        if (row_valid && prow < p.rows_cap) {
                             const long long T = p.total_tiles;
                             const int grid = gridDim.x;
                             auto slot_ptr = [&](int c) -> const float* {
@@ -886,17 +956,17 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                             };
                             float mmax = -INFINITY;
                             for (int c = c_first; c <= c_last; ++c)
-                                mmax = fmaxf(mmax, __ldcg(slot_ptr(c) + p.rows_cap * D + row));
+                                mmax = fmaxf(mmax, __ldcg(slot_ptr(c) + p.rows_cap * D + prow));
                             const float muse = (mmax == -INFINITY) ? 0.f : mmax;
                             float ltot = 0.f;
                             for (int c = c_first; c <= c_last; ++c) {
                                 const float* sl = slot_ptr(c);
-                                const float mw = __ldcg(sl + p.rows_cap * D + row);
+                                const float mw = __ldcg(sl + p.rows_cap * D + prow);
                                 if (mw != -INFINITY)
-                                    ltot += ptx::ex2(mw - muse) * __ldcg(sl + p.rows_cap * D + p.rows_cap + row);
+                                    ltot += ptx::ex2(mw - muse) * __ldcg(sl + p.rows_cap * D + p.rows_cap + prow);
                             }
                             const float inv = (ltot > 0.f) ? 1.f / ltot : 0.f;
-                            uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + row) * D);
+                            uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + prow) * D);
 #pragma unroll 1
                             for (int c0 = 0; c0 < D; c0 += CW) {
                                 float acc[CW];
@@ -904,10 +974,10 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                                 for (int c = 0; c < CW; ++c) acc[c] = 0.f;
                                 for (int c = c_first; c <= c_last; ++c) {
                                     const float* sl = slot_ptr(c);
-                                    const float mw = __ldcg(sl + p.rows_cap * D + row);
+                                    const float mw = __ldcg(sl + p.rows_cap * D + prow);
                                     if (mw == -INFINITY) continue;
                                     const float w = ptx::ex2(mw - muse);
-                                    const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + c0);
+                                    const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(prow) * D + c0);
 #pragma unroll
                                     for (int c4 = 0; c4 < CW / 4; ++c4) {
                                         const float4 v = __ldcg(so + c4);
@@ -921,7 +991,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                                 for (int c = 0; c < CW; c += 8) dst[(c0 + c) / 8] = pack8_bf16(&acc[c], inv);
                             }
                             if (p.lse != nullptr)
-                                p.lse[it.out_row0 + row] =
+                                p.lse[it.out_row0 + prow] =
                                     (ltot > 0.f) ? (mmax + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
                         }
                     }
