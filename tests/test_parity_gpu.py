@@ -159,3 +159,41 @@ def test_outputs_fully_written_deterministic_and_bounded():
 
 def test_no_device_wait_timed_out():
     assert attn.last_device_error() == 0
+
+
+def test_sampling_loop_with_appends_matches_oracle(oracle):
+    """The long-context sampling loop's structure at a reduced size: per block, two layers each
+    run a sampling call over the cached prefix (P grows by S per block, from 0), then the block
+    is appended to that layer's cache.  One workspace serves every call (its tickets must come
+    back to zero).  Every call is checked against the oracle; the caches bit for bit at the end."""
+    B, Hq, Hkv, S, d, blocks, layers = 2, 8, 2, 16, 128, 10, 2
+    cap = blocks * S
+    rng_seed = 5000
+    caches = []
+    for layer in range(layers):
+        kc = torch.zeros((B, Hkv, cap, d), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        caches.append([kc, vc, np.zeros((B, Hkv, cap, d), np.uint16), np.zeros((B, Hkv, cap, d), np.uint16)])
+    q0 = torch.empty((B, Hq, S, d), dtype=torch.bfloat16, device="cuda")
+    ws = attn.sample_workspace(q0, caches[0][0])
+    P = 0
+    for blk in range(blocks):
+        for layer in range(layers):
+            kc, vc, kbits, vbits = caches[layer]
+            seed = rng_seed + 100 * blk + 10 * layer
+            q = H.gen((B, Hq, S, d), seed)
+            kb = H.gen((B, Hkv, S, d), seed + 1)
+            vb = H.gen((B, Hkv, S, d), seed + 2)
+            out, lse = attn.decoder_sample(q[1], kc, vc, P, kb[1], vb[1], workspace=ws)
+            torch.cuda.synchronize()
+            ref_o, ref_l = oracle.decoder_sample(q[0].f32, synth.bf16_bits_to_f32(kbits),
+                                                 synth.bf16_bits_to_f32(vbits), P, kb[0].f32, vb[0].f32)
+            H.compare(out, lse, ref_o, ref_l, f"loop block {blk} layer {layer} P{P}")
+            attn.kv_cache_append(kc, vc, P, kb[1], vb[1])
+            oracle.kv_append(kbits, vbits, P, kb[0].bits, vb[0].bits)
+        P += S
+    torch.cuda.synchronize()
+    for kc, vc, kbits, vbits in caches:
+        np.testing.assert_array_equal(kc.cpu().view(torch.int16).numpy().view(np.uint16), kbits)
+        np.testing.assert_array_equal(vc.cpu().view(torch.int16).numpy().view(np.uint16), vbits)
+    assert int(ws[:1024].view(torch.int32).abs().sum().item()) == 0  # tickets back to zero
