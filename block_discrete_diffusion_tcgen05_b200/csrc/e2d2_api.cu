@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "e2d2_attn.h"
+#include "fmha_keyrow_sm100.cuh"
 #include "fmha_sm100.cuh"
 #include "kv_append.cuh"
 
@@ -127,6 +128,24 @@ e2d2_status launch_fmha(const FmhaParams& prm, int grid, cudaStream_t st) {
         configured_dev = dev;
     }
     kern<<<grid, kThreads, smem, st>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+}
+
+template <int N>
+e2d2_status launch_keyrow(const FmhaParams& prm, int grid, cudaStream_t st) {
+    using SM = KrSmem<N>;
+    static_assert(SM::ALLOC <= 232448, "shared memory budget");
+    auto kern = fmha_keyrow_kernel<N>;
+    const int smem = SM::ALLOC > 118784 ? SM::ALLOC : 118784;
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return E2D2_ERR_CUDA;
+        configured_dev = dev;
+    }
+    kern<<<grid, kKrThreads, smem, st>>>(prm);
     return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
 }
 
@@ -285,7 +304,11 @@ e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, con
     // warps then issue full-width TMEM loads and instruction streams for a quarter of the rows
     // each), so rows stay contiguous.
     const int q_chunk = kBlockM / 4;
-    bool ok = map_2d(&prm.tm_q, q_blk, D, rows, q_chunk) &&
+    // Short packed tiles at d = 128 take the kernel with keys on the TMEM lanes (S^T = K Q^T):
+    // its tensor-core rows are keys, so none is padding.  N = packed columns rounded up.
+    const int GS = G * S;
+    const int keyrow_n = (D != 128 || GS > 64) ? 0 : (GS <= 16 ? 16 : (GS <= 32 ? 32 : 64));
+    bool ok = map_2d(&prm.tm_q, q_blk, D, rows, keyrow_n ? keyrow_n : q_chunk) &&
               map_3d(&prm.tm_k0, k_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
               map_3d(&prm.tm_v0, v_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
               map_3d(&prm.tm_k1, k_blk, D, S, BHkv, S, box1) && map_3d(&prm.tm_v1, v_blk, D, S, BHkv, S, box1);
@@ -305,15 +328,30 @@ e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, con
     prm.box1_rows = box1;
     prm.scale_log2 = scale_log2(dims);
     prm.rows_per_unit = G * S;
-    prm.num_qtiles = (G * S + kBlockM - 1) / kBlockM;
+    prm.num_qtiles = keyrow_n ? 1 : (G * S + kBlockM - 1) / kBlockM;
     prm.tiles_per_unit = (S + kBlockN - 1) / kBlockN + (P + kBlockN - 1) / kBlockN;
-    prm.total_tiles = BHkv * prm.num_qtiles * static_cast<long long>(prm.tiles_per_unit);
     prm.rows_cap = w.rows_cap;
     prm.q_chunk = q_chunk;
     prm.slot_floats = w.slot_floats;
+    // Schedule: with U units on G CTAs, floor(U/G)*G units run whole (one CTA each, last); the
+    // other R units are split stream-K over at most 5R CTAs, so that a unit has at most about six
+    // partials to merge.
+    const long long Tu = prm.tiles_per_unit;
+    const long long U = BHkv * prm.num_qtiles;
     long long grid = di->sms < kSampleMaxCtas ? di->sms : kSampleMaxCtas;
-    if (grid > prm.total_tiles) grid = prm.total_tiles;
-    return dispatch_fmha<kDecoderSample>(D, prm, static_cast<int>(grid), stream);
+    if (grid > U * Tu) grid = U * Tu;
+    const long long R = U >= grid ? U % grid : U;
+    prm.split_units = static_cast<int>(R);
+    prm.whole_units = static_cast<int>(U - R);
+    prm.split_ctas = static_cast<int>(R * 5 < grid ? R * 5 : grid);
+    if (prm.split_ctas > R * Tu) prm.split_ctas = static_cast<int>(R * Tu);
+    prm.total_tiles = R * Tu;
+    switch (keyrow_n) {
+        case 16: return launch_keyrow<16>(prm, static_cast<int>(grid), stream);
+        case 32: return launch_keyrow<32>(prm, static_cast<int>(grid), stream);
+        case 64: return launch_keyrow<64>(prm, static_cast<int>(grid), stream);
+        default: return dispatch_fmha<kDecoderSample>(D, prm, static_cast<int>(grid), stream);
+    }
 }
 
 e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int P, const void* k_new,

@@ -80,7 +80,10 @@ struct alignas(64) FmhaParams {
     int num_qtiles;     // train: pairs of query tiles per head; sample: query tiles per (b, kv head)
     int rows_per_unit;  // sample: G * S packed query rows per (b, kv head)
     int tiles_per_unit; // sample: key tiles per unit
-    long long total_tiles;  // sample: units * tiles_per_unit
+    long long total_tiles;  // sample: key tiles of the split units (split_units * tiles_per_unit)
+    int split_units;    // sample: units split stream-K over CTAs [0, split_ctas), processed first
+    int split_ctas;
+    int whole_units;    // sample: units after the split ones, one CTA each, round robin
     int slot_floats;    // sample: floats per partial slot
     int rows_cap;       // sample: rows stored per partial slot
     int q_chunk;        // sample: packed query rows per TMEM lane quarter (multiple of 8, <= 32)
@@ -133,6 +136,11 @@ __device__ __forceinline__ long long range_begin(int c, long long T, int grid) {
     return (static_cast<long long>(c) * T) / grid;
 }
 
+// Sampling schedule.  The units (b, kv head, query tile) are taken in two phases: first the
+// split units [0, split_units), whose key tiles form one stream cut into equal contiguous ranges
+// for CTAs [0, split_ctas) (a unit whose tiles fall to several CTAs is merged by the last of them),
+// then the whole units, unit split_units + k going to CTA k mod grid.  Whole units last means a
+// CTA's final epilogue never waits for another CTA.
 // A unit of work: NQ consecutive 128-row query tiles against a contiguous range of key tiles.
 struct Item {
     int q_z;        // train: b*Hq + h (Q/O tensor-map z); sample: unit index
@@ -184,21 +192,33 @@ struct Scheduler {
     int k;               // train: next item index
 
     __device__ Scheduler(const FmhaParams& prm) : p(prm) {
+        k = blockIdx.x;
         if (MODE == kDecoderSample) {
-            pos = range_begin(blockIdx.x, p.total_tiles, gridDim.x);
-            end = range_begin(blockIdx.x + 1, p.total_tiles, gridDim.x);
-        } else {
-            k = blockIdx.x;
+            const int c = static_cast<int>(blockIdx.x);
+            pos = c < p.split_ctas ? range_begin(c, p.total_tiles, p.split_ctas) : 0;
+            end = c < p.split_ctas ? range_begin(c + 1, p.total_tiles, p.split_ctas) : 0;
         }
     }
 
     __device__ bool next(Item& it) {
         if (MODE == kDecoderSample) {
-            if (pos >= end) return false;
             const int Tu = p.tiles_per_unit;
-            const int u = static_cast<int>(pos / Tu);
-            const long long ubeg = static_cast<long long>(u) * Tu;
-            const long long seg_end = (end < ubeg + Tu) ? end : ubeg + Tu;
+            int u;
+            long long ubeg, seg_end;
+            if (pos < end) {
+                u = static_cast<int>(pos / Tu);
+                ubeg = static_cast<long long>(u) * Tu;
+                seg_end = (end < ubeg + Tu) ? end : ubeg + Tu;
+            } else if (k < p.whole_units) {
+                u = p.split_units + k;
+                k += gridDim.x;
+                ubeg = 0;
+                pos = 0;
+                seg_end = Tu;
+                end = 0;
+            } else {
+                return false;
+            }
             const int qt = u % p.num_qtiles;
             const int kvz = u / p.num_qtiles;  // b*Hkv + g
             const int b = kvz / p.kv_heads, g = kvz % p.kv_heads;
@@ -216,7 +236,7 @@ struct Scheduler {
             it.n0q[0] = it.n0q[1] = it.n0;
             it.t_begin = static_cast<int>(pos - ubeg);
             it.t_end = static_cast<int>(seg_end - ubeg);
-            pos = seg_end;
+            if (pos < end) pos = seg_end;
             return true;
         } else {
             if (k >= p.num_items) return false;
@@ -870,9 +890,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 long long ubeg = 0;
                 if (MODE == kDecoderSample && !whole) {
                     ubeg = static_cast<long long>(it.q_z) * Tu;
-                    c_first = owner_cta(ubeg, p.total_tiles, gridDim.x);
-                    c_last = owner_cta(ubeg + Tu - 1, p.total_tiles, gridDim.x);
-                    const int my_slot = (range_begin(blockIdx.x, p.total_tiles, gridDim.x) >= ubeg)
+                    c_first = owner_cta(ubeg, p.total_tiles, p.split_ctas);
+                    c_last = owner_cta(ubeg + Tu - 1, p.total_tiles, p.split_ctas);
+                    const int my_slot = (range_begin(blockIdx.x, p.total_tiles, p.split_ctas) >= ubeg)
                                             ? 2 * blockIdx.x
                                             : 2 * blockIdx.x + 1;
                     slot = p.ws_partial + static_cast<size_t>(my_slot) * p.slot_floats;
@@ -934,9 +954,11 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         slot[p.rows_cap * D + prow] = m;
                         slot[p.rows_cap * D + p.rows_cap + prow] = l;
                     }
-                    __threadfence();
+                    // Release: the barrier orders the warpgroup's slot stores before one thread's
+                    // fence and ticket.
                     ptx::named_barrier_sync(wg_bar, 128);
                     if (wtid == 0) {
+                        __threadfence();
                         const int ticket = atomicAdd(&p.ws_tickets[c_first], 1);
                         const int last = (ticket == c_last - c_first) ? 1 : 0;
                         if (last) p.ws_tickets[c_first] = 0;
@@ -949,21 +971,25 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         __threadfence();
                         if (row_valid && prow < p.rows_cap) {
                             const long long T = p.total_tiles;
-                            const int grid = gridDim.x;
+                            const int grid = p.split_ctas;
                             auto slot_ptr = [&](int c) -> const float* {
                                 const int si = (range_begin(c, T, grid) >= ubeg) ? 2 * c : 2 * c + 1;
                                 return p.ws_partial + static_cast<size_t>(si) * p.slot_floats;
                             };
+                            // Loads of different partials do not depend on each other: the loops are
+                            // unrolled so that several L2 round trips overlap.
                             float mmax = -INFINITY;
+#pragma unroll 4
                             for (int c = c_first; c <= c_last; ++c)
                                 mmax = fmaxf(mmax, __ldcg(slot_ptr(c) + p.rows_cap * D + prow));
                             const float muse = (mmax == -INFINITY) ? 0.f : mmax;
                             float ltot = 0.f;
+#pragma unroll 4
                             for (int c = c_first; c <= c_last; ++c) {
                                 const float* sl = slot_ptr(c);
                                 const float mw = __ldcg(sl + p.rows_cap * D + prow);
-                                if (mw != -INFINITY)
-                                    ltot += ptx::ex2(mw - muse) * __ldcg(sl + p.rows_cap * D + p.rows_cap + prow);
+                                const float lw = __ldcg(sl + p.rows_cap * D + p.rows_cap + prow);
+                                ltot += (mw == -INFINITY) ? 0.f : ptx::ex2(mw - muse) * lw;
                             }
                             const float inv = (ltot > 0.f) ? 1.f / ltot : 0.f;
                             uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + prow) * D);
@@ -972,19 +998,21 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                                 float acc[CW];
 #pragma unroll
                                 for (int c = 0; c < CW; ++c) acc[c] = 0.f;
+#pragma unroll 2
                                 for (int c = c_first; c <= c_last; ++c) {
                                     const float* sl = slot_ptr(c);
                                     const float mw = __ldcg(sl + p.rows_cap * D + prow);
-                                    if (mw == -INFINITY) continue;
-                                    const float w = ptx::ex2(mw - muse);
                                     const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(prow) * D + c0);
+                                    float4 v[CW / 4];
+#pragma unroll
+                                    for (int c4 = 0; c4 < CW / 4; ++c4) v[c4] = __ldcg(so + c4);
+                                    const float w = (mw == -INFINITY) ? 0.f : ptx::ex2(mw - muse);
 #pragma unroll
                                     for (int c4 = 0; c4 < CW / 4; ++c4) {
-                                        const float4 v = __ldcg(so + c4);
-                                        acc[4 * c4 + 0] += w * v.x;
-                                        acc[4 * c4 + 1] += w * v.y;
-                                        acc[4 * c4 + 2] += w * v.z;
-                                        acc[4 * c4 + 3] += w * v.w;
+                                        acc[4 * c4 + 0] += w * v[c4].x;
+                                        acc[4 * c4 + 1] += w * v[c4].y;
+                                        acc[4 * c4 + 2] += w * v[c4].z;
+                                        acc[4 * c4 + 3] += w * v[c4].w;
                                     }
                                 }
 #pragma unroll

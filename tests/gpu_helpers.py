@@ -57,11 +57,12 @@ def run_decoder_case(orc, B, Hq, Hkv, L, S, d, sigma=1.0, seed0=200):
 
 
 def sample_inputs(B, Hq, Hkv, S, cap, d, sigma, seed0):
+    # sigma sharpens the scores (Q, K); V stays N(0, 1) so the output tolerance keeps its meaning
     q = gen((B, Hq, S, d), seed0, sigma)
     kc = gen((B, Hkv, cap, d), seed0 + 1, sigma)
-    vc = gen((B, Hkv, cap, d), seed0 + 2, sigma)
+    vc = gen((B, Hkv, cap, d), seed0 + 2, 1.0)
     kb = gen((B, Hkv, S, d), seed0 + 3, sigma)
-    vb = gen((B, Hkv, S, d), seed0 + 4, sigma)
+    vb = gen((B, Hkv, S, d), seed0 + 4, 1.0)
     return q, kc, vc, kb, vb
 
 

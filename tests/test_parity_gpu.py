@@ -52,12 +52,25 @@ SAMPLE_CASES = [
     (2, 2, 2, 16, 333, 400, 32),
     (1, 8, 2, 100, 513, 600, 128),    # S not a multiple of 16; 4 query tiles
     (1, 2, 2, 1, 129, 130, 64),       # S = 1
+    # d = 128 with G*S <= 64: the keys-on-lanes kernel (S^T = K Q^T)
+    (2, 8, 8, 8, 700, 720, 128),      # G*S = 8: 16 packed columns, 8 of them padding
+    (3, 6, 2, 5, 260, 300, 128),      # G*S = 15, S not a multiple of 16
+    (1, 12, 4, 16, 400, 420, 128),    # G*S = 48: 64 columns, 16 of them padding
+    (1, 4, 4, 16, 5000, 5000, 128),   # 4 units of 41 key tiles split over ~37 CTAs each
 ]
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,S,P,cap,d", SAMPLE_CASES)
 def test_decoder_sample_parity(oracle, B, Hq, Hkv, S, P, cap, d):
     H.run_sample_case(oracle, B, Hq, Hkv, S, P, cap, d)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,S,P,cap,d", [(2, 8, 4, 16, 900, 1000, 128), (1, 8, 2, 16, 700, 700, 128),
+                                                 (2, 4, 2, 32, 600, 640, 128)])
+def test_decoder_sample_sharp_softmax(oracle, B, Hq, Hkv, S, P, cap, d):
+    """Q and K with sigma 3: running maxima move by more than the rescale threshold mid-unit,
+    so O is rescaled (and, split over CTAs, merged with unequal maxima)."""
+    H.run_sample_case(oracle, B, Hq, Hkv, S, P, cap, d, sigma=3.0, seed0=900)
 
 
 def test_train_pass_full_size_sampled_heads(oracle):
