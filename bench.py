@@ -51,13 +51,21 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-KERNEL_SOURCES = ("fmha_sm100.cuh", "ptx_sm100.cuh", "kv_append.cuh")
+# Device-code sources of each timed kernel (the sampling call at d = 128 with G*S <= 64 runs the
+# keys-on-lanes kernel, which shares the schedule and helpers of fmha_sm100.cuh).
+KERNEL_SOURCES = {
+    "encoder": ("fmha_sm100.cuh", "ptx_sm100.cuh"),
+    "decoder_train": ("fmha_sm100.cuh", "ptx_sm100.cuh"),
+    "decoder_sample": ("fmha_keyrow_sm100.cuh", "fmha_sm100.cuh", "ptx_sm100.cuh"),
+    "kv_append": ("kv_append.cuh",),
+}
 
 
-def kernel_source_hash() -> str:
-    """Hash of the device-code sources: ncu counters are only reported for the code they measured."""
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of a kernel's device-code sources: ncu counters are only reported for the code they
+    measured."""
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         h.update((ROOT / "block_discrete_diffusion_tcgen05_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()[:16]
 
@@ -68,10 +76,10 @@ def traffic_for(kernel: str):
         t = json.loads(TRAFFIC_FILE.read_text())
     except Exception:
         return None
-    if t.get("source_hash") != kernel_source_hash():
-        return None
     k = t.get("kernels", {}).get(kernel)
-    return None if k is None else k.get("dram_bytes_per_launch")
+    if k is None or k.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return k.get("dram_bytes_per_launch")
 
 
 class ClockSampler:

@@ -15,19 +15,20 @@
 // computed from tile indices and row numbers; key tiles outside every row's interval are
 // never loaded, and no mask matrix exists anywhere.
 //
-// CTA = 10 warps: warp 0 issues TMA loads, warp 1 owns tensor memory and issues tcgen05.mma,
-// warps 2..5 and 6..9 are two softmax warpgroups.  Per key tile of up to 128 keys:
+// CTA = 12 warps: warp 0 issues TMA loads, warp 1 owns tensor memory and issues tcgen05.mma,
+// warps 2..3 idle, warps 4..7 and 8..11 are two softmax warpgroups.  Per key tile of up to 128 keys:
 //     S  = Q K^T          tcgen05.mma, A = Q (smem), B = K (smem, K-major)  -> TMEM (fp32)
 //     P  = exp2(S*c - m)  softmax warpgroup, written back over S as bf16  -> TMEM
-//     O += P V            tcgen05.mma, A = P (TMEM), B = V (smem, MN-major) -> TMEM (fp32)
+//     O += P V            tcgen05.mma, A = P (TMEM), B = V (smem, MN-major) -> TMEM
 // Train calls take two 128-row query tiles per work item (one per softmax warpgroup) against
 // one shared K/V stream, and the MMA warp issues P.V(A, j-1), S(A, j), P.V(B, j-1), S(B, j):
 // while one warpgroup computes exponentials the other waits for its tensor-core work, so
-// the exponential unit and the tensor core stay busy (ping-pong).  The sampling call takes
-// one query tile (all G*S rows of a kv head) with S double-buffered in TMEM instead.
-// Each thread owns one query row (its TMEM lane) and all key columns of a tile, read from TMEM
-// in 64-column passes.  A running max is only moved when it grows by more than 2^8 (log2
-// units), so O is rescaled rarely; the final normalisation uses the same max and is exact.
+// the exponential unit and the tensor core stay busy (ping-pong).  The sampling call (shapes the
+// keys-on-lanes kernel of fmha_keyrow_sm100.cuh does not take) uses one query tile holding all
+// G*S packed rows of a kv head, with S double-buffered in TMEM instead.
+// Each thread owns one query row (its TMEM lane) and all 128 key columns of a tile, read from
+// TMEM in one pass.  A running max is only moved when it grows by more than 2^8 (log2 units), so
+// O is rescaled rarely; the final normalisation uses the same max and is exact.
 #pragma once
 
 #include <cstdint>
