@@ -428,8 +428,9 @@ def oracle_train_sample(budget_s: float):
     pairs = workloads.unmasked_pairs(tw.L, tw.S)
     flops = 2 * 4 * tw.head_dim * heads_done * pairs
     return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
-            "sample": f"E2D2 train pass (encoder + decoder-train, L1024 S16 d64), {heads_done} (batch, head) "
-                      f"pairs of the workload's {tw.batch * tw.q_heads}, fp64, {t_total:.2f} s",
+            "sample": f"E2D2 train pass (encoder + decoder-train, L1024 S16 d64), {heads_done} (batch, head) pairs "
+                      f"computed ({heads_done / (tw.batch * tw.q_heads):.2f} passes over the workload's "
+                      f"{tw.batch * tw.q_heads}), fp64, {t_total:.2f} s",
             "seconds": t_total}
 
 

@@ -56,7 +56,10 @@ SAMPLE_CASES = [
     (2, 8, 8, 8, 700, 720, 128),      # G*S = 8: 16 packed columns, 8 of them padding
     (3, 6, 2, 5, 260, 300, 128),      # G*S = 15, S not a multiple of 16
     (1, 12, 4, 16, 400, 420, 128),    # G*S = 48: 64 columns, 16 of them padding
-    (1, 4, 4, 16, 5000, 5000, 128),   # 4 units of 41 key tiles split over ~37 CTAs each
+    (1, 4, 4, 16, 5000, 5000, 128),   # 4 units of 41 key tiles, each split over 5 CTAs
+    # schedule corners on a 148-SM part: more units than CTAs
+    (75, 4, 2, 16, 300, 320, 128),    # 150 units: 148 whole, 2 split over 10 CTAs (keys-on-lanes kernel)
+    (40, 8, 4, 8, 200, 210, 64),      # 160 units: 148 whole, 12 split over 60 CTAs (generic kernel)
 ]
 
 
