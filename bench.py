@@ -181,6 +181,117 @@ def make_inputs(torch, dev, rank: int):
     return train, sample
 
 
+def run_workload_set(torch, attn, workloads, dev, peaks):
+    """The two other workloads of the scope table, timed on the device (CUDA events around the
+    whole loop; inputs drawn on the device from a seeded generator: timing only, values do not
+    change the work):
+      translation_train_chain  one step = 28 encoder + 4 decoder-train calls, B16 L512 S4 H16 d64,
+                               every layer on its own buffers (2.3 GB per step, no L2 reuse across
+                               layers); 3 warm-up + 20 timed steps.
+      long_sample_loop         B4 S16 Hq32 Hkv8 d128, 8 layers: for each of 512 blocks, 16 denoise
+                               steps x 8 decoder sampling calls with P = 16 n, then one KV-cache
+                               append per layer; eager launches from Python as a user would make
+                               them; device time per quarter of the loop (P ranges)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(4242)
+
+    def rnd(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    hbm, tc = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    res = {}
+    # ---- translation-shaped train chain
+    tc_shape = workloads.TRAIN_CHAIN
+    shp = (tc_shape.batch, tc_shape.q_heads, tc_shape.L, tc_shape.head_dim)
+    enc_layers = [tuple(rnd(*shp) for _ in range(3)) + (torch.empty(*shp, device=dev, dtype=torch.bfloat16),
+                                                        torch.empty(shp[:3], device=dev)) for _ in range(tc_shape.enc_calls)]
+    dec_layers = [tuple(rnd(*shp) for _ in range(5)) + (torch.empty(*shp, device=dev, dtype=torch.bfloat16),
+                                                        torch.empty(shp[:3], device=dev)) for _ in range(tc_shape.dec_calls)]
+    S = tc_shape.S
+
+    def chain_step():
+        for q, k, v, o, l in enc_layers:
+            attn.encoder_blockcausal(q, k, v, S, out=o, lse=l)
+        for q, ke, ve, kd, vd, o, l in dec_layers:
+            attn.decoder_train(q, ke, ve, kd, vd, S, out=o, lse=l)
+
+    for _ in range(3):
+        chain_step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = 20
+    a.record()
+    for _ in range(steps):
+        chain_step()
+    b.record()
+    torch.cuda.synchronize()
+    step_s = a.elapsed_time(b) * 1e-3 / steps
+    fl = (tc_shape.enc_calls + tc_shape.dec_calls) * workloads.useful_flops_train(tc_shape)
+    by = tc_shape.enc_calls * workloads.bytes_train(tc_shape, False) + tc_shape.dec_calls * workloads.bytes_train(tc_shape, True)
+    attainable = min(tc * 1e12, fl / by * hbm * 1e9)
+    res["translation_train_chain"] = {
+        "workload": tc_shape.name, "steps": steps, "ms_per_step": step_s * 1e3,
+        "useful_tflops": fl / step_s / 1e12, "gbs": by / step_s / 1e9,
+        "frac_tensor": fl / step_s / 1e12 / tc, "frac_attainable": fl / step_s / attainable,
+        "launches_per_step": tc_shape.enc_calls + tc_shape.dec_calls}
+    del enc_layers, dec_layers
+    # ---- long-context sample loop
+    w = workloads.SAMPLE_LOOP
+    B, Hq, Hkv, Sb, d, layers = w["batch"], w["q_heads"], w["kv_heads"], w["S"], w["head_dim"], w["layers"]
+    steps_pb, nblocks = w["steps_per_block"], w["P_max"] // w["S"]
+    cap = w["P_max"] + Sb
+    caches = [(rnd(B, Hkv, cap, d), rnd(B, Hkv, cap, d)) for _ in range(layers)]
+    qb, kb, vb = rnd(B, Hq, Sb, d), rnd(B, Hkv, Sb, d), rnd(B, Hkv, Sb, d)
+    kn, vn = rnd(B, Hkv, Sb, d), rnd(B, Hkv, Sb, d)
+    out = torch.empty_like(qb)
+    lse = torch.empty(B, Hq, Sb, device=dev)
+    ws = attn.sample_workspace(qb, caches[0][0])
+
+    def block(P):
+        for _ in range(steps_pb):
+            for kc, vc in caches:
+                attn.decoder_sample(qb, kc, vc, P, kb, vb, workspace=ws, out=out, lse=lse)
+        for kc, vc in caches:
+            attn.kv_cache_append(kc, vc, P, kn, vn)
+
+    for n in range(4):  # warm-up on the first blocks
+        block(16 * n)
+    torch.cuda.synchronize()
+    quarters = 4
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(quarters + 1)]
+    ev[0].record()
+    for qi in range(quarters):
+        for n in range(qi * nblocks // quarters, (qi + 1) * nblocks // quarters):
+            block(16 * n)
+        ev[qi + 1].record()
+    torch.cuda.synchronize()
+    q_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(quarters)]
+    calls = steps_pb * layers
+
+    def loop_bytes(n0, n1):
+        tot = 0
+        for n in range(n0, n1):
+            shp_n = workloads.SampleShape("", batch=B, P=16 * n, S=Sb, q_heads=Hq, kv_heads=Hkv, head_dim=d)
+            tot += calls * workloads.bytes_sample(shp_n) + layers * 2 * 2 * B * Hkv * Sb * d * 2
+        return tot
+
+    buckets = []
+    for qi in range(quarters):
+        n0, n1 = qi * nblocks // quarters, (qi + 1) * nblocks // quarters
+        by = loop_bytes(n0, n1)
+        buckets.append({"P": [16 * n0, 16 * (n1 - 1)], "ms": q_ms[qi], "gbs": by / (q_ms[qi] * 1e-3) / 1e9,
+                        "us_per_sample_call": q_ms[qi] * 1e3 / ((n1 - n0) * calls)})
+    total_ms = sum(q_ms)
+    by = loop_bytes(0, nblocks)
+    res["long_sample_loop"] = {
+        "workload": w["name"], "blocks": nblocks, "sample_calls": nblocks * calls, "appends": nblocks * layers,
+        "ms_per_loop": total_ms, "gbs": by / (total_ms * 1e-3) / 1e9, "frac_hbm": by / (total_ms * 1e-3) / 1e9 / hbm,
+        "by_prefix_quarter": buckets, "launch": "eager (one Python call per kernel)"}
+    del caches
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
@@ -298,6 +409,11 @@ def run_ours(args, rank, world, local_rank):
                           "frac_attainable": (fl / s) / min(tc_peak * 1e12, fl / by * hbm_peak * 1e9)}
     kern_detail["kv_append"] = {"avg_us": per_kernel_ms["kv_append"] * 1e3 / K}
 
+    # ---- the other workloads of the scope table (rank 0 of a single-GPU run) ---------------
+    workload_set = None
+    if world == 1 and not args.no_workload_set:
+        workload_set = run_workload_set(torch, attn, workloads, dev, peaks)
+
     # ---- e2e: the same train metric through the public API with host buffers --------------
     e2e = None
     if not args.no_e2e:
@@ -320,6 +436,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "e2e": e2e,
     }
+    if workload_set is not None:
+        line["workload_set"] = workload_set
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
     if dist is not None:
@@ -481,6 +599,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workload-set", action="store_true",
+                    help="skip timing the translation train chain and the long sample loop")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-step-budget", type=float, default=8.0, help="max seconds of oracle work per reference step")
     ap.add_argument("--ref-total-budget", type=float, default=150.0, help="seconds of oracle work for the whole reference run")

@@ -112,6 +112,44 @@ def test_sampling_step_full_size_sampled_batches(oracle):
         H.compare(out[sl], lse[sl], ro, rl, f"sampling step b{b}")
 
 
+def test_translation_train_full_size_sampled_heads(oracle):
+    """Translation-shaped train pass at full size (B16 L512 S4 H16 d64: the shape of the 28 encoder
+    and 4 decoder calls of one step); the oracle recomputes two (batch, head) pairs per call."""
+    w = workloads.TRAIN_CHAIN
+    B, Hq, L, d, S = w.batch, w.q_heads, w.L, w.head_dim, w.S
+    q = H.gen((B, Hq, L, d), synth.seed_for(4, 0, "q"), w.sigma)
+    k = H.gen((B, Hq, L, d), synth.seed_for(4, 0, "k"), w.sigma)
+    v = H.gen((B, Hq, L, d), synth.seed_for(4, 0, "v"), 1.0)
+    ke = H.gen((B, Hq, L, d), synth.seed_for(4, 0, "k_enc"), w.sigma)
+    ve = H.gen((B, Hq, L, d), synth.seed_for(4, 0, "v_enc"), 1.0)
+    out_e, lse_e = attn.encoder_blockcausal(q[1], k[1], v[1], S)
+    out_d, lse_d = attn.decoder_train(q[1], ke[1], ve[1], k[1], v[1], S)
+    torch.cuda.synchronize()
+    for b, h in ((0, 0), (15, 11)):
+        bs, hs = slice(b, b + 1), slice(h, h + 1)
+        qq, kk, vv = q[0].f32[bs, hs], k[0].f32[bs, hs], v[0].f32[bs, hs]
+        ro, rl = oracle.encoder(qq, kk, vv, S)
+        H.compare(out_e[bs, hs], lse_e[bs, hs], ro, rl, f"translation encoder b{b} h{h}")
+        ro, rl = oracle.decoder_train(qq, ke[0].f32[bs, hs], ve[0].f32[bs, hs], kk, vv, S)
+        H.compare(out_d[bs, hs], lse_d[bs, hs], ro, rl, f"translation decoder b{b} h{h}")
+
+
+@pytest.mark.parametrize("P", [0, 16, 1008, 4080, 8176])
+def test_long_sample_loop_shapes(oracle, P):
+    """Sampling calls of the long-context loop (B4 S16 Hq32 Hkv8 d128) at prefix lengths of its
+    blocks 0, 1, 63, 255 and 511, full size; the oracle recomputes two batch entries."""
+    w = workloads.SAMPLE_LOOP
+    B, Hq, Hkv, S, d = w["batch"], w["q_heads"], w["kv_heads"], w["S"], w["head_dim"]
+    cap = w["P_max"] + S
+    q, kc, vc, kb, vb = H.sample_inputs(B, Hq, Hkv, S, cap, d, 1.0, 5000 + P)
+    out, lse = attn.decoder_sample(q[1], kc[1], vc[1], P, kb[1], vb[1])
+    torch.cuda.synchronize()
+    for b in (0, 3):
+        sl = slice(b, b + 1)
+        ro, rl = oracle.decoder_sample(q[0].f32[sl], kc[0].f32[sl], vc[0].f32[sl], P, kb[0].f32[sl], vb[0].f32[sl])
+        H.compare(out[sl], lse[sl], ro, rl, f"long loop P{P} b{b}")
+
+
 def test_sample_equals_train_rows():
     """On the GPU: a sampling call for block b over the encoder prefix [0, bS) reproduces the
     decoder-train rows of block b (same inputs)."""
