@@ -82,8 +82,8 @@ struct KrSmem {
     static constexpr int OFF_BAR = OFF_STG + STG_BYTES;
     // q_full[2], q_empty[2], k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2],
     // s_free[2], p_full[2], pv_done[2], o_full[2], o_free[2], l_ready[2], l_free[2], qk_drain,
-    // pv_drain, tmem_done
-    static constexpr int NBAR = 4 + 2 * C::NK + 2 * C::NV + 16 + 3;
+    // pv_drain, tmem_done, merge_full
+    static constexpr int NBAR = 4 + 2 * C::NK + 2 * C::NV + 16 + 4;
     static constexpr int OFF_VOTE = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;  // u32 [2 wg][2 parity][4 warps]
     static constexpr int OFF_CMAX = OFF_VOTE + 2 * 2 * 4 * 4;     // float [2 wg][2 parity][4 warps][NH]
     static constexpr int OFF_LRED = OFF_CMAX + 2 * 2 * 4 * C::NH * 4;  // float [2 ob][2 wg][4 warps][NH]
@@ -169,12 +169,13 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
     uint64_t* qk_drain = l_free + 2;                                                                  \
     uint64_t* pv_drain = qk_drain + 1;                                                                \
     uint64_t* tmem_done = pv_drain + 1;     /* softmax and epilogue threads are done with TMEM */    \
+    uint64_t* merge_full = tmem_done + 1;   /* partial slots copied in for the final merge */        \
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);                         \
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);              \
     volatile int* bcast = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 16);                  \
     (void)q_full; (void)q_empty; (void)k_full; (void)k_empty; (void)v_full; (void)v_empty;            \
     (void)s_full; (void)s_free; (void)p_full; (void)pv_done; (void)o_full; (void)o_free;              \
-    (void)l_ready; (void)l_free; (void)qk_drain; (void)pv_drain; (void)tmem_done;                     \
+    (void)l_ready; (void)l_free; (void)qk_drain; (void)pv_drain; (void)tmem_done; (void)merge_full;   \
     (void)tmem_holder; (void)abort_flag; (void)bcast;
     uint32_t tmem_base;
     {
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         ptx::mbar_init(qk_drain, 1);
         ptx::mbar_init(pv_drain, 1);
         ptx::mbar_init(tmem_done, kSoftmaxThreads + 128);
+        ptx::mbar_init(merge_full, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -633,7 +635,61 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 ptx::named_barrier_sync(3, 128);
                 const int is_last = *bcast;
                 ptx::named_barrier_sync(3, 128);
-                if (is_last) {
+                // In the CTA's last unit every K/V, Q and P^T buffer is free (the producers are done
+                // and every product of the unit has landed), and so is the staging buffer (this
+                // CTA's slot copies completed before the ticket): the partial slots are then copied
+                // in with one bulk copy each, all in flight at once, and merged from shared memory.
+                const int nparts = c_last - c_first + 1;
+                const uint32_t slot_bytes = static_cast<uint32_t>(p.slot_floats) * 4u;
+                Scheduler<kDecoderSample> peek = sched;
+                Item next_it;
+                const bool in_smem = is_last && !peek.next(next_it) &&
+                                     static_cast<uint32_t>(nparts) * slot_bytes <=
+                                         static_cast<uint32_t>(SM::OFF_STG + SM::STG_BYTES - SM::OFF_Q);
+                if (in_smem) {
+                    __threadfence();
+                    uint8_t* region = smem + SM::OFF_Q;
+                    if (wtid == 0) {
+                        ptx::fence_proxy_async_global();
+                        ptx::mbar_arrive_expect_tx(merge_full, static_cast<uint32_t>(nparts) * slot_bytes);
+                        for (int c = c_first; c <= c_last; ++c)
+                            ptx::bulk_load_g2s(region + (c - c_first) * slot_bytes, slot_of(c), slot_bytes, merge_full);
+                    }
+                    wait_bar_warp(merge_full, 0, abort_flag, p.err);
+                    const int dq = (wtid & 3) * 32;
+#pragma unroll 1
+                    for (int col = wtid >> 2; col < cap; col += 32) {
+                        float mm = -INFINITY, ll = 0.f, acc[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll 1
+                        for (int c = 0; c < nparts; ++c) {
+                            const float* sl = reinterpret_cast<const float*>(region + c * slot_bytes);
+                            const float mc = sl[cap * D + col];
+                            const float lc = sl[cap * D + cap + col];
+                            const float4* so = reinterpret_cast<const float4*>(sl + col * D + dq);
+                            const float mn = fmaxf(mm, mc);
+                            const float wa = (mm == -INFINITY) ? 0.f : ptx::ex2(mm - mn);
+                            const float wb = (mc == -INFINITY) ? 0.f : ptx::ex2(mc - mn);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float4 v = so[i];
+                                acc[4 * i + 0] = acc[4 * i + 0] * wa + v.x * wb;
+                                acc[4 * i + 1] = acc[4 * i + 1] * wa + v.y * wb;
+                                acc[4 * i + 2] = acc[4 * i + 2] * wa + v.z * wb;
+                                acc[4 * i + 3] = acc[4 * i + 3] * wa + v.w * wb;
+                            }
+                            ll = ll * wa + lc * wb;
+                            mm = mn;
+                        }
+                        const float inv = ll > 0.f ? 1.f / ll : 0.f;
+                        uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + col) * D + dq);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dst[i] = pack8_bf16(&acc[8 * i], inv);
+                        if (p.lse != nullptr && dq == 0)
+                            p.lse[it.out_row0 + col] = ll > 0.f ? (mm + __log2f(ll)) * 0.69314718055994531f : -INFINITY;
+                    }
+                } else if (is_last) {
                     __threadfence();
                     // Online merge over the partials in CTA order (the result does not depend on
                     // which CTA merges).  Thread = (column, 32 head-dim values): the ten loads of

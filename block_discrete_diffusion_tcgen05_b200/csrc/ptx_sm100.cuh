@@ -126,6 +126,15 @@ __device__ __forceinline__ void tma_store_wait_all() {
 }
 
 // Bulk copy (no tensor map) of `bytes` (multiple of 16; both addresses 16-byte aligned) from
+// global to shared memory, completing on an mbarrier (complete_tx), no multicast.
+__device__ __forceinline__ void bulk_load_g2s(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(sdst)),
+                 "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Bulk copy (no tensor map) of `bytes` (multiple of 16; both addresses 16-byte aligned) from
 // shared to global memory, tracked by the bulk-group mechanism (commit / wait_group).
 __device__ __forceinline__ void bulk_store_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
