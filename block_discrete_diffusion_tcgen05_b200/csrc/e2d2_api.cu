@@ -334,8 +334,10 @@ e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, con
     prm.q_chunk = q_chunk;
     prm.slot_floats = w.slot_floats;
     // Schedule: with U units on G CTAs, floor(U/G)*G units run whole (one CTA each, last); the
-    // other R units are split stream-K over at most 5R CTAs, so that a unit has at most about six
-    // partials to merge.
+    // other R units are split stream-K over at most 5R CTAs (a unit has at most about six partials
+    // to merge), and only as far as every piece keeps about kMinSplitTiles key tiles: publishing and
+    // merging a partial costs several microseconds, more than streaming a few tiles.  A split never
+    // uses fewer CTAs than there are units.
     const long long Tu = prm.tiles_per_unit;
     const long long U = BHkv * prm.num_qtiles;
     long long grid = di->sms < kSampleMaxCtas ? di->sms : kSampleMaxCtas;
@@ -343,9 +345,16 @@ e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, con
     const long long R = U >= grid ? U % grid : U;
     prm.split_units = static_cast<int>(R);
     prm.whole_units = static_cast<int>(U - R);
-    prm.split_ctas = static_cast<int>(R * 5 < grid ? R * 5 : grid);
-    if (prm.split_ctas > R * Tu) prm.split_ctas = static_cast<int>(R * Tu);
+    constexpr long long kMinSplitTiles = 6;
+    long long sc = R * 5 < grid ? R * 5 : grid;
+    if (sc > R * Tu / kMinSplitTiles) sc = R * Tu / kMinSplitTiles;
+    if (sc < R) sc = R;
+    if (sc > R * Tu) sc = R * Tu;
+    prm.split_ctas = static_cast<int>(sc);
     prm.total_tiles = R * Tu;
+    // Whole units exist only when U >= grid, and then every CTA takes some; otherwise only the
+    // CTAs of the split phase have work.
+    if (prm.whole_units == 0) grid = prm.split_ctas;
     switch (keyrow_n) {
         case 16: return launch_keyrow<16>(prm, static_cast<int>(grid), stream);
         case 32: return launch_keyrow<32>(prm, static_cast<int>(grid), stream);
