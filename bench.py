@@ -552,12 +552,92 @@ def oracle_train_sample(budget_s: float):
             "seconds": t_total}
 
 
+def oracle_other_workloads():
+    """The oracle on bounded samples of the other three workloads (a few seconds in all):
+      sample_step              one full sampling call (B32 P2048 S16 Hq16 Hkv8 d128), HBM GB/s of
+                               the algorithmic bytes, as the GPU line reports it;
+      translation_train_chain  one encoder and one decoder-train call of B16 L512 S4 H16 d64 on a
+                               subset of the heads, scaled to the step of 28 + 4 calls;
+      long_sample_loop         single sampling calls of the loop (B4 S16 Hq32 Hkv8 d128) at
+                               P = 0, 1024, 4096, 8176, extrapolated linearly in (P + 16) over the
+                               512 x 128 calls of the loop (labelled as extrapolated)."""
+    import numpy as np
+
+    from block_discrete_diffusion_tcgen05_b200 import synth, workloads
+
+    orc, _ = _oracle_inputs()
+    out = {}
+    # one sampling step
+    sw = workloads.SAMPLE
+    cap = sw.P + sw.S
+    g = lambda shape, t: synth.normal_bf16(shape, synth.seed_for(3, 0, t), sw.sigma).f32
+    q = g((sw.batch, sw.q_heads, sw.S, sw.head_dim), "q")
+    kc, vc = g((sw.batch, sw.kv_heads, cap, sw.head_dim), "k_cache"), g((sw.batch, sw.kv_heads, cap, sw.head_dim), "v_cache")
+    kb, vb = g((sw.batch, sw.kv_heads, sw.S, sw.head_dim), "k_new"), g((sw.batch, sw.kv_heads, sw.S, sw.head_dim), "v_new")
+    t0 = time.perf_counter()
+    orc.decoder_sample(q, kc, vc, sw.P, kb, vb)
+    dt = time.perf_counter() - t0
+    out["sample_step"] = {"value": workloads.bytes_sample(sw) / dt / 1e9, "unit": "GB/s", "seconds": dt,
+                          "sample": f"{sw.name}: one whole call, fp64"}
+    # translation-shaped chain: the heads of one batch entry of each call, scaled
+    tc = workloads.TRAIN_CHAIN
+    nh = tc.q_heads
+    shp = (1, nh, tc.L, tc.head_dim)
+    g4 = lambda t: synth.normal_bf16(shp, synth.seed_for(4, 0, t), tc.sigma).f32
+    q4, k4, v4, ke4, ve4 = (g4(t) for t in ("q", "k", "v", "k_enc", "v_enc"))
+    t0 = time.perf_counter()
+    orc.encoder(q4, k4, v4, tc.S)
+    t_enc = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    orc.decoder_train(q4, ke4, ve4, k4, v4, tc.S)
+    t_dec = time.perf_counter() - t0
+    scale = tc.batch * tc.q_heads / nh
+    step_s = (tc.enc_calls * t_enc + tc.dec_calls * t_dec) * scale
+    fl = (tc.enc_calls + tc.dec_calls) * workloads.useful_flops_train(tc)
+    out["translation_train_chain"] = {
+        "value": fl / step_s / 1e12, "unit": "TFLOP/s", "seconds": t_enc + t_dec,
+        "sample": f"{tc.name}: one encoder and one decoder-train call on {nh} of the {tc.batch * tc.q_heads} "
+                  f"(batch, head) pairs, fp64, scaled to the 28 + 4 calls of a step"}
+    # long-context loop: calls at four prefix lengths, extrapolated
+    w = workloads.SAMPLE_LOOP
+    B, Hq, Hkv, S, d = w["batch"], w["q_heads"], w["kv_heads"], w["S"], w["head_dim"]
+    Pmax = w["P_max"] - S
+    gl = lambda shape, t: synth.normal_bf16(shape, synth.seed_for(5, 0, t), 1.0).f32
+    ql = gl((B, Hq, S, d), "q")
+    kcl, vcl = gl((B, Hkv, Pmax + S, d), "k_cache"), gl((B, Hkv, Pmax + S, d), "v_cache")
+    kbl, vbl = gl((B, Hkv, S, d), "k_new"), gl((B, Hkv, S, d), "v_new")
+    pts = []
+    for P in (0, 1024, 4096, Pmax):
+        t0 = time.perf_counter()
+        orc.decoder_sample(ql, np.ascontiguousarray(kcl[:, :, :P + S]), np.ascontiguousarray(vcl[:, :, :P + S]), P, kbl, vbl)
+        pts.append((P + S, time.perf_counter() - t0))
+    xs, ys = np.array([p[0] for p in pts], float), np.array([p[1] for p in pts])
+    a, b0 = np.polyfit(xs, ys, 1)
+    calls = w["steps_per_block"] * w["layers"]
+    nblocks = w["P_max"] // S
+    loop_s = sum(calls * (a * (16 * n + S) + b0) for n in range(nblocks))
+    loop_bytes = sum(calls * workloads.bytes_sample(workloads.SampleShape("", batch=B, P=16 * n, S=S, q_heads=Hq,
+                                                                          kv_heads=Hkv, head_dim=d))
+                     for n in range(nblocks))
+    out["long_sample_loop"] = {
+        "value": loop_bytes / loop_s / 1e9, "unit": "GB/s", "seconds": float(ys.sum()), "extrapolated": True,
+        "loop_s": loop_s,
+        "sample": f"{w['name']}: single calls at P = 0, 1024, 4096, {Pmax} (fp64), time fitted linearly in P + 16 "
+                  f"and summed over the {nblocks} x {calls} calls of the loop (extrapolated)"}
+    return out
+
+
 def cpu_baseline(budget_s: float):
     try:
-        return oracle_train_sample(budget_s)
+        res = oracle_train_sample(budget_s)
     except Exception as exc:  # the baseline is reported, never required
         return {"value": None, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
                 "sample": f"failed: {exc}"}
+    try:
+        res["workloads"] = oracle_other_workloads()
+    except Exception as exc:
+        res["workloads"] = {"failed": str(exc)}
+    return res
 
 
 def run_reference(args, rank, world):
