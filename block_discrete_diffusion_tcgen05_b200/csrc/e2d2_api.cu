@@ -162,8 +162,8 @@ e2d2_status dispatch_fmha(int D, const FmhaParams& prm, int grid, cudaStream_t s
 constexpr long long kMaxI32 = 0x7fffffffLL;
 
 e2d2_status check_train_shape(const e2d2_dims& dm, int L, int S) {
+    // S need not divide L: the last block then has L mod S rows; S >= L is one block.
     if (L <= 0 || S <= 0) return E2D2_ERR_INVALID_ARG;
-    if (S > L || L % S != 0) return E2D2_ERR_SHAPE;
     const long long rows = static_cast<long long>(dm.batch) * dm.q_heads * L;
     if (rows > kMaxI32 / 8) return E2D2_ERR_SHAPE;
     return E2D2_OK;

@@ -53,7 +53,7 @@ typedef enum {
     E2D2_OK = 0,
     E2D2_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad GQA ratio            */
     E2D2_ERR_UNSUPPORTED = 2, /* head_dim not in {32, 64, 128}, or not an sm_100 device     */
-    E2D2_ERR_SHAPE = 3,       /* L % S != 0, S > L, or a dimension too large                 */
+    E2D2_ERR_SHAPE = 3,       /* a dimension too large for the 32-bit row indexing           */
     E2D2_ERR_ALIGNMENT = 4,   /* a pointer not 16-byte aligned                              */
     E2D2_ERR_CAPACITY = 5,    /* P + S_new > capacity, or P > capacity                      */
     E2D2_ERR_WORKSPACE = 6,   /* workspace missing or smaller than the _workspace query     */
@@ -74,7 +74,10 @@ typedef struct {
  * attends to every key j with floor(j/S) <= floor(i/S) (its own block, bidirectionally, and
  * every earlier block).
  *   q   [batch][q_heads][L][d]   k, v [batch][kv_heads][L][d]   out [batch][q_heads][L][d]
- *   lse [batch][q_heads][L] or NULL.   Requires 1 <= S <= L and L % S == 0.
+ *   lse [batch][q_heads][L] or NULL.   Requires L >= 1 and S >= 1.  If S does not divide L the
+ *   last block is shorter (L mod S rows, as block diffusion allows: "Block Diffusion:
+ *   Interpolating Between Autoregressive and Diffusion Language Models", sec. 3); S >= L makes
+ *   the whole sequence one block.
  */
 E2D2_API e2d2_status e2d2_attn_encoder_blockcausal(const void* q, const void* k, const void* v, void* out,
                                           float* lse, e2d2_dims dims, int L, int S,
@@ -86,7 +89,8 @@ E2D2_API e2d2_status e2d2_attn_encoder_blockcausal(const void* q, const void* k,
  * blocks strictly before the query's block, and the decoder-side keys k_dec/v_dec of the
  * query's own block (bidirectional inside the block).
  *   q_dec [batch][q_heads][L][d]; k_enc, v_enc, k_dec, v_dec [batch][kv_heads][L][d];
- *   out [batch][q_heads][L][d]; lse [batch][q_heads][L] or NULL.  Requires L % S == 0.
+ *   out [batch][q_heads][L][d]; lse [batch][q_heads][L] or NULL.  Blocks as for the encoder
+ *   call (a shorter last block when S does not divide L).
  */
 E2D2_API e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_enc, const void* v_enc,
                                     const void* k_dec, const void* v_dec, void* out, float* lse,

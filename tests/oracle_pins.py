@@ -306,7 +306,40 @@ def pin_append_is_concatenation(orc):
     np.testing.assert_array_equal(vc[:, :, P:], vc0[:, :, P:])
 
 
+# ---------------------------------------------------------------------------------------
+# 12. Short last block (the block-diffusion page lets the last block be shorter when S does not
+#     divide L): with L = n S + r, 0 < r < S, full block b has S rows attending (b + 1) S keys and
+#     the r rows of the last block attend all L keys, so both masks hold S^2 n (n+1)/2 + r L
+#     pairs; S >= L is one block (n = 0, r = L: L^2 pairs).  A brute-force check on a tiny case
+#     takes the block rule with the last block clipped at L.
+# ---------------------------------------------------------------------------------------
+def pin_short_last_block(orc):
+    for L, S in ((10, 4), (13, 5), (7, 3), (100, 16), (200, 48), (5, 8), (9, 9)):
+        n, r = L // S, L % S
+        closed = S * S * n * (n + 1) // 2 + r * L
+        assert int(orc.mask_encoder(L, S).sum()) == closed, ("encoder", L, S)
+        assert int(orc.mask_decoder(L, S).sum()) == closed, ("decoder", L, S)
+    B, Hq, Hkv, L, S, d = 1, 2, 2, 10, 4, 4
+    q = _rand((B, Hq, L, d), 970).astype(np.float64)
+    k, v, ke, ve = (_rand((B, Hkv, L, d), 971 + t).astype(np.float64) for t in range(4))
+    scale = 0.6
+    out_e, lse_e = orc.encoder(q, k, v, S=S, scale=scale)
+    out_d, lse_d = orc.decoder_train(q, ke, ve, k, v, S=S, scale=scale)
+    for h in range(Hq):
+        for i in range(L):
+            b0 = (i // S) * S
+            end = min(L, b0 + S)  # the last block stops at L
+            o, l = _brute_row(q[0, h, i], [k[0, h, j] for j in range(end)], [v[0, h, j] for j in range(end)], scale)
+            np.testing.assert_allclose(out_e[0, h, i], o, rtol=0, atol=1e-12)
+            assert abs(lse_e[0, h, i] - l) < 1e-12
+            keys = [ke[0, h, j] for j in range(b0)] + [k[0, h, j] for j in range(b0, end)]
+            vals = [ve[0, h, j] for j in range(b0)] + [v[0, h, j] for j in range(b0, end)]
+            o, l = _brute_row(q[0, h, i], keys, vals, scale)
+            np.testing.assert_allclose(out_d[0, h, i], o, rtol=0, atol=1e-12)
+            assert abs(lse_d[0, h, i] - l) < 1e-12
+
+
 ALL_PINS = [pin_pair_count, pin_golden_pairs, pin_block_size_one_is_causal,
             pin_block_size_L_is_bidirectional, pin_masked_against_torch, pin_brute_force,
             pin_zero_keys_closed_form, pin_constant_values, pin_gqa_is_repeated_heads,
-            pin_sample_is_train_slice, pin_append_is_concatenation]
+            pin_sample_is_train_slice, pin_append_is_concatenation, pin_short_last_block]

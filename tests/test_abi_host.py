@@ -52,8 +52,11 @@ def test_encoder_argument_errors(lib):
     assert f(P16, P16, P16, P16, None, _lib.Dims(2, 4, 2, 96, 0.0), 64, 8, None) == 2  # head_dim
     assert f(P16, P16, P16, P16, None, _lib.Dims(2, 4, 3, 64, 0.0), 64, 8, None) == 1  # GQA ratio
     assert f(P16, P16, P16, P16, None, _lib.Dims(0, 4, 2, 64, 0.0), 64, 8, None) == 1  # batch
-    assert f(P16, P16, P16, P16, None, DIMS, 60, 8, None) == 3           # S does not divide L
-    assert f(P16, P16, P16, P16, None, DIMS, 8, 16, None) == 3           # S > L
+    # S need not divide L (short last block) and may exceed L (one block): such calls get past
+    # the shape checks to the alignment check (a misaligned lse keeps them from launching)
+    for L, S in ((60, 8), (8, 16)):
+        assert f(P16, P16, P16, P16, P16 + 2, DIMS, L, S, None) == 4
+    assert f(P16, P16, P16, P16, None, DIMS, 64, 0, None) == 1           # S = 0
     assert f(P16, P16, P16, P16, None, DIMS, 0, 8, None) == 1            # L = 0
     assert f(P16 + 8, P16, P16, P16, None, DIMS, 64, 8, None) == 4       # misaligned q
     assert f(P16, P16, P16, P16, P16 + 2, DIMS, 64, 8, None) == 4        # misaligned lse
@@ -64,7 +67,7 @@ def test_decoder_train_argument_errors(lib):
     f = lib.e2d2_attn_decoder_train
     assert f(P16, P16, P16, None, P16, P16, None, DIMS, 64, 8, None) == 1
     assert f(P16, P16, P16, P16, P16 + 4, P16, None, DIMS, 64, 8, None) == 4
-    assert f(P16, P16, P16, P16, P16, P16, None, DIMS, 64, 7, None) == 3
+    assert f(P16, P16, P16, P16, P16, P16, None, DIMS, 64, -1, None) == 1
 
 
 def test_sample_workspace_query_needs_no_gpu(lib):

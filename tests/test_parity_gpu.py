@@ -27,6 +27,11 @@ TRAIN_CASES = [
     (1, 2, 2, 130, 130, 64, 1.0),    # S = L, ragged
     (2, 2, 2, 512, 4, 64, 1.0),      # translation-shaped block size
     (1, 1, 1, 1024, 16, 64, 1.0),    # many tiles per row
+    # short last block (S does not divide L) and S > L (one block)
+    (1, 2, 2, 200, 48, 64, 1.0),     # blocks of 48, last one 8 rows
+    (1, 4, 2, 300, 7, 32, 1.0),      # last block 6 rows, GQA 2, d 32
+    (2, 2, 2, 130, 16, 128, 1.0),    # last block 2 rows, d 128
+    (1, 2, 1, 100, 160, 64, 1.0),    # S > L
 ]
 
 
