@@ -17,7 +17,7 @@ STATUS = {0: "E2D2_OK", 1: "E2D2_ERR_INVALID_ARG", 2: "E2D2_ERR_UNSUPPORTED", 3:
 EXPORTS = ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
            "e2d2_attn_decoder_sample_workspace", "e2d2_attn_decoder_sample",
            "e2d2_kv_cache_append", "e2d2_status_string", "e2d2_last_device_error", "e2d2_version",
-           "e2d2_attn_decoder_sample_noalloc")
+           "e2d2_attn_decoder_sample_noalloc", "e2d2_attn_encoder_block_step")
 
 # E2D2_SAMPLE_NOALLOC_MAX_BYTES of include/e2d2_attn.h
 SAMPLE_NOALLOC_MAX_BYTES = 32 << 20
@@ -58,6 +58,8 @@ def load(path: Path | str | None = None):
     lib.e2d2_attn_decoder_sample.argtypes = [vp, vp, vp, ci, ci, vp, vp, vp, fp, Dims, ci, vp,
                                              ctypes.c_size_t, st]
     lib.e2d2_kv_cache_append.argtypes = [vp, vp, ci, ci, vp, vp, ci, Dims, st]
+    lib.e2d2_attn_encoder_block_step.argtypes = [vp, vp, vp, ci, ci, vp, vp, vp, fp, Dims, ci, vp,
+                                                 ctypes.c_size_t, st]
     lib.e2d2_attn_decoder_sample_noalloc.argtypes = [vp, vp, vp, ci, ci, vp, vp, vp, fp, Dims, ci, st]
     lib.e2d2_attn_decoder_sample_noalloc.restype = ctypes.c_int
     lib.e2d2_status_string.argtypes = [ci]

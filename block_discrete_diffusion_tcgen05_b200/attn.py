@@ -117,6 +117,33 @@ def decoder_sample(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=None
     return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
 
 
+def encoder_block_step(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=None, scale=None,
+                       out=None, lse=True):
+    """Encoder incremental block step: the block's S clean queries attend to k_cache[:, :, :P] and
+    to their own block (block-causal rows of the encoder), and k_blk/v_blk are written to cache
+    rows P..P+S-1 in the same launch.  Returns (out, lse); the new prefix length is P + S."""
+    lib = _lib.load()
+    for t, n in ((q_blk, "q_blk"), (k_cache, "k_cache"), (v_cache, "v_cache"), (k_blk, "k_blk"),
+                 (v_blk, "v_blk")):
+        _need(t, n)
+    B, Hq, S, d = q_blk.shape
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, cap, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [B, Hkv, capacity, d]")
+    if k_blk.shape != (B, Hkv, S, d) or v_blk.shape != k_blk.shape:
+        raise ValueError("k_blk/v_blk must be [B, Hkv, S, d]")
+    ws = sample_workspace(q_blk, k_cache) if workspace is None else workspace
+    out = torch.empty_like(q_blk) if out is None else out
+    lse_t = torch.empty((B, Hq, S), dtype=torch.float32, device=q_blk.device) if lse is True else lse
+    st = lib.e2d2_attn_encoder_block_step(q_blk.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cap, int(P),
+                                          k_blk.data_ptr(), v_blk.data_ptr(), out.data_ptr(),
+                                          None if lse_t is None or lse_t is False else lse_t.data_ptr(),
+                                          _dims(B, Hq, Hkv, d, scale), S, ws.data_ptr(),
+                                          ws.numel() * ws.element_size(), _stream(q_blk))
+    _lib.check(st, "e2d2_attn_encoder_block_step")
+    return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
+
+
 def kv_cache_append(k_cache, v_cache, P: int, k_new, v_new):
     """Writes k_new/v_new [B,Hkv,S_new,d] into rows P..P+S_new-1 of the caches; returns P+S_new."""
     lib = _lib.load()

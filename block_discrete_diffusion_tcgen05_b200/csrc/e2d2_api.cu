@@ -227,58 +227,16 @@ SampleLayout sample_layout(const e2d2_dims& dm, int S) {
     return w;
 }
 
-}  // namespace
-}  // namespace e2d2
-
-using namespace e2d2;
-
-extern "C" {
-
-const char* e2d2_status_string(e2d2_status s) {
-    switch (s) {
-        case E2D2_OK: return "E2D2_OK";
-        case E2D2_ERR_INVALID_ARG: return "E2D2_ERR_INVALID_ARG";
-        case E2D2_ERR_UNSUPPORTED: return "E2D2_ERR_UNSUPPORTED";
-        case E2D2_ERR_SHAPE: return "E2D2_ERR_SHAPE";
-        case E2D2_ERR_ALIGNMENT: return "E2D2_ERR_ALIGNMENT";
-        case E2D2_ERR_CAPACITY: return "E2D2_ERR_CAPACITY";
-        case E2D2_ERR_WORKSPACE: return "E2D2_ERR_WORKSPACE";
-        case E2D2_ERR_CUDA: return "E2D2_ERR_CUDA";
-        case E2D2_ERR_TIMEOUT: return "E2D2_ERR_TIMEOUT";
-    }
-    return "E2D2_ERR_UNKNOWN";
-}
-
-int e2d2_version(void) { return 100; }
-
-e2d2_status e2d2_attn_encoder_blockcausal(const void* q, const void* k, const void* v, void* out,
-                                          float* lse, e2d2_dims dims, int L, int S,
-                                          cudaStream_t stream) {
-    if (!q || !k || !v || !out) return E2D2_ERR_INVALID_ARG;
-    return train_common(kEncoder, q, k, v, nullptr, nullptr, out, lse, dims, L, S, stream);
-}
-
-e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_enc, const void* v_enc,
-                                    const void* k_dec, const void* v_dec, void* out, float* lse,
-                                    e2d2_dims dims, int L, int S, cudaStream_t stream) {
-    if (!q_dec || !k_enc || !v_enc || !k_dec || !v_dec || !out) return E2D2_ERR_INVALID_ARG;
-    return train_common(kDecoderTrain, q_dec, k_enc, v_enc, k_dec, v_dec, out, lse, dims, L, S, stream);
-}
-
-size_t e2d2_attn_decoder_sample_workspace(e2d2_dims dims, int S, int capacity) {
-    if (check_dims(dims) != E2D2_OK || S <= 0 || capacity < 0) return 0;
-    return sample_layout(dims, S).bytes;
-}
-
-e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, const void* v_cache,
-                                     int capacity, int P, const void* k_blk, const void* v_blk,
-                                     void* out, float* lse, e2d2_dims dims, int S, void* workspace,
-                                     size_t ws_bytes, cudaStream_t stream) {
+// The sampling call; `append` (encoder block step) also writes the block's K/V to cache rows
+// P..P+S-1 from inside the same launch.
+e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, const void* v_cache, int capacity,
+                        int P, const void* k_blk, const void* v_blk, void* out, float* lse, e2d2_dims dims, int S,
+                        void* workspace, size_t ws_bytes, cudaStream_t stream) {
     if (!q_blk || !k_cache || !v_cache || !k_blk || !v_blk || !out) return E2D2_ERR_INVALID_ARG;
     e2d2_status s = check_dims(dims);
     if (s != E2D2_OK) return s;
     if (S <= 0 || capacity < 0 || P < 0) return E2D2_ERR_INVALID_ARG;
-    if (P > capacity) return E2D2_ERR_CAPACITY;
+    if (P > capacity || (append && static_cast<long long>(P) + S > capacity)) return E2D2_ERR_CAPACITY;
     const long long rows = static_cast<long long>(dims.batch) * dims.q_heads * S;
     if (rows > kMaxI32 / 8 || static_cast<long long>(capacity) * dims.batch * dims.kv_heads > kMaxI32)
         return E2D2_ERR_SHAPE;
@@ -333,6 +291,13 @@ e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, con
     prm.rows_cap = w.rows_cap;
     prm.q_chunk = q_chunk;
     prm.slot_floats = w.slot_floats;
+    if (append) {
+        prm.app_src_k = static_cast<const uint4*>(k_blk);
+        prm.app_src_v = static_cast<const uint4*>(v_blk);
+        prm.app_dst_k = static_cast<uint4*>(const_cast<void*>(k_cache));
+        prm.app_dst_v = static_cast<uint4*>(const_cast<void*>(v_cache));
+        prm.app_capacity = capacity;
+    }
     // Schedule: with U units on G CTAs, floor(U/G)*G units run whole (one CTA each, last); the
     // other R units are split stream-K over at most 5R CTAs (a unit has at most about six partials
     // to merge), and only as far as every piece keeps about kMinSplitTiles key tiles: publishing and
@@ -361,6 +326,65 @@ e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, con
         case 64: return launch_keyrow<64>(prm, static_cast<int>(grid), stream);
         default: return dispatch_fmha<kDecoderSample>(D, prm, static_cast<int>(grid), stream);
     }
+}
+
+}  // namespace
+}  // namespace e2d2
+
+using namespace e2d2;
+
+extern "C" {
+
+const char* e2d2_status_string(e2d2_status s) {
+    switch (s) {
+        case E2D2_OK: return "E2D2_OK";
+        case E2D2_ERR_INVALID_ARG: return "E2D2_ERR_INVALID_ARG";
+        case E2D2_ERR_UNSUPPORTED: return "E2D2_ERR_UNSUPPORTED";
+        case E2D2_ERR_SHAPE: return "E2D2_ERR_SHAPE";
+        case E2D2_ERR_ALIGNMENT: return "E2D2_ERR_ALIGNMENT";
+        case E2D2_ERR_CAPACITY: return "E2D2_ERR_CAPACITY";
+        case E2D2_ERR_WORKSPACE: return "E2D2_ERR_WORKSPACE";
+        case E2D2_ERR_CUDA: return "E2D2_ERR_CUDA";
+        case E2D2_ERR_TIMEOUT: return "E2D2_ERR_TIMEOUT";
+    }
+    return "E2D2_ERR_UNKNOWN";
+}
+
+int e2d2_version(void) { return 100; }
+
+e2d2_status e2d2_attn_encoder_blockcausal(const void* q, const void* k, const void* v, void* out,
+                                          float* lse, e2d2_dims dims, int L, int S,
+                                          cudaStream_t stream) {
+    if (!q || !k || !v || !out) return E2D2_ERR_INVALID_ARG;
+    return train_common(kEncoder, q, k, v, nullptr, nullptr, out, lse, dims, L, S, stream);
+}
+
+e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_enc, const void* v_enc,
+                                    const void* k_dec, const void* v_dec, void* out, float* lse,
+                                    e2d2_dims dims, int L, int S, cudaStream_t stream) {
+    if (!q_dec || !k_enc || !v_enc || !k_dec || !v_dec || !out) return E2D2_ERR_INVALID_ARG;
+    return train_common(kDecoderTrain, q_dec, k_enc, v_enc, k_dec, v_dec, out, lse, dims, L, S, stream);
+}
+
+size_t e2d2_attn_decoder_sample_workspace(e2d2_dims dims, int S, int capacity) {
+    if (check_dims(dims) != E2D2_OK || S <= 0 || capacity < 0) return 0;
+    return sample_layout(dims, S).bytes;
+}
+
+e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, const void* v_cache,
+                                     int capacity, int P, const void* k_blk, const void* v_blk,
+                                     void* out, float* lse, e2d2_dims dims, int S, void* workspace,
+                                     size_t ws_bytes, cudaStream_t stream) {
+    return sample_call(false, q_blk, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims, S, workspace,
+                       ws_bytes, stream);
+}
+
+e2d2_status e2d2_attn_encoder_block_step(const void* q_blk, void* k_cache, void* v_cache, int capacity, int P,
+                                         const void* k_blk, const void* v_blk, void* out, float* lse,
+                                         e2d2_dims dims, int S, void* workspace, size_t ws_bytes,
+                                         cudaStream_t stream) {
+    return sample_call(true, q_blk, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims, S, workspace,
+                       ws_bytes, stream);
 }
 
 e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int P, const void* k_new,

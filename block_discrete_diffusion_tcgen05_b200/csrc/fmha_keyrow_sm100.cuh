@@ -539,6 +539,9 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         uint32_t item_idx = 0;
         while (sched.next(it)) {
             const uint32_t ob = item_idx & 1;
+            // Encoder block step: the unit's own block joins the cache (the CTA that takes the
+            // own-block tile writes it, while its first products are still running).
+            if (p.app_dst_k != nullptr && it.t_begin == 0) append_block_rows(p, D, it.kv_z, wtid, 128);
             wait_bar_warp(&o_full[ob], (item_idx >> 1) & 1, abort_flag, p.err);
             wait_bar_warp(&l_ready[ob], (item_idx >> 1) & 1, abort_flag, p.err);
             ptx::tc_fence_after();

@@ -88,7 +88,30 @@ struct alignas(64) FmhaParams {
     int slot_floats;    // sample: floats per partial slot
     int rows_cap;       // sample: rows stored per partial slot
     int q_chunk;        // sample: packed query rows per TMEM lane quarter (multiple of 8, <= 32)
+    // sample, encoder block step only (null otherwise): the block's K/V rows are also written to
+    // the cache, rows P..P+S-1 of every (batch, kv head), by the CTA that takes the unit's own-block
+    // tile.  Rows [0, P) are the only cache rows the attention reads, so the two never overlap.
+    const uint4* app_src_k;  // [B*Hkv][S][D] bf16
+    const uint4* app_src_v;
+    uint4* app_dst_k;        // [B*Hkv][capacity][D] bf16
+    uint4* app_dst_v;
+    int app_capacity;
 };
+
+// Copies the S block rows of kv head kv_z (K and V) into cache rows P..P+S-1, 16 bytes per
+// thread-step, with `n` threads numbered `tid`.
+__device__ __forceinline__ void append_block_rows(const FmhaParams& p, int D, int kv_z, int tid, int n) {
+    const int vec_row = D / 8;
+    const int per = p.S * vec_row;
+    const size_t src0 = static_cast<size_t>(kv_z) * per;
+    const size_t dst0 = (static_cast<size_t>(kv_z) * p.app_capacity + p.P) * vec_row;
+    for (int i = tid; i < 2 * per; i += n) {
+        const bool is_v = i >= per;
+        const int e = is_v ? i - per : i;
+        const uint4 x = __ldg((is_v ? p.app_src_v : p.app_src_k) + src0 + e);
+        (is_v ? p.app_dst_v : p.app_dst_k)[dst0 + e] = x;
+    }
+}
 
 template <int D, int MODE>
 struct Cfg {
@@ -769,7 +792,14 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, kTmemCols);
     } else if (warp < 4) {
-        ptx::setmaxnreg_dec<kRegsControl>();  // idle warps of warpgroup 0
+        ptx::setmaxnreg_dec<kRegsControl>();
+        // Warps 2-3: the cache write of an encoder block step (sampling calls only), else idle.
+        if (MODE == kDecoderSample && p.app_dst_k != nullptr) {
+            Scheduler<MODE> sched(p);
+            Item it;
+            while (sched.next(it))
+                if (it.t_begin == 0 && it.q_row0 == 0) append_block_rows(p, D, it.kv_z, threadIdx.x - 64, 64);
+        }
     } else {
         ptx::setmaxnreg_inc<kRegsSoftmax>();
         // ------------------------------------------------------------------ softmax warpgroups

@@ -142,6 +142,21 @@ E2D2_API e2d2_status e2d2_attn_decoder_sample_noalloc(const void* q_blk, const v
                                              float* lse, e2d2_dims dims, int S, cudaStream_t stream);
 
 /*
+ * Encoder incremental block step ([E2D2 notes, sec. 3]: a finished block goes through the
+ * encoder, which updates the KV cache; sec. 4: the encoder's block-causal mask): the S clean
+ * queries of block b attend to the cached prefix (rows 0..P-1, P = bS) and, bidirectionally, to
+ * their own block -- the same rows of e2d2_attn_encoder_blockcausal over the whole sequence --
+ * and the block's K/V (k_blk, v_blk) are written to cache rows P..P+S-1 in the same launch.
+ *   Same layouts, workspace and errors as e2d2_attn_decoder_sample; requires P + S <= capacity
+ *   (else E2D2_ERR_CAPACITY, nothing launched).  Cache rows other than P..P+S-1 are not written.
+ *   The caller sets P += S after E2D2_OK.
+ */
+E2D2_API e2d2_status e2d2_attn_encoder_block_step(const void* q_blk, void* k_cache, void* v_cache, int capacity,
+                                                  int P, const void* k_blk, const void* v_blk, void* out,
+                                                  float* lse, e2d2_dims dims, int S, void* workspace,
+                                                  size_t ws_bytes, cudaStream_t stream);
+
+/*
  * KV-cache append ([E2D2 notes, sec. 3]: after a block is decoded the encoder absorbs it and
  * the cache grows by that block): rows P..P+S_new-1 of every (batch, kv head) cache take the
  * rows of k_new / v_new, bit for bit.  k_new, v_new [batch][kv_heads][S_new][d].  The cache

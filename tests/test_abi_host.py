@@ -70,6 +70,15 @@ def test_decoder_train_argument_errors(lib):
     assert f(P16, P16, P16, P16, P16, P16, None, DIMS, 64, -1, None) == 1
 
 
+def test_encoder_block_step_argument_errors(lib):
+    f = lib.e2d2_attn_encoder_block_step
+    ws = 1 << 20
+    # (q, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims, S, workspace, ws_bytes, stream)
+    assert f(P16, P16, P16, 20, 10, P16, P16, P16, None, DIMS, 16, P16, ws, None) == 5  # P + S > capacity
+    assert f(P16, P16, P16, 20, 21, P16, P16, P16, None, DIMS, 16, P16, ws, None) == 5  # P > capacity
+    assert f(P16, None, P16, 64, 0, P16, P16, P16, None, DIMS, 16, P16, ws, None) == 1  # null cache
+
+
 def test_sample_workspace_query_needs_no_gpu(lib):
     n = lib.e2d2_attn_decoder_sample_workspace(_lib.Dims(32, 16, 8, 128, 0.0), 16, 2064)
     assert n > 0

@@ -155,6 +155,31 @@ def test_long_sample_loop_shapes(oracle, P):
         H.compare(out[sl], lse[sl], ro, rl, f"long loop P{P} b{b}")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,S,b,d", [(2, 4, 2, 16, 5, 128), (1, 8, 2, 16, 200, 128), (2, 4, 4, 8, 20, 64),
+                                           (1, 2, 2, 16, 0, 128)])
+def test_encoder_block_step_matches_encoder_rows(oracle, B, Hq, Hkv, S, b, d):
+    """Encoder block step for block b (cache holding blocks 0..b-1) reproduces block b's rows of
+    the encoder over the whole (b+1) S tokens, and leaves the cache equal to the concatenation:
+    block b in rows bS..bS+S-1 bit for bit, earlier rows unchanged, later rows untouched."""
+    L, P = (b + 1) * S, b * S
+    cap = P + S + 24
+    q = H.gen((B, Hq, L, d), 7100 + b, 1.0)
+    k = H.gen((B, Hkv, L, d), 7101 + b, 1.0)
+    v = H.gen((B, Hkv, L, d), 7102 + b, 1.0)
+    kc = torch.full((B, Hkv, cap, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vc = torch.full_like(kc, float("nan"))
+    kc[:, :, :P] = k[1][:, :, :P]
+    vc[:, :, :P] = v[1][:, :, :P]
+    out, lse = attn.encoder_block_step(q[1][:, :, P:].contiguous(), kc, vc, P, k[1][:, :, P:].contiguous(),
+                                       v[1][:, :, P:].contiguous())
+    torch.cuda.synchronize()
+    ro, rl = oracle.encoder(q[0].f32, k[0].f32, v[0].f32, S)
+    H.compare(out, lse, ro[:, :, P:], rl[:, :, P:], f"encoder block step b{b} S{S} d{d}")
+    for cache, src in ((kc, k[1]), (vc, v[1])):
+        assert torch.equal(cache[:, :, :L].view(torch.int16), src.view(torch.int16))
+        assert torch.isnan(cache[:, :, L:].float()).all()
+
+
 def test_sample_equals_train_rows():
     """On the GPU: a sampling call for block b over the encoder prefix [0, bS) reproduces the
     decoder-train rows of block b (same inputs)."""
