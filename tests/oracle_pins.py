@@ -339,7 +339,41 @@ def pin_short_last_block(orc):
             assert abs(lse_d[0, h, i] - l) < 1e-12
 
 
+# ---------------------------------------------------------------------------------------
+# 13. Decoder-only block diffusion (BD3LM) for comparison: its training forward takes the clean
+#     and the noised sequence together (2L tokens) at attention cost 4ND(L^2 + LS) ([E2D2 notes],
+#     sec. 1 and the FLOPs table of sec. 4).  Read as: noised tokens see the noised tokens of their
+#     own block and the clean tokens of earlier blocks, clean tokens are block-causal.  That mask
+#     has L^2 + LS pairs (twice one E2D2 pass), and it is the decoder mask on the noised rows and
+#     the encoder mask on the clean rows; attention over the 2L tokens (torch SDPA on the explicit
+#     mask) equals one encoder call plus one decoder-train call with the same network's K/V.
+# ---------------------------------------------------------------------------------------
+def pin_bd3lm_vectorized_mask(orc):
+    for L, S in ((8, 2), (12, 3), (16, 4), (64, 8), (48, 16)):
+        blk = np.arange(L) // S
+        nn = blk[:, None] == blk[None, :]  # noised -> noised: own block
+        nc = blk[None, :] < blk[:, None]   # noised -> clean: earlier blocks
+        cc = blk[None, :] <= blk[:, None]  # clean -> clean: block-causal
+        full = np.block([[nn, nc], [np.zeros((L, L), dtype=bool), cc]])
+        assert int(full.sum()) == L * L + L * S, (L, S)
+        dec = orc.mask_decoder(L, S).astype(bool)  # columns 0..L-1 clean (encoder), L..2L-1 noised
+        assert (dec[:, :L] == nc).all() and (dec[:, L:] == nn).all(), (L, S)
+        assert (orc.mask_encoder(L, S).astype(bool) == cc).all(), (L, S)
+    B, H, L, S, d = 1, 2, 12, 4, 8
+    qn, kn, vn, qc, kc, vc = (_rand((B, H, L, d), 990 + t).astype(np.float64) for t in range(6))
+    blk = np.arange(L) // S
+    full = np.block([[blk[:, None] == blk[None, :], blk[None, :] < blk[:, None]],
+                     [np.zeros((L, L), dtype=bool), blk[None, :] <= blk[:, None]]])
+    q2, k2, v2 = (torch.from_numpy(np.concatenate(x, axis=2)) for x in ((qn, qc), (kn, kc), (vn, vc)))
+    ref = torch.nn.functional.scaled_dot_product_attention(q2, k2, v2, attn_mask=torch.from_numpy(full)).numpy()
+    out_n, _ = orc.decoder_train(qn, kc, vc, kn, vn, S=S)
+    out_c, _ = orc.encoder(qc, kc, vc, S=S)
+    np.testing.assert_allclose(out_n, ref[:, :, :L], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(out_c, ref[:, :, L:], rtol=0, atol=1e-10)
+
+
 ALL_PINS = [pin_pair_count, pin_golden_pairs, pin_block_size_one_is_causal,
             pin_block_size_L_is_bidirectional, pin_masked_against_torch, pin_brute_force,
             pin_zero_keys_closed_form, pin_constant_values, pin_gqa_is_repeated_heads,
-            pin_sample_is_train_slice, pin_append_is_concatenation, pin_short_last_block]
+            pin_sample_is_train_slice, pin_append_is_concatenation, pin_short_last_block,
+            pin_bd3lm_vectorized_mask]
