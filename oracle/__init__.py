@@ -69,8 +69,10 @@ class Oracle:
         lib.oracle_decoder_sample.argtypes = [_f32p, _f32p, _f32p, ii, ii, _f32p, _f32p,
                                               ii, ii, ii, ii, ii, ctypes.c_double, _f64p, _f64p]
         lib.oracle_kv_append.argtypes = [_u16p, _u16p, ii, ii, _u16p, _u16p, ii, ii, ii, ii]
+        lib.oracle_encoder_backward.argtypes = [_f32p] * 4 + [ii] * 6 + [ctypes.c_double] + [_f64p] * 3
+        lib.oracle_decoder_train_backward.argtypes = [_f32p] * 6 + [ii] * 6 + [ctypes.c_double] + [_f64p] * 5
         for name in ("oracle_encoder", "oracle_decoder_train", "oracle_decoder_sample",
-                     "oracle_kv_append"):
+                     "oracle_kv_append", "oracle_encoder_backward", "oracle_decoder_train_backward"):
             getattr(lib, name).restype = ctypes.c_int
         self.lib = lib
 
@@ -131,6 +133,39 @@ class Oracle:
         if rc:
             raise RuntimeError(f"oracle_decoder_train failed ({rc})")
         return out, lse
+
+    # ---- backward of the train calls ----------------------------------------------
+    def encoder_backward(self, q, k, v, dout, S: int, scale: float = 0.0):
+        """Gradients of sum(dout * encoder(q, k, v)) -> (dq [B,Hq,L,d], dk, dv [B,Hkv,L,d]), fp64."""
+        B, Hq, L, d = q.shape
+        Hkv = k.shape[1]
+        assert k.shape == (B, Hkv, L, d) and v.shape == k.shape and dout.shape == q.shape
+        arrs = [self._f32(t) for t in (q, k, v, dout)]
+        dq = np.zeros((B, Hq, L, d), dtype=np.float64)
+        dk = np.zeros((B, Hkv, L, d), dtype=np.float64)
+        dv = np.zeros((B, Hkv, L, d), dtype=np.float64)
+        rc = self.lib.oracle_encoder_backward(*[p for _, p in arrs], B, Hq, Hkv, L, S, d, float(scale),
+                                              *[t.ctypes.data_as(_f64p) for t in (dq, dk, dv)])
+        if rc:
+            raise RuntimeError(f"oracle_encoder_backward failed ({rc})")
+        return dq, dk, dv
+
+    def decoder_train_backward(self, q, k_enc, v_enc, k_dec, v_dec, dout, S: int, scale: float = 0.0):
+        """Gradients of sum(dout * decoder_train(...)) -> (dq, dk_enc, dv_enc, dk_dec, dv_dec), fp64."""
+        B, Hq, L, d = q.shape
+        Hkv = k_enc.shape[1]
+        for t in (k_enc, v_enc, k_dec, v_dec):
+            assert t.shape == (B, Hkv, L, d)
+        assert dout.shape == q.shape
+        arrs = [self._f32(t) for t in (q, k_enc, v_enc, k_dec, v_dec, dout)]
+        dq = np.zeros((B, Hq, L, d), dtype=np.float64)
+        grads = [np.zeros((B, Hkv, L, d), dtype=np.float64) for _ in range(4)]
+        rc = self.lib.oracle_decoder_train_backward(*[p for _, p in arrs], B, Hq, Hkv, L, S, d, float(scale),
+                                                    dq.ctypes.data_as(_f64p),
+                                                    *[t.ctypes.data_as(_f64p) for t in grads])
+        if rc:
+            raise RuntimeError(f"oracle_decoder_train_backward failed ({rc})")
+        return (dq, *grads)
 
     def decoder_sample(self, q, k_cache, v_cache, P: int, k_blk, v_blk, scale: float = 0.0):
         """q [B,Hq,S,d]; caches [B,Hkv,cap,d] (first P rows valid); k_blk/v_blk [B,Hkv,S,d]."""

@@ -252,3 +252,153 @@ int oracle_kv_append(uint16_t* k_cache, uint16_t* v_cache, int capacity, int P,
             }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Backward of the train calls ([E2D2 notes, sec. 4]: the training algorithm takes one
+ * encoder pass and one decoder pass over all blocks, forward and backward).  From the chain
+ * rule applied to the definition at the top of this file, with p_ij = exp(s_ij - lse_i) over
+ * the allowed keys of row i and dout the gradient of the loss with respect to out:
+ *   dv_j   += sum_i p_ij dout_i
+ *   dp_ij   = dout_i . v_j
+ *   ds_ij   = p_ij (dp_ij - sum_j' p_ij' dp_ij')
+ *   dq_i    = scale sum_j ds_ij k_j
+ *   dk_j   += scale sum_i ds_ij q_i
+ * The forward quantities are recomputed here (no reuse of the kernel's LSE).  dk, dv of a kv
+ * head collect the contributions of all G query heads that share it.
+ * --------------------------------------------------------------------------------------- */
+
+/* One query head: nq queries over nk keys.  Writes dq [nq][d], adds into dk, dv [nk][d]. */
+static int attend_backward(const float* q, const double* keys, const double* vals, const uint8_t* mask,
+                           const float* dout, int nq, int nk, int d, double scale, double* dq,
+                           double* dk, double* dv) {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1));
+    double* dp = (double*)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1));
+    if (!s || !dp) { free(s); free(dp); return -2; }
+    int rc = 0;
+    for (int i = 0; i < nq; ++i) {
+        const uint8_t* mrow = mask + (size_t)i * nk;
+        const float* qi = q + (size_t)i * d;
+        const float* gi = dout + (size_t)i * d;
+        double* dqi = dq + (size_t)i * d;
+        for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+        double m = -INFINITY;
+        int any = 0;
+        for (int j = 0; j < nk; ++j) {
+            if (!mrow[j]) continue;
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += (double)qi[c] * keys[(size_t)j * d + c];
+            s[j] = scale * acc;
+            if (!any || s[j] > m) m = s[j];
+            any = 1;
+        }
+        if (!any) { rc = -1; continue; }
+        double l = 0.0;
+        for (int j = 0; j < nk; ++j)
+            if (mrow[j]) l += exp(s[j] - m);
+        const double lse = m + log(l);
+        double dsum = 0.0;  /* sum_j p_ij dp_ij */
+        for (int j = 0; j < nk; ++j) {
+            if (!mrow[j]) continue;
+            const double p = exp(s[j] - lse);
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) {
+                acc += (double)gi[c] * vals[(size_t)j * d + c];
+                dv[(size_t)j * d + c] += p * (double)gi[c];
+            }
+            dp[j] = acc;
+            dsum += p * acc;
+        }
+        for (int j = 0; j < nk; ++j) {
+            if (!mrow[j]) continue;
+            const double ds = exp(s[j] - lse) * (dp[j] - dsum);
+            for (int c = 0; c < d; ++c) {
+                dqi[c] += scale * ds * keys[(size_t)j * d + c];
+                dk[(size_t)j * d + c] += scale * ds * (double)qi[c];
+            }
+        }
+    }
+    free(s);
+    free(dp);
+    return rc;
+}
+
+/* Encoder backward.  q, dout: [B][Hq][L][d]; k, v: [B][Hkv][L][d];
+ * dq: [B][Hq][L][d]; dk, dv: [B][Hkv][L][d] (fp64, overwritten). */
+int oracle_encoder_backward(const float* q, const float* k, const float* v, const float* dout, int B, int Hq,
+                            int Hkv, int L, int S, int d, double scale, double* dq, double* dk, double* dv) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L < 0 || S <= 0 || d <= 0) return -3;
+    const int G = Hq / Hkv;
+    scale = resolve_scale(scale, d);
+    uint8_t* mask = (uint8_t*)malloc((size_t)L * L + 1);
+    if (!mask) return -2;
+    oracle_mask_encoder(L, S, mask);
+    int rc = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : rc)
+    for (int b = 0; b < B; ++b) {
+        for (int g = 0; g < Hkv; ++g) {
+            const size_t ko = ((size_t)b * Hkv + g) * L * d;
+            double* kd = (double*)malloc(sizeof(double) * ((size_t)L * d + 1));
+            double* vd = (double*)malloc(sizeof(double) * ((size_t)L * d + 1));
+            if (!kd || !vd) { rc |= 2; free(kd); free(vd); continue; }
+            rows_to_double(k + ko, L, d, kd);
+            rows_to_double(v + ko, L, d, vd);
+            for (size_t t = 0; t < (size_t)L * d; ++t) { dk[ko + t] = 0.0; dv[ko + t] = 0.0; }
+            for (int h = g * G; h < (g + 1) * G; ++h) {
+                const size_t qo = ((size_t)b * Hq + h) * L * d;
+                if (attend_backward(q + qo, kd, vd, mask, dout + qo, L, L, d, scale, dq + qo, dk + ko, dv + ko))
+                    rc |= 1;
+            }
+            free(kd);
+            free(vd);
+        }
+    }
+    free(mask);
+    return rc ? -1 : 0;
+}
+
+/* Decoder-train backward over the 2L keys (k_enc rows, then k_dec rows).  q, dout:
+ * [B][Hq][L][d]; k_*, v_*: [B][Hkv][L][d]; dq: [B][Hq][L][d]; dk_enc, dv_enc, dk_dec,
+ * dv_dec: [B][Hkv][L][d] (fp64, overwritten). */
+int oracle_decoder_train_backward(const float* q, const float* k_enc, const float* v_enc, const float* k_dec,
+                                  const float* v_dec, const float* dout, int B, int Hq, int Hkv, int L, int S,
+                                  int d, double scale, double* dq, double* dk_enc, double* dv_enc,
+                                  double* dk_dec, double* dv_dec) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L < 0 || S <= 0 || d <= 0) return -3;
+    const int G = Hq / Hkv;
+    scale = resolve_scale(scale, d);
+    const size_t W = (size_t)2 * L;
+    uint8_t* mask = (uint8_t*)malloc((size_t)L * W + 1);
+    if (!mask) return -2;
+    oracle_mask_decoder(L, S, mask);
+    int rc = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : rc)
+    for (int b = 0; b < B; ++b) {
+        for (int g = 0; g < Hkv; ++g) {
+            const size_t ko = ((size_t)b * Hkv + g) * L * d;
+            double* kd = (double*)malloc(sizeof(double) * (W * d + 1));
+            double* vd = (double*)malloc(sizeof(double) * (W * d + 1));
+            double* dkd = (double*)calloc(W * d + 1, sizeof(double));
+            double* dvd = (double*)calloc(W * d + 1, sizeof(double));
+            if (!kd || !vd || !dkd || !dvd) { rc |= 2; free(kd); free(vd); free(dkd); free(dvd); continue; }
+            rows_to_double(k_enc + ko, L, d, kd);
+            rows_to_double(k_dec + ko, L, d, kd + (size_t)L * d);
+            rows_to_double(v_enc + ko, L, d, vd);
+            rows_to_double(v_dec + ko, L, d, vd + (size_t)L * d);
+            for (int h = g * G; h < (g + 1) * G; ++h) {
+                const size_t qo = ((size_t)b * Hq + h) * L * d;
+                if (attend_backward(q + qo, kd, vd, mask, dout + qo, L, (int)W, d, scale, dq + qo, dkd, dvd))
+                    rc |= 1;
+            }
+            memcpy(dk_enc + ko, dkd, sizeof(double) * (size_t)L * d);
+            memcpy(dk_dec + ko, dkd + (size_t)L * d, sizeof(double) * (size_t)L * d);
+            memcpy(dv_enc + ko, dvd, sizeof(double) * (size_t)L * d);
+            memcpy(dv_dec + ko, dvd + (size_t)L * d, sizeof(double) * (size_t)L * d);
+            free(kd);
+            free(vd);
+            free(dkd);
+            free(dvd);
+        }
+    }
+    free(mask);
+    return rc ? -1 : 0;
+}

@@ -372,8 +372,79 @@ def pin_bd3lm_vectorized_mask(orc):
     np.testing.assert_allclose(out_c, ref[:, :, L:], rtol=0, atol=1e-10)
 
 
+# ---------------------------------------------------------------------------------------
+# 14. Backward of the train calls ([E2D2 notes, sec. 4]: one encoder and one decoder pass, forward
+#     and backward).  (a) torch autograd in fp64 through SDPA on masks built here from the block
+#     rule (GQA through repeated kv heads, whose gradients autograd sums; a short last block);
+#     (b) central differences of the oracle's forward on exactly representable inputs;
+#     (c) constant values: out does not depend on q or k (dq = dk = 0) and the dv rows sum to the
+#     dout rows (every softmax row sums to one).
+# ---------------------------------------------------------------------------------------
+def _block_masks(L, S):
+    blk = np.arange(L) // S
+    enc = blk[None, :] <= blk[:, None]
+    dec = np.concatenate([blk[None, :] < blk[:, None], blk[None, :] == blk[:, None]], axis=1)
+    return enc, dec
+
+
+def pin_backward_against_autograd(orc):
+    B, Hq, Hkv, L, S, d, scale = 2, 4, 2, 20, 6, 8, 0.5
+    G = Hq // Hkv
+    q, dout = (_rand((B, Hq, L, d), 1000 + t) for t in range(2))
+    k, v, ke, ve = (_rand((B, Hkv, L, d), 1002 + t) for t in range(4))
+    enc_m, dec_m = (torch.from_numpy(m) for m in _block_masks(L, S))
+    t64 = lambda a: torch.tensor(np.asarray(a, dtype=np.float64), requires_grad=True)
+    rep = lambda t: t.repeat_interleave(G, dim=1)
+    sdpa = torch.nn.functional.scaled_dot_product_attention
+    g = torch.from_numpy(np.asarray(dout, dtype=np.float64))
+    # encoder
+    tq, tk, tv = t64(q), t64(k), t64(v)
+    (sdpa(tq, rep(tk), rep(tv), attn_mask=enc_m, scale=scale) * g).sum().backward()
+    dq, dk, dv = orc.encoder_backward(q, k, v, dout, S=S, scale=scale)
+    for mine, ref in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(mine, ref.grad.numpy(), rtol=0, atol=1e-10)
+    # decoder-train: keys are the encoder-side rows, then the decoder-side rows
+    tq, tke, tve, tkd, tvd = t64(q), t64(ke), t64(ve), t64(k), t64(v)
+    kk, vv = torch.cat([rep(tke), rep(tkd)], dim=2), torch.cat([rep(tve), rep(tvd)], dim=2)
+    (sdpa(tq, kk, vv, attn_mask=dec_m, scale=scale) * g).sum().backward()
+    grads = orc.decoder_train_backward(q, ke, ve, k, v, dout, S=S, scale=scale)
+    for mine, ref in zip(grads, (tq, tke, tve, tkd, tvd)):
+        np.testing.assert_allclose(mine, ref.grad.numpy(), rtol=0, atol=1e-10)
+
+
+def pin_backward_finite_differences(orc):
+    B, Hq, Hkv, L, S, d, scale = 1, 1, 1, 5, 2, 3, 0.8
+    rng = np.random.default_rng(1010)
+    grid = lambda shape: (rng.integers(-512, 512, size=shape) / 1024.0).astype(np.float32)  # exact in fp32
+    q, k, v, ke, ve, dout = (grid((B, Hq, L, d)) for _ in range(6))
+    h = np.float32(2.0 ** -8)
+
+    def f_enc(qq, kk, vv):
+        return float((orc.encoder(qq, kk, vv, S=S, scale=scale)[0] * dout).sum())
+
+    def f_dec(qq, kke, vve, kkd, vvd):
+        return float((orc.decoder_train(qq, kke, vve, kkd, vvd, S=S, scale=scale)[0] * dout).sum())
+
+    grads_e = orc.encoder_backward(q, k, v, dout, S=S, scale=scale)
+    grads_d = orc.decoder_train_backward(q, ke, ve, k, v, dout, S=S, scale=scale)
+    for f, args, grads in ((f_enc, [q, k, v], grads_e), (f_dec, [q, ke, ve, k, v], grads_d)):
+        for a, ga in zip(range(len(args)), grads):
+            for idx in ((0, 0, 0, 0), (0, 0, 2, 1), (0, 0, L - 1, d - 1), (0, 0, 3, 2)):
+                plus = [x.copy() for x in args]
+                minus = [x.copy() for x in args]
+                plus[a][idx] += h
+                minus[a][idx] -= h
+                num = (f(*plus) - f(*minus)) / (2.0 * float(h))
+                assert abs(num - ga[idx]) <= 2e-4 + 2e-3 * abs(ga[idx]), (f.__name__, a, idx, num, ga[idx])
+    # constant values
+    vc = np.full_like(v, 0.375)
+    dq, dk, dv = orc.encoder_backward(q, k, vc, dout, S=S, scale=scale)
+    assert np.abs(dq).max() < 1e-12 and np.abs(dk).max() < 1e-12
+    np.testing.assert_allclose(dv.sum(axis=2), dout.astype(np.float64).sum(axis=2), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [pin_pair_count, pin_golden_pairs, pin_block_size_one_is_causal,
             pin_block_size_L_is_bidirectional, pin_masked_against_torch, pin_brute_force,
             pin_zero_keys_closed_form, pin_constant_values, pin_gqa_is_repeated_heads,
             pin_sample_is_train_slice, pin_append_is_concatenation, pin_short_last_block,
-            pin_bd3lm_vectorized_mask]
+            pin_bd3lm_vectorized_mask, pin_backward_against_autograd, pin_backward_finite_differences]

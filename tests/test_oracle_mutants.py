@@ -44,6 +44,17 @@ MUTANTS = [
     ("append-off-by-one", "capacity + P + r) * d;", "capacity + P + r + 1) * d;"),
     ("append-swaps-k-and-v", "memcpy(v_cache + dst, v_new + src, sizeof(uint16_t) * d);",
      "memcpy(v_cache + dst, k_new + src, sizeof(uint16_t) * d);"),
+    # backward of the train calls
+    ("bwd-drops-row-term", "const double ds = exp(s[j] - lse) * (dp[j] - dsum);",
+     "const double ds = exp(s[j] - lse) * dp[j];"),
+    ("bwd-dk-wrong-sign", "dk[(size_t)j * d + c] += scale * ds * (double)qi[c];",
+     "dk[(size_t)j * d + c] -= scale * ds * (double)qi[c];"),
+    ("bwd-dq-missing-scale", "dqi[c] += scale * ds * keys[(size_t)j * d + c];",
+     "dqi[c] += ds * keys[(size_t)j * d + c];"),
+    ("bwd-dv-without-p", "dv[(size_t)j * d + c] += p * (double)gi[c];",
+     "dv[(size_t)j * d + c] += (double)gi[c];"),
+    ("bwd-dec-swaps-sources", "memcpy(dk_enc + ko, dkd, sizeof(double) * (size_t)L * d);",
+     "memcpy(dk_enc + ko, dkd + (size_t)L * d, sizeof(double) * (size_t)L * d);"),
 ]
 
 _RUNNER = r"""
