@@ -17,7 +17,9 @@ STATUS = {0: "E2D2_OK", 1: "E2D2_ERR_INVALID_ARG", 2: "E2D2_ERR_UNSUPPORTED", 3:
 EXPORTS = ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
            "e2d2_attn_decoder_sample_workspace", "e2d2_attn_decoder_sample",
            "e2d2_kv_cache_append", "e2d2_status_string", "e2d2_last_device_error", "e2d2_version",
-           "e2d2_attn_decoder_sample_noalloc", "e2d2_attn_encoder_block_step")
+           "e2d2_attn_decoder_sample_noalloc", "e2d2_attn_encoder_block_step",
+           "e2d2_attn_train_backward_workspace", "e2d2_attn_encoder_backward",
+           "e2d2_attn_decoder_train_backward")
 
 # E2D2_SAMPLE_NOALLOC_MAX_BYTES of include/e2d2_attn.h
 SAMPLE_NOALLOC_MAX_BYTES = 32 << 20
@@ -62,12 +64,18 @@ def load(path: Path | str | None = None):
                                                  ctypes.c_size_t, st]
     lib.e2d2_attn_decoder_sample_noalloc.argtypes = [vp, vp, vp, ci, ci, vp, vp, vp, fp, Dims, ci, st]
     lib.e2d2_attn_decoder_sample_noalloc.restype = ctypes.c_int
+    lib.e2d2_attn_train_backward_workspace.argtypes = [Dims, ci]
+    lib.e2d2_attn_train_backward_workspace.restype = ctypes.c_size_t
+    lib.e2d2_attn_encoder_backward.argtypes = [vp, vp, vp, fp, vp, vp, vp, vp, Dims, ci, ci, vp,
+                                               ctypes.c_size_t, st]
+    lib.e2d2_attn_decoder_train_backward.argtypes = [vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, vp, vp,
+                                                     Dims, ci, ci, vp, ctypes.c_size_t, st]
     lib.e2d2_status_string.argtypes = [ci]
     lib.e2d2_status_string.restype = ctypes.c_char_p
     lib.e2d2_last_device_error.argtypes = [st]
     for name in ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
                  "e2d2_attn_decoder_sample", "e2d2_kv_cache_append", "e2d2_last_device_error",
-                 "e2d2_version"):
+                 "e2d2_version", "e2d2_attn_encoder_backward", "e2d2_attn_decoder_train_backward"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib

@@ -3,11 +3,13 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
+#include "attn_bwd_simple.cuh"
 #include "e2d2_attn.h"
 #include "fmha_keyrow_sm100.cuh"
 #include "fmha_sm100.cuh"
@@ -211,6 +213,60 @@ e2d2_status train_common(int mode, const void* q, const void* k0, const void* v0
                             : dispatch_fmha<kDecoderTrain>(D, prm, grid, st);
 }
 
+// Backward of the train calls: dq (and D_i = sum_j p_ij dout_i.v_j into the workspace), then dk/dv.
+e2d2_status train_backward(bool decoder, const BwdParams& base, const e2d2_dims& dm, int L, int S,
+                           void* workspace, size_t ws_bytes, cudaStream_t st) {
+    e2d2_status s = check_dims(dm);
+    if (s != E2D2_OK) return s;
+    s = check_train_shape(dm, L, S);
+    if (s != E2D2_OK) return s;
+    const size_t need = static_cast<size_t>(dm.batch) * dm.q_heads * L * sizeof(float);
+    if (!workspace || ws_bytes < need) return E2D2_ERR_WORKSPACE;
+    const void* ptrs[] = {base.q, base.k0, base.v0, base.dout, base.dq, base.dk0, base.dv0, workspace};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return E2D2_ERR_ALIGNMENT;
+    if (decoder && (!aligned16(base.k1) || !aligned16(base.v1) || !aligned16(base.dk1) || !aligned16(base.dv1)))
+        return E2D2_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(base.lse) & 3u) return E2D2_ERR_ALIGNMENT;
+    DeviceInfo* di = nullptr;
+    s = device_info(&di);
+    if (s != E2D2_OK) return s;
+
+    BwdParams prm = base;
+    prm.dsum = static_cast<float*>(workspace);
+    prm.batch = dm.batch;
+    prm.q_heads = dm.q_heads;
+    prm.kv_heads = dm.kv_heads;
+    prm.group = dm.q_heads / dm.kv_heads;
+    prm.L = L;
+    prm.S = S;
+    prm.scale = static_cast<float>(dm.scale > 0.f ? static_cast<double>(dm.scale)
+                                                  : 1.0 / std::sqrt(static_cast<double>(dm.head_dim)));
+    prm.decoder = decoder ? 1 : 0;
+    constexpr int kWarpsPerBlock = 8;
+    const long long cap = static_cast<long long>(di->sms) * 16;  // 16 blocks of 8 warps per SM
+    const long long rows = static_cast<long long>(dm.batch) * dm.q_heads * L;
+    const long long keys = static_cast<long long>(dm.batch) * dm.kv_heads * L * (decoder ? 2 : 1);
+    const unsigned g1 = static_cast<unsigned>(std::min(cap, (rows + kWarpsPerBlock - 1) / kWarpsPerBlock));
+    const unsigned g2 = static_cast<unsigned>(std::min(cap, (keys + kWarpsPerBlock - 1) / kWarpsPerBlock));
+    switch (dm.head_dim) {
+        case 32:
+            attn_bwd_dq_kernel<32><<<g1, 32 * kWarpsPerBlock, 0, st>>>(prm);
+            attn_bwd_dkv_kernel<32><<<g2, 32 * kWarpsPerBlock, 0, st>>>(prm);
+            break;
+        case 64:
+            attn_bwd_dq_kernel<64><<<g1, 32 * kWarpsPerBlock, 0, st>>>(prm);
+            attn_bwd_dkv_kernel<64><<<g2, 32 * kWarpsPerBlock, 0, st>>>(prm);
+            break;
+        case 128:
+            attn_bwd_dq_kernel<128><<<g1, 32 * kWarpsPerBlock, 0, st>>>(prm);
+            attn_bwd_dkv_kernel<128><<<g2, 32 * kWarpsPerBlock, 0, st>>>(prm);
+            break;
+        default: return E2D2_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+}
+
 struct SampleLayout {
     int rows_cap;
     int slot_floats;
@@ -364,6 +420,53 @@ e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_enc, const 
                                     e2d2_dims dims, int L, int S, cudaStream_t stream) {
     if (!q_dec || !k_enc || !v_enc || !k_dec || !v_dec || !out) return E2D2_ERR_INVALID_ARG;
     return train_common(kDecoderTrain, q_dec, k_enc, v_enc, k_dec, v_dec, out, lse, dims, L, S, stream);
+}
+
+size_t e2d2_attn_train_backward_workspace(e2d2_dims dims, int L) {
+    if (check_dims(dims) != E2D2_OK || L <= 0) return 0;
+    return static_cast<size_t>(dims.batch) * dims.q_heads * L * sizeof(float);
+}
+
+e2d2_status e2d2_attn_encoder_backward(const void* q, const void* k, const void* v, const float* lse,
+                                       const void* dout, void* dq, void* dk, void* dv, e2d2_dims dims, int L,
+                                       int S, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!q || !k || !v || !lse || !dout || !dq || !dk || !dv) return E2D2_ERR_INVALID_ARG;
+    BwdParams b;
+    std::memset(&b, 0, sizeof(b));
+    b.q = static_cast<const __nv_bfloat16*>(q);
+    b.k0 = static_cast<const __nv_bfloat16*>(k);
+    b.v0 = static_cast<const __nv_bfloat16*>(v);
+    b.lse = lse;
+    b.dout = static_cast<const __nv_bfloat16*>(dout);
+    b.dq = static_cast<__nv_bfloat16*>(dq);
+    b.dk0 = static_cast<__nv_bfloat16*>(dk);
+    b.dv0 = static_cast<__nv_bfloat16*>(dv);
+    return train_backward(false, b, dims, L, S, workspace, ws_bytes, stream);
+}
+
+e2d2_status e2d2_attn_decoder_train_backward(const void* q_dec, const void* k_enc, const void* v_enc,
+                                             const void* k_dec, const void* v_dec, const float* lse,
+                                             const void* dout, void* dq, void* dk_enc, void* dv_enc, void* dk_dec,
+                                             void* dv_dec, e2d2_dims dims, int L, int S, void* workspace,
+                                             size_t ws_bytes, cudaStream_t stream) {
+    if (!q_dec || !k_enc || !v_enc || !k_dec || !v_dec || !lse || !dout || !dq || !dk_enc ||
+        !dv_enc || !dk_dec || !dv_dec)
+        return E2D2_ERR_INVALID_ARG;
+    BwdParams b;
+    std::memset(&b, 0, sizeof(b));
+    b.q = static_cast<const __nv_bfloat16*>(q_dec);
+    b.k0 = static_cast<const __nv_bfloat16*>(k_enc);
+    b.v0 = static_cast<const __nv_bfloat16*>(v_enc);
+    b.k1 = static_cast<const __nv_bfloat16*>(k_dec);
+    b.v1 = static_cast<const __nv_bfloat16*>(v_dec);
+    b.lse = lse;
+    b.dout = static_cast<const __nv_bfloat16*>(dout);
+    b.dq = static_cast<__nv_bfloat16*>(dq);
+    b.dk0 = static_cast<__nv_bfloat16*>(dk_enc);
+    b.dv0 = static_cast<__nv_bfloat16*>(dv_enc);
+    b.dk1 = static_cast<__nv_bfloat16*>(dk_dec);
+    b.dv1 = static_cast<__nv_bfloat16*>(dv_dec);
+    return train_backward(true, b, dims, L, S, workspace, ws_bytes, stream);
 }
 
 size_t e2d2_attn_decoder_sample_workspace(e2d2_dims dims, int S, int capacity) {

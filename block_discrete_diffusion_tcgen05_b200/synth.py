@@ -12,7 +12,7 @@ from dataclasses import dataclass
 import numpy as np
 
 TENSOR_ID = {"q": 0, "k": 1, "v": 2, "k_enc": 3, "v_enc": 4, "k_dec": 5, "v_dec": 6,
-             "k_new": 7, "v_new": 8, "k_cache": 9, "v_cache": 10}
+             "k_new": 7, "v_new": 8, "k_cache": 9, "v_cache": 10, "dout": 11}
 
 
 def seed_for(workload: int, layer: int, tensor: str) -> int:

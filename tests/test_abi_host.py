@@ -27,7 +27,9 @@ def header_functions():
 def test_header_declares_the_boundary():
     names = set(header_functions())
     assert {"e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train", "e2d2_attn_decoder_sample",
-            "e2d2_kv_cache_append", "e2d2_attn_decoder_sample_workspace"} <= names
+            "e2d2_kv_cache_append", "e2d2_attn_decoder_sample_workspace", "e2d2_attn_encoder_block_step",
+            "e2d2_attn_train_backward_workspace", "e2d2_attn_encoder_backward",
+            "e2d2_attn_decoder_train_backward"} <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -77,6 +79,45 @@ def test_encoder_block_step_argument_errors(lib):
     assert f(P16, P16, P16, 20, 10, P16, P16, P16, None, DIMS, 16, P16, ws, None) == 5  # P + S > capacity
     assert f(P16, P16, P16, 20, 21, P16, P16, P16, None, DIMS, 16, P16, ws, None) == 5  # P > capacity
     assert f(P16, None, P16, 64, 0, P16, P16, P16, None, DIMS, 16, P16, ws, None) == 1  # null cache
+
+
+def test_train_backward_workspace_query_needs_no_gpu(lib):
+    # one float (D_i = dout_i . out_i) per query row
+    assert lib.e2d2_attn_train_backward_workspace(DIMS, 64) == 2 * 4 * 64 * 4
+    assert lib.e2d2_attn_train_backward_workspace(_lib.Dims(2, 4, 2, 96, 0.0), 64) == 0
+    assert lib.e2d2_attn_train_backward_workspace(DIMS, 0) == 0
+
+
+def test_encoder_backward_argument_errors(lib):
+    f = lib.e2d2_attn_encoder_backward
+    ws = lib.e2d2_attn_train_backward_workspace(DIMS, 64)
+    # (q, k, v, lse, dout, dq, dk, dv, dims, L, S, workspace, ws_bytes, stream)
+    a = [P16] * 8
+    assert f(*a[:3], None, *a[4:], DIMS, 64, 8, P16, ws, None) == 1                 # lse is required
+    assert f(*a[:7], None, DIMS, 64, 8, P16, ws, None) == 1                         # null dv
+    assert f(*a, DIMS, 64, 8, P16, ws - 1, None) == 6                               # small workspace
+    assert f(*a, DIMS, 64, 8, None, ws, None) == 6                                  # no workspace
+    assert f(P16 + 8, *a[1:], DIMS, 64, 8, P16, ws, None) == 4                      # misaligned q
+    assert f(*a[:3], P16 + 2, *a[4:], DIMS, 64, 8, P16, ws, None) == 4              # misaligned lse
+    assert f(*a, DIMS, 64, 8, P16 + 4, ws, None) == 4                               # misaligned workspace
+    assert f(*a, DIMS, 64, 0, P16, ws, None) == 1                                   # S = 0
+    assert f(*a, _lib.Dims(2, 4, 2, 96, 0.0), 64, 8, P16, ws, None) == 2            # head_dim
+    assert f(*a, _lib.Dims(2, 4, 3, 64, 0.0), 64, 8, P16, ws, None) == 1            # GQA ratio
+    # a short last block passes the shape checks (stopped here by the misaligned lse)
+    assert f(*a[:3], P16 + 2, *a[4:], DIMS, 60, 8, P16, ws, None) == 4
+
+
+def test_decoder_train_backward_argument_errors(lib):
+    f = lib.e2d2_attn_decoder_train_backward
+    ws = lib.e2d2_attn_train_backward_workspace(DIMS, 64)
+    # (q, k_enc, v_enc, k_dec, v_dec, lse, dout, dq, dk_enc, dv_enc, dk_dec, dv_dec, dims, L, S,
+    #  workspace, ws_bytes, stream)
+    a = [P16] * 12
+    assert f(*a[:11], None, DIMS, 64, 8, P16, ws, None) == 1                        # null dv_dec
+    assert f(*a[:5], None, *a[6:], DIMS, 64, 8, P16, ws, None) == 1                 # lse is required
+    assert f(*a[:10], P16 + 8, a[11], DIMS, 64, 8, P16, ws, None) == 4              # misaligned dk_dec
+    assert f(*a, DIMS, 64, 8, P16, ws - 4, None) == 6
+    assert f(*a, DIMS, -1, 8, P16, ws, None) == 1
 
 
 def test_sample_workspace_query_needs_no_gpu(lib):
