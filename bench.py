@@ -191,7 +191,9 @@ def run_workload_set(torch, attn, workloads, dev, peaks):
       long_sample_loop         B4 S16 Hq32 Hkv8 d128, 8 layers: for each of 512 blocks, 16 denoise
                                steps x 8 decoder sampling calls with P = 16 n, then one KV-cache
                                append per layer; eager launches from Python as a user would make
-                               them; device time per quarter of the loop (P ranges)."""
+                               them; device time per quarter of the loop (P ranges).
+    and the backward of the train pass (B8 L1024 S16 H16 d64: encoder and decoder-train backward
+    calls, 2 warm-up + 5 timed, no L2 flush: each call lasts milliseconds)."""
     g = torch.Generator(device=dev)
     g.manual_seed(4242)
 
@@ -235,6 +237,34 @@ def run_workload_set(torch, attn, workloads, dev, peaks):
         "frac_tensor": fl / step_s / 1e12 / tc, "frac_attainable": fl / step_s / attainable,
         "launches_per_step": tc_shape.enc_calls + tc_shape.dec_calls}
     del enc_layers, dec_layers
+    # ---- backward of the train pass (first, CUDA-core kernels)
+    tr = workloads.TRAIN
+    shp = (tr.batch, tr.q_heads, tr.L, tr.head_dim)
+    q, k, v, ke, ve, go = (rnd(*shp) for _ in range(6))
+    _, lse_e = attn.encoder_blockcausal(q, k, v, tr.S)
+    _, lse_d = attn.decoder_train(q, ke, ve, k, v, tr.S)
+    ws_b = torch.empty(tr.batch * tr.q_heads * tr.L, device=dev)
+    bev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    enc_ms = dec_ms = 0.0
+    reps = 5
+    for it in range(2 + reps):
+        bev[0].record()
+        attn.encoder_backward(q, k, v, lse_e, go, tr.S, workspace=ws_b)
+        bev[1].record()
+        attn.decoder_train_backward(q, ke, ve, k, v, lse_d, go, tr.S, workspace=ws_b)
+        bev[2].record()
+        torch.cuda.synchronize()
+        if it >= 2:
+            enc_ms += bev[0].elapsed_time(bev[1]) / reps
+            dec_ms += bev[1].elapsed_time(bev[2]) / reps
+    # five products of 2 d FLOPs per unmasked pair (recomputed Q K^T, dP, dV, dQ, dK): 2.5x forward
+    fl_b = 2.5 * workloads.useful_flops_train(tr)
+    res["train_pass_backward"] = {
+        "workload": tr.name + " backward", "kernels": "CUDA cores (dq pass, then dk/dv pass), fp32",
+        "encoder_ms": enc_ms, "decoder_ms": dec_ms,
+        "useful_tflops": 2 * fl_b / ((enc_ms + dec_ms) * 1e-3) / 1e12,
+        "frac_tensor": 2 * fl_b / ((enc_ms + dec_ms) * 1e-3) / 1e12 / tc}
+    del q, k, v, ke, ve, go, ws_b
     # ---- long-context sample loop
     w = workloads.SAMPLE_LOOP
     B, Hq, Hkv, Sb, d, layers = w["batch"], w["q_heads"], w["kv_heads"], w["S"], w["head_dim"], w["layers"]
