@@ -68,11 +68,15 @@ class Oracle:
         lib.oracle_decoder_train.argtypes = [_f32p] * 5 + [ii] * 6 + [ctypes.c_double, _f64p, _f64p]
         lib.oracle_decoder_sample.argtypes = [_f32p, _f32p, _f32p, ii, ii, _f32p, _f32p,
                                               ii, ii, ii, ii, ii, ctypes.c_double, _f64p, _f64p]
+        lib.oracle_decoder_sample_ragged.argtypes = [_f32p, _f32p, _f32p, ii, ctypes.POINTER(ctypes.c_int),
+                                                     _f32p, _f32p, ii, ii, ii, ii, ii, ctypes.c_double,
+                                                     _f64p, _f64p]
         lib.oracle_kv_append.argtypes = [_u16p, _u16p, ii, ii, _u16p, _u16p, ii, ii, ii, ii]
         lib.oracle_encoder_backward.argtypes = [_f32p] * 4 + [ii] * 6 + [ctypes.c_double] + [_f64p] * 3
         lib.oracle_decoder_train_backward.argtypes = [_f32p] * 6 + [ii] * 6 + [ctypes.c_double] + [_f64p] * 5
         for name in ("oracle_encoder", "oracle_decoder_train", "oracle_decoder_sample",
-                     "oracle_kv_append", "oracle_encoder_backward", "oracle_decoder_train_backward"):
+                     "oracle_kv_append", "oracle_encoder_backward", "oracle_decoder_train_backward",
+                     "oracle_decoder_sample_ragged"):
             getattr(lib, name).restype = ctypes.c_int
         self.lib = lib
 
@@ -182,6 +186,25 @@ class Oracle:
                                             lse.ctypes.data_as(_f64p))
         if rc:
             raise RuntimeError(f"oracle_decoder_sample failed ({rc})")
+        return out, lse
+
+    def decoder_sample_ragged(self, q, k_cache, v_cache, P, k_blk, v_blk, scale: float = 0.0):
+        """Sampling step with a prefix length per batch entry: P is a sequence of B ints."""
+        B, Hq, S, d = q.shape
+        Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+        assert k_cache.shape == (B, Hkv, cap, d) and v_cache.shape == k_cache.shape
+        assert k_blk.shape == (B, Hkv, S, d) and v_blk.shape == k_blk.shape
+        Pa = np.ascontiguousarray(np.asarray(P, dtype=np.int32))
+        assert Pa.shape == (B,)
+        arrs = [self._f32(t) for t in (q, k_cache, v_cache, k_blk, v_blk)]
+        out = np.zeros((B, Hq, S, d), dtype=np.float64)
+        lse = np.zeros((B, Hq, S), dtype=np.float64)
+        rc = self.lib.oracle_decoder_sample_ragged(arrs[0][1], arrs[1][1], arrs[2][1], cap,
+                                                   Pa.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                                   arrs[3][1], arrs[4][1], B, Hq, Hkv, S, d, float(scale),
+                                                   out.ctypes.data_as(_f64p), lse.ctypes.data_as(_f64p))
+        if rc:
+            raise RuntimeError(f"oracle_decoder_sample_ragged failed ({rc})")
         return out, lse
 
     def kv_append(self, k_cache_bits, v_cache_bits, P: int, k_new_bits, v_new_bits):

@@ -235,6 +235,48 @@ int oracle_decoder_sample(const float* q, const float* k_cache, const float* v_c
     return rc ? -1 : 0;
 }
 
+/* Sampling step over a batch whose sequences have decoded different numbers of clean tokens
+ * (ragged prefixes): the plainest extension of [E2D2 notes, sec. 3] to such a batch -- batch
+ * entry b's S noised queries see the first P[b] rows of its own cache and its own block, exactly
+ * the single-prefix step with P = P[b].  Each P[b] lies in [0, capacity].  Layouts as for
+ * oracle_decoder_sample. */
+int oracle_decoder_sample_ragged(const float* q, const float* k_cache, const float* v_cache, int capacity,
+                                 const int* P, const float* k_blk, const float* v_blk, int B, int Hq,
+                                 int Hkv, int S, int d, double scale, double* out, double* lse) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || S <= 0 || d <= 0 || capacity < 0 || (B > 0 && !P))
+        return -3;
+    for (int b = 0; b < B; ++b)
+        if (P[b] < 0 || P[b] > capacity) return -3;
+    const int G = Hq / Hkv;
+    scale = resolve_scale(scale, d);
+    int rc = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : rc)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            const int Pb = P[b];
+            const int nk = Pb + S;
+            uint8_t* mask = (uint8_t*)malloc((size_t)S * nk + 1);
+            double* kd = (double*)malloc(sizeof(double) * ((size_t)nk * d + 1));
+            double* vd = (double*)malloc(sizeof(double) * ((size_t)nk * d + 1));
+            if (!mask || !kd || !vd) { rc |= 2; free(mask); free(kd); free(vd); continue; }
+            oracle_mask_sample(S, Pb, mask);
+            const size_t co = ((size_t)b * Hkv + g) * (size_t)capacity * d;
+            const size_t bo = ((size_t)b * Hkv + g) * (size_t)S * d;
+            rows_to_double(k_cache + co, Pb, d, kd);
+            rows_to_double(k_blk + bo, S, d, kd + (size_t)Pb * d);
+            rows_to_double(v_cache + co, Pb, d, vd);
+            rows_to_double(v_blk + bo, S, d, vd + (size_t)Pb * d);
+            const size_t qo = ((size_t)b * Hq + h) * S;
+            if (attend(q + qo * d, kd, vd, mask, S, nk, d, scale, out + qo * d, lse + qo)) rc |= 1;
+            free(mask);
+            free(kd);
+            free(vd);
+        }
+    }
+    return rc ? -1 : 0;
+}
+
 /* KV-cache append ([E2D2 notes, sec. 3]: once a block is decoded the encoder absorbs it and
  * the cache grows by that block): rows P..P+S_new-1 of every (b, kv head) cache become the
  * new rows.  Caches are [B][Hkv][capacity][d]; new rows [B][Hkv][S_new][d].  Values are

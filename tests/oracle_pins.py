@@ -443,8 +443,44 @@ def pin_backward_finite_differences(orc):
     np.testing.assert_allclose(dv.sum(axis=2), dout.astype(np.float64).sum(axis=2), rtol=0, atol=1e-12)
 
 
+# ---------------------------------------------------------------------------------------
+# Ragged prefixes: a batch whose entries have decoded different numbers of clean tokens.  The
+# plainest reading of the sampling step of [E2D2 notes, sec. 3] for such a batch: entry b sees
+# the first P[b] rows of its own cache and its own block.  Pinned against torch's attention
+# routine with an explicit per-entry mask over [whole cache ; block], the cache rows at or past
+# each entry's prefix filled with large values that must not matter, and entry by entry against
+# the single-prefix step (itself pinned above).
+# ---------------------------------------------------------------------------------------
+def pin_ragged_prefix_against_torch(orc):
+    B, Hq, Hkv, S, cap, d = 5, 4, 2, 5, 23, 8
+    G = Hq // Hkv
+    P = [0, 7, 23, 12, 5]   # empty prefix, unaligned, full capacity, unaligned, one block
+    q = _rand((B, Hq, S, d), 1100)
+    kc, vc = _rand((B, Hkv, cap, d), 1101), _rand((B, Hkv, cap, d), 1102)
+    kb, vb = _rand((B, Hkv, S, d), 1103), _rand((B, Hkv, S, d), 1104)
+    for b, pb in enumerate(P):
+        kc[b, :, pb:] = 8192.0
+        vc[b, :, pb:] = -8192.0
+    scale = 0.4
+    out, lse = orc.decoder_sample_ragged(q, kc, vc, P, kb, vb, scale=scale)
+    keys = np.repeat(np.concatenate([kc, kb], axis=2), G, axis=1)
+    vals = np.repeat(np.concatenate([vc, vb], axis=2), G, axis=1)
+    mask = np.zeros((B, 1, S, cap + S), dtype=bool)
+    for b, pb in enumerate(P):
+        mask[b, :, :, :pb] = True
+        mask[b, :, :, cap:] = True
+    np.testing.assert_allclose(out, _sdpa(q, keys, vals, scale, mask=mask), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, _torch_lse(q, keys, scale, mask), rtol=0, atol=1e-12)
+    for b, pb in enumerate(P):
+        sl = slice(b, b + 1)
+        o, l = orc.decoder_sample(q[sl], kc[sl], vc[sl], pb, kb[sl], vb[sl], scale=scale)
+        np.testing.assert_allclose(out[sl], o, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[sl], l, rtol=0, atol=1e-13)
+
+
 ALL_PINS = [pin_pair_count, pin_golden_pairs, pin_block_size_one_is_causal,
             pin_block_size_L_is_bidirectional, pin_masked_against_torch, pin_brute_force,
             pin_zero_keys_closed_form, pin_constant_values, pin_gqa_is_repeated_heads,
             pin_sample_is_train_slice, pin_append_is_concatenation, pin_short_last_block,
-            pin_bd3lm_vectorized_mask, pin_backward_against_autograd, pin_backward_finite_differences]
+            pin_bd3lm_vectorized_mask, pin_backward_against_autograd, pin_backward_finite_differences,
+            pin_ragged_prefix_against_torch]

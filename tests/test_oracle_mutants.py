@@ -55,6 +55,10 @@ MUTANTS = [
      "dv[(size_t)j * d + c] += (double)gi[c];"),
     ("bwd-dec-swaps-sources", "memcpy(dk_enc + ko, dkd, sizeof(double) * (size_t)L * d);",
      "memcpy(dk_enc + ko, dkd + (size_t)L * d, sizeof(double) * (size_t)L * d);"),
+    # ragged prefixes
+    ("ragged-first-entry-prefix", "const int Pb = P[b];", "const int Pb = P[0];"),
+    ("ragged-block-read-from-cache", "rows_to_double(k_blk + bo, S, d, kd + (size_t)Pb * d);",
+     "rows_to_double(k_cache + co + (size_t)Pb * d, S, d, kd + (size_t)Pb * d);"),
 ]
 
 _RUNNER = r"""
