@@ -710,7 +710,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workload-set", action="store_true",
-                    help="skip timing the translation train chain and the long sample loop")
+                    help="skip timing the translation train chain, the long sample loop and the backward")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-step-budget", type=float, default=8.0, help="max seconds of oracle work per reference step")
     ap.add_argument("--ref-total-budget", type=float, default=150.0, help="seconds of oracle work for the whole reference run")
