@@ -110,8 +110,9 @@ E2D2_API e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_en
  *   forward call; lse (NOT NULL) is that call's lse; dout [batch][q_heads][L][d] bf16.
  *   dq [batch][q_heads][L][d]; dk, dv (dk_enc, dv_enc, dk_dec, dv_dec) [batch][kv_heads][L][d],
  *   bf16, every element written (no accumulation into them).
- *   workspace: device memory of at least e2d2_attn_train_backward_workspace(dims, L) bytes,
- *   16-byte aligned, contents ignored (holds D_i between the two launches of the call).
+ *   workspace: device memory of at least e2d2_attn_train_backward_workspace(dims, L) bytes
+ *   (batch * q_heads * L floats; the query returns 0 for invalid dims or L <= 0 and needs no
+ *   GPU), 16-byte aligned, contents ignored (holds D_i between the two launches of the call).
  *   Launches two kernels on `stream`: dq with D_i, then dk/dv.  Errors as for the forward
  *   calls; a NULL lse is E2D2_ERR_INVALID_ARG; a small workspace is E2D2_ERR_WORKSPACE.
  */
