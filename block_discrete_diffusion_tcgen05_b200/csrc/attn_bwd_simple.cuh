@@ -1,7 +1,8 @@
 // attn_bwd_simple.cuh -- backward of the E2D2 train calls (encoder block-causal self-attention
 // and the decoder's fused self+cross attention over 2L keys; "Encoder-Decoder Diffusion Language
-// Models for Efficient Training and Inference", paper notes, sec. 4: the training algorithm runs
-// one encoder and one decoder pass over all blocks, forward and backward).
+// Models for Efficient Training and Inference", paper notes, sec. 4: one encoder and one decoder
+// pass with custom masks train all blocks; the page gives no backward, so this is the plain
+// derivative of those two attention calls that a gradient step through them needs).
 //
 // First, plain version on the CUDA cores (fp32 arithmetic, bf16 in and out), recomputing the
 // probabilities from the forward's LSE:

@@ -97,8 +97,9 @@ E2D2_API e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_en
                                     e2d2_dims dims, int L, int S, cudaStream_t stream);
 
 /*
- * Backward of the two train calls ([E2D2 notes, sec. 4]: the training algorithm runs one
- * encoder and one decoder pass over all blocks, forward and backward).  Gradients of
+ * Backward of the two train calls ([E2D2 notes, sec. 4]: one encoder and one decoder pass with
+ * custom masks train all blocks; the page gives no backward, so these are the plain derivatives
+ * of the two calls that a gradient step through them needs).  Gradients of
  * sum(dout * out) with respect to every input, the probabilities recomputed from the forward's
  * lse:  p_ij = exp(scale q_i.k_j - lse_i) over the keys the forward's mask lets row i see,
  * dp_ij = dout_i.v_j,  D_i = sum_j p_ij dp_ij (dout_i.out_i in exact arithmetic, formed here

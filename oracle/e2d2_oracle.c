@@ -296,8 +296,9 @@ int oracle_kv_append(uint16_t* k_cache, uint16_t* v_cache, int capacity, int P,
 }
 
 /* ---------------------------------------------------------------------------------------
- * Backward of the train calls ([E2D2 notes, sec. 4]: the training algorithm takes one
- * encoder pass and one decoder pass over all blocks, forward and backward).  From the chain
+ * Backward of the train calls ([E2D2 notes, sec. 4]: one encoder pass and one decoder pass
+ * with custom masks train all blocks; the page gives no backward, so this is the plain
+ * derivative of those passes that a gradient step needs).  From the chain
  * rule applied to the definition at the top of this file, with p_ij = exp(s_ij - lse_i) over
  * the allowed keys of row i and dout the gradient of the loss with respect to out:
  *   dv_j   += sum_i p_ij dout_i
