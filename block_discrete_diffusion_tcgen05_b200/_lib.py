@@ -19,7 +19,7 @@ EXPORTS = ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
            "e2d2_kv_cache_append", "e2d2_status_string", "e2d2_last_device_error", "e2d2_version",
            "e2d2_attn_decoder_sample_noalloc", "e2d2_attn_encoder_block_step",
            "e2d2_attn_train_backward_workspace", "e2d2_attn_encoder_backward",
-           "e2d2_attn_decoder_train_backward")
+           "e2d2_attn_decoder_train_backward", "e2d2_attn_decoder_sample_plan")
 
 # E2D2_SAMPLE_NOALLOC_MAX_BYTES of include/e2d2_attn.h
 SAMPLE_NOALLOC_MAX_BYTES = 32 << 20
@@ -30,6 +30,14 @@ class Dims(ctypes.Structure):
 
     _fields_ = [("batch", ctypes.c_int), ("q_heads", ctypes.c_int), ("kv_heads", ctypes.c_int),
                 ("head_dim", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class SamplePlan(ctypes.Structure):
+    """e2d2_sample_plan."""
+
+    _fields_ = [("kernel", ctypes.c_int), ("units", ctypes.c_int), ("tiles_per_unit", ctypes.c_int),
+                ("split_units", ctypes.c_int), ("split_ctas", ctypes.c_int), ("whole_units", ctypes.c_int),
+                ("grid", ctypes.c_int)]
 
 
 class E2D2Error(RuntimeError):
@@ -70,6 +78,8 @@ def load(path: Path | str | None = None):
                                                ctypes.c_size_t, st]
     lib.e2d2_attn_decoder_train_backward.argtypes = [vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, vp, vp,
                                                      Dims, ci, ci, vp, ctypes.c_size_t, st]
+    lib.e2d2_attn_decoder_sample_plan.argtypes = [Dims, ci, ci, ci, ctypes.POINTER(SamplePlan)]
+    lib.e2d2_attn_decoder_sample_plan.restype = ctypes.c_int
     lib.e2d2_status_string.argtypes = [ci]
     lib.e2d2_status_string.restype = ctypes.c_char_p
     lib.e2d2_last_device_error.argtypes = [st]

@@ -5,6 +5,7 @@ Argument marshalling only: every step of the attention runs in the CUDA kernels 
 the tensors' device).  Names follow the C ABI (include/e2d2_attn.h)."""
 from __future__ import annotations
 
+import ctypes
 import math
 
 import torch
@@ -138,6 +139,16 @@ def sample_workspace_bytes(batch, q_heads, kv_heads, head_dim, S, capacity) -> i
     lib = _lib.load()
     return int(lib.e2d2_attn_decoder_sample_workspace(_dims(batch, q_heads, kv_heads, head_dim, None),
                                                       S, capacity))
+
+
+def sample_plan(batch, q_heads, kv_heads, head_dim, S, P, num_sms) -> dict:
+    """Work plan of a sampling call on a GPU with num_sms SMs (no GPU needed)."""
+    lib = _lib.load()
+    plan = _lib.SamplePlan()
+    st = lib.e2d2_attn_decoder_sample_plan(_dims(batch, q_heads, kv_heads, head_dim, None), S, P, num_sms,
+                                           ctypes.byref(plan))
+    _lib.check(st, "e2d2_attn_decoder_sample_plan")
+    return {name: getattr(plan, name) for name, _ in _lib.SamplePlan._fields_}
 
 
 def sample_workspace(q_blk: torch.Tensor, k_cache: torch.Tensor) -> torch.Tensor:

@@ -283,6 +283,56 @@ SampleLayout sample_layout(const e2d2_dims& dm, int S) {
     return w;
 }
 
+// Work plan of a sampling call: which kernel, how many units and key tiles, and the two-phase
+// split.  With U units on G CTAs, floor(U/G)*G units run whole (one CTA each, last); the other R
+// units are split stream-K over at most 5R CTAs (a unit has at most about six partials to merge),
+// and only as far as every piece keeps about kMinSplitTiles key tiles: publishing and merging a
+// partial costs several microseconds, more than streaming a few tiles.  A split never uses fewer
+// CTAs than there are units, so a CTA's tile range meets at most two units (two partial slots).
+struct SamplePlan {
+    int keyrow_n;        // 0: generic kernel; 16/32/64: keys-on-lanes kernel with N query columns
+    int num_qtiles;      // query tiles per (batch, kv head)
+    int tiles_per_unit;  // 128-key tiles per unit: prefix tiles + own-block tiles
+    int split_units;     // R
+    int whole_units;     // U - R
+    int split_ctas;      // CTAs of the split phase
+    long long total_tiles;  // key tiles of the split phase (R * tiles_per_unit)
+    long long grid;      // CTAs launched
+};
+
+SamplePlan plan_sample(const e2d2_dims& dims, int S, int P, int sms) {
+    SamplePlan pl;
+    const int D = dims.head_dim;
+    const int G = dims.q_heads / dims.kv_heads;
+    const long long BHkv = static_cast<long long>(dims.batch) * dims.kv_heads;
+    // Short packed tiles at d = 128 take the kernel with keys on the TMEM lanes (S^T = K Q^T):
+    // its tensor-core rows are keys, so none is padding.  N = packed columns rounded up.
+    const int GS = G * S;
+    pl.keyrow_n = (D != 128 || GS > 64) ? 0 : (GS <= 16 ? 16 : (GS <= 32 ? 32 : 64));
+    pl.num_qtiles = pl.keyrow_n ? 1 : (G * S + kBlockM - 1) / kBlockM;
+    pl.tiles_per_unit = (S + kBlockN - 1) / kBlockN + (P + kBlockN - 1) / kBlockN;
+    const long long Tu = pl.tiles_per_unit;
+    const long long U = BHkv * pl.num_qtiles;
+    long long grid = sms < kSampleMaxCtas ? sms : kSampleMaxCtas;
+    if (grid > U * Tu) grid = U * Tu;
+    const long long R = U >= grid ? U % grid : U;
+    pl.split_units = static_cast<int>(R);
+    pl.whole_units = static_cast<int>(U - R);
+    constexpr long long kMinSplitTiles = 6;
+    long long sc = R * 5 < grid ? R * 5 : grid;
+    if (sc > R * Tu / kMinSplitTiles) sc = R * Tu / kMinSplitTiles;
+    if (sc < R) sc = R;
+    if (sc > R * Tu) sc = R * Tu;
+    pl.split_ctas = static_cast<int>(sc);
+    pl.total_tiles = R * Tu;
+    // Whole units exist only when U >= grid, and then every CTA takes some; otherwise only the
+    // CTAs of the split phase have work.
+    if (pl.whole_units == 0) grid = pl.split_ctas;
+    pl.grid = grid;
+    return pl;
+}
+// (end of plan_sample)
+
 // The sampling call; `append` (encoder block step) also writes the block's K/V to cache rows
 // P..P+S-1 from inside the same launch.
 e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, const void* v_cache, int capacity,
@@ -318,10 +368,8 @@ e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, con
     // warps then issue full-width TMEM loads and instruction streams for a quarter of the rows
     // each), so rows stay contiguous.
     const int q_chunk = kBlockM / 4;
-    // Short packed tiles at d = 128 take the kernel with keys on the TMEM lanes (S^T = K Q^T):
-    // its tensor-core rows are keys, so none is padding.  N = packed columns rounded up.
-    const int GS = G * S;
-    const int keyrow_n = (D != 128 || GS > 64) ? 0 : (GS <= 16 ? 16 : (GS <= 32 ? 32 : 64));
+    const SamplePlan plan = plan_sample(dims, S, P, di->sms);
+    const int keyrow_n = plan.keyrow_n;
     bool ok = map_2d(&prm.tm_q, q_blk, D, rows, keyrow_n ? keyrow_n : q_chunk) &&
               map_3d(&prm.tm_k0, k_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
               map_3d(&prm.tm_v0, v_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
@@ -342,8 +390,8 @@ e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, con
     prm.box1_rows = box1;
     prm.scale_log2 = scale_log2(dims);
     prm.rows_per_unit = G * S;
-    prm.num_qtiles = keyrow_n ? 1 : (G * S + kBlockM - 1) / kBlockM;
-    prm.tiles_per_unit = (S + kBlockN - 1) / kBlockN + (P + kBlockN - 1) / kBlockN;
+    prm.num_qtiles = plan.num_qtiles;
+    prm.tiles_per_unit = plan.tiles_per_unit;
     prm.rows_cap = w.rows_cap;
     prm.q_chunk = q_chunk;
     prm.slot_floats = w.slot_floats;
@@ -354,28 +402,11 @@ e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, con
         prm.app_dst_v = static_cast<uint4*>(const_cast<void*>(v_cache));
         prm.app_capacity = capacity;
     }
-    // Schedule: with U units on G CTAs, floor(U/G)*G units run whole (one CTA each, last); the
-    // other R units are split stream-K over at most 5R CTAs (a unit has at most about six partials
-    // to merge), and only as far as every piece keeps about kMinSplitTiles key tiles: publishing and
-    // merging a partial costs several microseconds, more than streaming a few tiles.  A split never
-    // uses fewer CTAs than there are units.
-    const long long Tu = prm.tiles_per_unit;
-    const long long U = BHkv * prm.num_qtiles;
-    long long grid = di->sms < kSampleMaxCtas ? di->sms : kSampleMaxCtas;
-    if (grid > U * Tu) grid = U * Tu;
-    const long long R = U >= grid ? U % grid : U;
-    prm.split_units = static_cast<int>(R);
-    prm.whole_units = static_cast<int>(U - R);
-    constexpr long long kMinSplitTiles = 6;
-    long long sc = R * 5 < grid ? R * 5 : grid;
-    if (sc > R * Tu / kMinSplitTiles) sc = R * Tu / kMinSplitTiles;
-    if (sc < R) sc = R;
-    if (sc > R * Tu) sc = R * Tu;
-    prm.split_ctas = static_cast<int>(sc);
-    prm.total_tiles = R * Tu;
-    // Whole units exist only when U >= grid, and then every CTA takes some; otherwise only the
-    // CTAs of the split phase have work.
-    if (prm.whole_units == 0) grid = prm.split_ctas;
+    prm.split_units = plan.split_units;
+    prm.whole_units = plan.whole_units;
+    prm.split_ctas = plan.split_ctas;
+    prm.total_tiles = plan.total_tiles;
+    const long long grid = plan.grid;
     switch (keyrow_n) {
         case 16: return launch_keyrow<16>(prm, static_cast<int>(grid), stream);
         case 32: return launch_keyrow<32>(prm, static_cast<int>(grid), stream);
@@ -472,6 +503,22 @@ e2d2_status e2d2_attn_decoder_train_backward(const void* q_dec, const void* k_en
 size_t e2d2_attn_decoder_sample_workspace(e2d2_dims dims, int S, int capacity) {
     if (check_dims(dims) != E2D2_OK || S <= 0 || capacity < 0) return 0;
     return sample_layout(dims, S).bytes;
+}
+
+e2d2_status e2d2_attn_decoder_sample_plan(e2d2_dims dims, int S, int P, int num_sms, e2d2_sample_plan* plan) {
+    if (!plan) return E2D2_ERR_INVALID_ARG;
+    e2d2_status s = check_dims(dims);
+    if (s != E2D2_OK) return s;
+    if (S <= 0 || P < 0 || num_sms <= 0) return E2D2_ERR_INVALID_ARG;
+    const SamplePlan pl = plan_sample(dims, S, P, num_sms);
+    plan->kernel = pl.keyrow_n;
+    plan->units = static_cast<int>(static_cast<long long>(dims.batch) * dims.kv_heads * pl.num_qtiles);
+    plan->tiles_per_unit = pl.tiles_per_unit;
+    plan->split_units = pl.split_units;
+    plan->split_ctas = pl.split_ctas;
+    plan->whole_units = pl.whole_units;
+    plan->grid = static_cast<int>(pl.grid);
+    return E2D2_OK;
 }
 
 e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_cache, const void* v_cache,

@@ -155,6 +155,32 @@ E2D2_API e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_c
                                      size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Work plan of a sampling call (e2d2_attn_decoder_sample, _noalloc and
+ * e2d2_attn_encoder_block_step) for these dims, block size S and prefix length P on a GPU with
+ * num_sms SMs (the calls use the current device's count).  Needs no GPU; launches nothing.  The
+ * calls cut the work into units of (batch entry, kv head, query tile), each a stream of
+ * tiles_per_unit tiles of 128 keys (ceil(P/128) prefix tiles + ceil(S/128) own-block tiles).
+ * With U units and G = min(num_sms, 256) CTAs, floor(U/G)*G units are taken whole, one CTA each,
+ * after the split phase; the other split_units units are cut into equal contiguous tile ranges
+ * over split_ctas CTAs, whose fp32 partials the last CTA to finish a unit merges in CTA order.
+ *   kernel: 0 = the generic kernel, 16/32/64 = the kernel with keys on the tensor-memory lanes
+ *   and that many packed query columns (head_dim 128 and G*S <= 64).
+ * Returns E2D2_ERR_INVALID_ARG for a NULL plan, bad dims, S <= 0, P < 0 or num_sms <= 0.
+ */
+typedef struct {
+    int kernel;         /* 0 generic; 16, 32, 64: keys-on-lanes kernel with N query columns */
+    int units;          /* work units: batch * kv_heads * query tiles per kv head            */
+    int tiles_per_unit; /* 128-key tiles per unit                                             */
+    int split_units;    /* units cut over the split phase's CTAs                              */
+    int split_ctas;     /* CTAs of the split phase                                            */
+    int whole_units;    /* units taken whole, one CTA each                                    */
+    int grid;           /* CTAs launched                                                      */
+} e2d2_sample_plan;
+
+E2D2_API e2d2_status e2d2_attn_decoder_sample_plan(e2d2_dims dims, int S, int P, int num_sms,
+                                                   e2d2_sample_plan* plan);
+
+/*
  * Sampling step that allocates nothing: same arguments and result as e2d2_attn_decoder_sample
  * minus the workspace.  The paper has no counterpart; this exists for callers that cannot
  * allocate device memory (an engine that gives all of HBM to its own pool and no allocator to
