@@ -6,6 +6,7 @@ the tensors' device).  Names follow the C ABI (include/e2d2_attn.h)."""
 from __future__ import annotations
 
 import ctypes
+import functools
 import math
 
 import torch
@@ -32,6 +33,59 @@ def _need(t: torch.Tensor, name: str, dtype=_BF16, ndim=4):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _device_guard(fn):
+    """Runs a call with the GPU of its first tensor current (the C calls read the current device:
+    SM count, error word) and rejects tensors spread over several devices."""
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        first = args[0] if args else None
+        if isinstance(first, torch.Tensor) and first.is_cuda:
+            idx = first.get_device()
+            for a in (*args, *kwargs.values()):
+                if isinstance(a, torch.Tensor) and a.get_device() != idx:
+                    raise ValueError(f"{fn.__name__}: every tensor must be on cuda:{idx}")
+            if idx != torch.cuda.current_device():
+                with torch.cuda.device(idx):
+                    return fn(*args, **kwargs)
+        return fn(*args, **kwargs)
+
+    return wrapper
+
+
+def _out_tensor(out, like: torch.Tensor) -> torch.Tensor:
+    """The output buffer: a new one like `like`, or the caller's, checked (the kernels write
+    every element of it through a plain pointer)."""
+    if out is None:
+        return torch.empty_like(like)
+    _need(out, "out")
+    if out.shape != like.shape:
+        raise ValueError(f"out must have shape {tuple(like.shape)}, got {tuple(out.shape)}")
+    return out
+
+
+def _lse_tensor(lse, shape, device):
+    """lse=True: a new fp32 tensor; None/False: not computed; a tensor: the caller's, checked."""
+    if lse is True:
+        return torch.empty(shape, dtype=torch.float32, device=device)
+    if lse is None or lse is False:
+        return None
+    _need(lse, "lse", dtype=torch.float32, ndim=3)
+    if tuple(lse.shape) != tuple(shape):
+        raise ValueError(f"lse must have shape {tuple(shape)}, got {tuple(lse.shape)}")
+    return lse
+
+
+def _need_workspace(ws: torch.Tensor) -> torch.Tensor:
+    if not isinstance(ws, torch.Tensor) or not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ws
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
 def _stream(t: torch.Tensor):
     return ctypes_stream(torch.cuda.current_stream(t.device))
 
@@ -40,6 +94,7 @@ def ctypes_stream(s: torch.cuda.Stream):
     return s.cuda_stream
 
 
+@_device_guard
 def encoder_blockcausal(q, k, v, S: int, scale=None, out=None, lse=True):
     """Block-causal encoder self-attention.  q [B,Hq,L,d], k/v [B,Hkv,L,d] (bf16, CUDA).
     Returns (out [B,Hq,L,d] bf16, lse [B,Hq,L] fp32 or None)."""
@@ -50,15 +105,15 @@ def encoder_blockcausal(q, k, v, S: int, scale=None, out=None, lse=True):
     Hkv = k.shape[1]
     if k.shape != (B, Hkv, L, d) or v.shape != k.shape:
         raise ValueError("k/v must be [B, Hkv, L, d] matching q")
-    out = torch.empty_like(q) if out is None else out
-    lse_t = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device) if lse is True else lse
-    st = lib.e2d2_attn_encoder_blockcausal(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                           None if lse_t is None or lse_t is False else lse_t.data_ptr(),
+    out = _out_tensor(out, q)
+    lse_t = _lse_tensor(lse, (B, Hq, L), q.device)
+    st = lib.e2d2_attn_encoder_blockcausal(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse_t),
                                            _dims(B, Hq, Hkv, d, scale), L, S, _stream(q))
     _lib.check(st, "e2d2_attn_encoder_blockcausal")
-    return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
+    return out, lse_t
 
 
+@_device_guard
 def decoder_train(q, k_enc, v_enc, k_dec, v_dec, S: int, scale=None, out=None, lse=True):
     """Decoder fused self+cross attention (training mode) over 2L keys."""
     lib = _lib.load()
@@ -69,23 +124,23 @@ def decoder_train(q, k_enc, v_enc, k_dec, v_dec, S: int, scale=None, out=None, l
     for t in (k_enc, v_enc, k_dec, v_dec):
         if t.shape != (B, Hkv, L, d):
             raise ValueError("k_enc/v_enc/k_dec/v_dec must be [B, Hkv, L, d] matching q")
-    out = torch.empty_like(q) if out is None else out
-    lse_t = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device) if lse is True else lse
+    out = _out_tensor(out, q)
+    lse_t = _lse_tensor(lse, (B, Hq, L), q.device)
     st = lib.e2d2_attn_decoder_train(q.data_ptr(), k_enc.data_ptr(), v_enc.data_ptr(), k_dec.data_ptr(),
-                                     v_dec.data_ptr(), out.data_ptr(),
-                                     None if lse_t is None or lse_t is False else lse_t.data_ptr(),
+                                     v_dec.data_ptr(), out.data_ptr(), _ptr(lse_t),
                                      _dims(B, Hq, Hkv, d, scale), L, S, _stream(q))
     _lib.check(st, "e2d2_attn_decoder_train")
-    return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
+    return out, lse_t
 
 
 def _train_backward_ws(lib, B, Hq, Hkv, d, L, scale, device, workspace):
     need = lib.e2d2_attn_train_backward_workspace(_dims(B, Hq, Hkv, d, scale), L)
     if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
-    return workspace
+        return torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    return _need_workspace(workspace)
 
 
+@_device_guard
 def encoder_backward(q, k, v, lse, dout, S: int, scale=None, workspace=None):
     """Gradients of the encoder call: (dq [B,Hq,L,d], dk, dv [B,Hkv,L,d]) bf16, from the forward's
     lse (fp32) and the output gradient dout."""
@@ -109,6 +164,7 @@ def encoder_backward(q, k, v, lse, dout, S: int, scale=None, workspace=None):
     return dq, dk, dv
 
 
+@_device_guard
 def decoder_train_backward(q, k_enc, v_enc, k_dec, v_dec, lse, dout, S: int, scale=None, workspace=None):
     """Gradients of the decoder train call: (dq, dk_enc, dv_enc, dk_dec, dv_dec) bf16."""
     lib = _lib.load()
@@ -151,6 +207,7 @@ def sample_plan(batch, q_heads, kv_heads, head_dim, S, P, num_sms) -> dict:
     return {name: getattr(plan, name) for name, _ in _lib.SamplePlan._fields_}
 
 
+@_device_guard
 def sample_workspace(q_blk: torch.Tensor, k_cache: torch.Tensor) -> torch.Tensor:
     """A zero-filled workspace for decoder_sample with these shapes."""
     B, Hq, S, d = q_blk.shape
@@ -159,6 +216,7 @@ def sample_workspace(q_blk: torch.Tensor, k_cache: torch.Tensor) -> torch.Tensor
     return torch.zeros(n, dtype=torch.uint8, device=q_blk.device)
 
 
+@_device_guard
 def decoder_sample(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=None, scale=None,
                    out=None, lse=True):
     """Decoder sampling step over the cached prefix k_cache[:, :, :P] plus the own block."""
@@ -172,18 +230,19 @@ def decoder_sample(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=None
         raise ValueError("caches must be [B, Hkv, capacity, d]")
     if k_blk.shape != (B, Hkv, S, d) or v_blk.shape != k_blk.shape:
         raise ValueError("k_blk/v_blk must be [B, Hkv, S, d]")
-    ws = sample_workspace(q_blk, k_cache) if workspace is None else workspace
-    out = torch.empty_like(q_blk) if out is None else out
-    lse_t = torch.empty((B, Hq, S), dtype=torch.float32, device=q_blk.device) if lse is True else lse
+    ws = sample_workspace(q_blk, k_cache) if workspace is None else _need_workspace(workspace)
+    out = _out_tensor(out, q_blk)
+    lse_t = _lse_tensor(lse, (B, Hq, S), q_blk.device)
     st = lib.e2d2_attn_decoder_sample(q_blk.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cap, int(P),
                                       k_blk.data_ptr(), v_blk.data_ptr(), out.data_ptr(),
-                                      None if lse_t is None or lse_t is False else lse_t.data_ptr(),
+                                      _ptr(lse_t),
                                       _dims(B, Hq, Hkv, d, scale), S, ws.data_ptr(),
                                       ws.numel() * ws.element_size(), _stream(q_blk))
     _lib.check(st, "e2d2_attn_decoder_sample")
-    return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
+    return out, lse_t
 
 
+@_device_guard
 def encoder_block_step(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=None, scale=None,
                        out=None, lse=True):
     """Encoder incremental block step: the block's S clean queries attend to k_cache[:, :, :P] and
@@ -199,18 +258,19 @@ def encoder_block_step(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=
         raise ValueError("caches must be [B, Hkv, capacity, d]")
     if k_blk.shape != (B, Hkv, S, d) or v_blk.shape != k_blk.shape:
         raise ValueError("k_blk/v_blk must be [B, Hkv, S, d]")
-    ws = sample_workspace(q_blk, k_cache) if workspace is None else workspace
-    out = torch.empty_like(q_blk) if out is None else out
-    lse_t = torch.empty((B, Hq, S), dtype=torch.float32, device=q_blk.device) if lse is True else lse
+    ws = sample_workspace(q_blk, k_cache) if workspace is None else _need_workspace(workspace)
+    out = _out_tensor(out, q_blk)
+    lse_t = _lse_tensor(lse, (B, Hq, S), q_blk.device)
     st = lib.e2d2_attn_encoder_block_step(q_blk.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cap, int(P),
                                           k_blk.data_ptr(), v_blk.data_ptr(), out.data_ptr(),
-                                          None if lse_t is None or lse_t is False else lse_t.data_ptr(),
+                                          _ptr(lse_t),
                                           _dims(B, Hq, Hkv, d, scale), S, ws.data_ptr(),
                                           ws.numel() * ws.element_size(), _stream(q_blk))
     _lib.check(st, "e2d2_attn_encoder_block_step")
-    return out, (lse_t if isinstance(lse_t, torch.Tensor) else None)
+    return out, lse_t
 
 
+@_device_guard
 def kv_cache_append(k_cache, v_cache, P: int, k_new, v_new):
     """Writes k_new/v_new [B,Hkv,S_new,d] into rows P..P+S_new-1 of the caches; returns P+S_new."""
     lib = _lib.load()
