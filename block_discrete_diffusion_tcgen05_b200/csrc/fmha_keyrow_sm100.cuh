@@ -30,9 +30,11 @@
 //
 // CTA = 16 warps: warp 0 loads Q and K, warp 1 owns tensor memory and issues S^T = K Q^T, warp 2
 // loads V, warp 3 issues O^T += V^T P^T, warps 4..11 are the two softmax warpgroups, warps
-// 12..15 the epilogue warpgroup.  The work split over CTAs (stream-K over the key tiles of all
-// units, last arriver merges) and the partial-slot format are those of the generic sampling
-// kernel in fmha_sm100.cuh.
+// 12..15 the epilogue warpgroup (which, in an encoder block step, first copies the block's K/V
+// into the cache for the units whose own-block tile it takes).  The work split over CTAs (units
+// that fill whole rounds of the grid taken whole, last; the rest split stream-K over their key
+// tiles, the last CTA to finish a unit merging the partials in CTA order) and the partial-slot
+// format are those of the generic sampling kernel in fmha_sm100.cuh.
 #pragma once
 
 #include <cstdint>

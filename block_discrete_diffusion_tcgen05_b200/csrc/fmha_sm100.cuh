@@ -16,7 +16,8 @@
 // never loaded, and no mask matrix exists anywhere.
 //
 // CTA = 12 warps: warp 0 issues TMA loads, warp 1 owns tensor memory and issues tcgen05.mma,
-// warps 2..3 idle, warps 4..7 and 8..11 are two softmax warpgroups.  Per key tile of up to 128 keys:
+// warps 2..3 write the block's K/V into the cache in an encoder block step (otherwise idle),
+// warps 4..7 and 8..11 are two softmax warpgroups.  Per key tile of up to 128 keys:
 //     S  = Q K^T          tcgen05.mma, A = Q (smem), B = K (smem, K-major)  -> TMEM (fp32)
 //     P  = exp2(S*c - m)  softmax warpgroup, written back over S as bf16  -> TMEM
 //     O += P V            tcgen05.mma, A = P (TMEM), B = V (smem, MN-major) -> TMEM
@@ -46,7 +47,7 @@ constexpr int kBlockN = 128;            // keys per tile
 constexpr int kThreads = 384;           // 12 warps = 3 warpgroups
 constexpr int kSoftmaxThreads = 256;    // warpgroups 1 and 2 (warps 4..11)
 // Register split (setmaxnreg): the launch gives every thread kRegsLaunch registers; warpgroup 0
-// (TMA producer, MMA issuer, two idle warps) gives most of its share to the softmax groups.
+// (TMA producer, MMA issuer, two mostly idle warps) gives most of its share to the softmax groups.
 constexpr int kRegsLaunch = 168;
 constexpr int kRegsControl = 88;
 constexpr int kRegsSoftmax = 208;
