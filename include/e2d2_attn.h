@@ -113,7 +113,8 @@ E2D2_API e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_en
  *   bf16, every element written (no accumulation into them).
  *   workspace: device memory of at least e2d2_attn_train_backward_workspace(dims, L) bytes
  *   (batch * q_heads * L floats; the query returns 0 for invalid dims or L <= 0 and needs no
- *   GPU), 16-byte aligned, contents ignored (holds D_i between the two launches of the call).
+ *   GPU), 16-byte aligned, contents ignored (holds D_i between the two launches of the call);
+ *   calls that may run at the same time (different streams) need different workspaces.
  *   Launches two kernels on `stream`: dq with D_i, then dk/dv.  Errors as for the forward
  *   calls; a NULL lse is E2D2_ERR_INVALID_ARG; a small workspace is E2D2_ERR_WORKSPACE.
  */
