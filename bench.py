@@ -673,6 +673,11 @@ def cpu_baseline(budget_s: float):
 def run_reference(args, rank, world):
     if rank != 0:
         return
+    if world > 1:
+        # the launcher starts every rank with one OpenMP thread; rank 0 works alone, so it takes
+        # every core it may run on
+        _oracle_inputs()
+        _ORACLE_CACHE["orc"].set_num_threads(len(os.sched_getaffinity(0)))
     t0 = time.perf_counter()
     per_step = []
     # Keep the whole reference run to a few minutes whatever --steps/--warmup are.

@@ -59,6 +59,8 @@ class Oracle:
         self.path = Path(path)
         lib = ctypes.CDLL(str(self.path))
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = None
         for name in ("oracle_mask_encoder", "oracle_mask_decoder"):
             getattr(lib, name).argtypes = [ctypes.c_int, ctypes.c_int, _u8p]
         lib.oracle_mask_sample.argtypes = [ctypes.c_int, ctypes.c_int, _u8p]
@@ -88,6 +90,9 @@ class Oracle:
 
     def num_threads(self) -> int:
         return int(self.lib.oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        self.lib.oracle_set_num_threads(int(n))
 
     # ---- masks -------------------------------------------------------------------
     def mask_encoder(self, L: int, S: int) -> np.ndarray:

@@ -55,6 +55,16 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads of the parallel loops that follow on the calling thread (n >= 1; ignored without
+ * OpenMP).  Lets a caller that was started with OMP_NUM_THREADS=1 use every host core. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Encoder block-causal mask [L][L] ([E2D2 notes, sec. 4]): allowed(i, j) iff the block of
  * key j is the block of query i or an earlier one. */
 void oracle_mask_encoder(int L, int S, uint8_t* mask) {

@@ -56,11 +56,13 @@ def test_reference_arm_prints_on_rank_zero_only():
                     env_extra={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert res.returncode == 0, res.stderr
     assert json_lines(res.stdout) == []
+    # the launcher gives every rank one OpenMP thread; rank 0, working alone, takes every core
     res = run_bench(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", *FAST_REF],
-                    env_extra={"RANK": "0", "WORLD_SIZE": "2", "LOCAL_RANK": "0"})
+                    env_extra={"RANK": "0", "WORLD_SIZE": "2", "LOCAL_RANK": "0", "OMP_NUM_THREADS": "1"})
     assert res.returncode == 0, res.stderr
     lines = json_lines(res.stdout)
     assert len(lines) == 1 and lines[0]["n_gpus"] == 2
+    assert lines[0]["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
 
 
 def test_fewer_than_three_warmup_steps_are_refused():
