@@ -331,7 +331,6 @@ SamplePlan plan_sample(const e2d2_dims& dims, int S, int P, int sms) {
     pl.grid = grid;
     return pl;
 }
-// (end of plan_sample)
 
 // The sampling call; `append` (encoder block step) also writes the block's K/V to cache rows
 // P..P+S-1 from inside the same launch.
