@@ -237,21 +237,22 @@ def run_workload_set(torch, attn, workloads, dev, peaks):
         "frac_tensor": fl / step_s / 1e12 / tc, "frac_attainable": fl / step_s / attainable,
         "launches_per_step": tc_shape.enc_calls + tc_shape.dec_calls}
     del enc_layers, dec_layers
-    # ---- backward of the train pass (first, CUDA-core kernels)
+    # ---- backward of the train pass (tcgen05 kernels: dq with D_i, then dk/dv)
     tr = workloads.TRAIN
     shp = (tr.batch, tr.q_heads, tr.L, tr.head_dim)
     q, k, v, ke, ve, go = (rnd(*shp) for _ in range(6))
-    _, lse_e = attn.encoder_blockcausal(q, k, v, tr.S)
-    _, lse_d = attn.decoder_train(q, ke, ve, k, v, tr.S)
-    ws_b = torch.empty(tr.batch * tr.q_heads * tr.L, device=dev)
+    o_e, lse_e = attn.encoder_blockcausal(q, k, v, tr.S)
+    o_d, lse_d = attn.decoder_train(q, ke, ve, k, v, tr.S)
+    ws_b = torch.empty(attn.train_backward_workspace_bytes(tr.batch, tr.q_heads, tr.kv_heads, tr.head_dim, tr.L),
+                       dtype=torch.uint8, device=dev)
     bev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     enc_ms = dec_ms = 0.0
     reps = 5
     for it in range(2 + reps):
         bev[0].record()
-        attn.encoder_backward(q, k, v, lse_e, go, tr.S, workspace=ws_b)
+        attn.encoder_backward(q, k, v, o_e, lse_e, go, tr.S, workspace=ws_b)
         bev[1].record()
-        attn.decoder_train_backward(q, ke, ve, k, v, lse_d, go, tr.S, workspace=ws_b)
+        attn.decoder_train_backward(q, ke, ve, k, v, o_d, lse_d, go, tr.S, workspace=ws_b)
         bev[2].record()
         torch.cuda.synchronize()
         if it >= 2:
@@ -260,11 +261,47 @@ def run_workload_set(torch, attn, workloads, dev, peaks):
     # five products of 2 d FLOPs per unmasked pair (recomputed Q K^T, dP, dV, dQ, dK): 2.5x forward
     fl_b = 2.5 * workloads.useful_flops_train(tr)
     res["train_pass_backward"] = {
-        "workload": tr.name + " backward", "kernels": "CUDA cores (dq pass, then dk/dv pass), fp32",
+        "workload": tr.name + " backward",
+        "kernels": "tcgen05: dq + D_i (query rows on TMEM lanes), then dk/dv (keys on TMEM lanes)",
         "encoder_ms": enc_ms, "decoder_ms": dec_ms,
         "useful_tflops": 2 * fl_b / ((enc_ms + dec_ms) * 1e-3) / 1e12,
-        "frac_tensor": 2 * fl_b / ((enc_ms + dec_ms) * 1e-3) / 1e12 / tc}
-    del q, k, v, ke, ve, go, ws_b
+        "frac_tensor": 2 * fl_b / ((enc_ms + dec_ms) * 1e-3) / 1e12 / tc,
+        # the two launches issue eight products of 2 d FLOPs per pair (S and dP twice, p K and u K,
+        # p^T dO and ds^T Q) against the five of the definition
+        "issued_mma_flops_per_useful": 8 / 5}
+    # ---- one BD3LM layer against one E2D2 encoder / decoder layer (same shapes, same kernels):
+    # BD3LM's 2L-token attention = a decoder-train call on the noised rows + an encoder call on the
+    # clean rows; the FLOPs table puts it at twice an E2D2 layer.  L2 flushed before every call.
+    qn, kn, vn, qc, kc, vc = q, k, v, ke, ve, go
+    on, oc = torch.empty_like(qn), torch.empty_like(qc)
+    ln, lc = torch.empty(shp[:3], device=dev), torch.empty(shp[:3], device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    cases = {
+        "bd3lm_layer": lambda: (attn.decoder_train(qn, kc, vc, kn, vn, tr.S, out=on, lse=ln),
+                                attn.encoder_blockcausal(qc, kc, vc, tr.S, out=oc, lse=lc)),
+        "e2d2_encoder_layer": lambda: attn.encoder_blockcausal(qc, kc, vc, tr.S, out=oc, lse=lc),
+        "e2d2_decoder_layer": lambda: attn.decoder_train(qn, kc, vc, kn, vn, tr.S, out=on, lse=ln),
+    }
+    lay = {}
+    for name, fn in cases.items():
+        tot, reps = 0.0, 20
+        for it in range(3 + reps):
+            flush.zero_()
+            bev[0].record()
+            fn()
+            bev[1].record()
+            torch.cuda.synchronize()
+            if it >= 3:
+                tot += bev[0].elapsed_time(bev[1]) * 1e3 / reps
+        lay[name + "_us"] = tot
+    pairs_e2d2 = (tr.L * tr.L + tr.L * tr.S) // 2
+    res["bd3lm_vs_e2d2"] = {
+        "workload": tr.name + " (one attention layer each)", **lay,
+        "time_ratio_vs_encoder_layer": lay["bd3lm_layer_us"] / lay["e2d2_encoder_layer_us"],
+        "time_ratio_vs_decoder_layer": lay["bd3lm_layer_us"] / lay["e2d2_decoder_layer_us"],
+        "pairs_per_head": {"bd3lm": 2 * pairs_e2d2, "e2d2_layer": pairs_e2d2}, "pages_flops_ratio": 2.0,
+        "l2": "flushed before every call"}
+    del q, k, v, ke, ve, go, ws_b, flush, on, oc
     # ---- long-context sample loop
     w = workloads.SAMPLE_LOOP
     B, Hq, Hkv, Sb, d, layers = w["batch"], w["q_heads"], w["kv_heads"], w["S"], w["head_dim"], w["layers"]

@@ -74,9 +74,9 @@ def load(path: Path | str | None = None):
     lib.e2d2_attn_decoder_sample_noalloc.restype = ctypes.c_int
     lib.e2d2_attn_train_backward_workspace.argtypes = [Dims, ci]
     lib.e2d2_attn_train_backward_workspace.restype = ctypes.c_size_t
-    lib.e2d2_attn_encoder_backward.argtypes = [vp, vp, vp, fp, vp, vp, vp, vp, Dims, ci, ci, vp,
+    lib.e2d2_attn_encoder_backward.argtypes = [vp, vp, vp, vp, fp, vp, vp, vp, vp, Dims, ci, ci, vp,
                                                ctypes.c_size_t, st]
-    lib.e2d2_attn_decoder_train_backward.argtypes = [vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, vp, vp,
+    lib.e2d2_attn_decoder_train_backward.argtypes = [vp, vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, vp, vp,
                                                      Dims, ci, ci, vp, ctypes.c_size_t, st]
     lib.e2d2_attn_decoder_sample_plan.argtypes = [Dims, ci, ci, ci, ctypes.POINTER(SamplePlan)]
     lib.e2d2_attn_decoder_sample_plan.restype = ctypes.c_int

@@ -133,6 +133,12 @@ def decoder_train(q, k_enc, v_enc, k_dec, v_dec, S: int, scale=None, out=None, l
     return out, lse_t
 
 
+def train_backward_workspace_bytes(batch, q_heads, kv_heads, head_dim, L) -> int:
+    """Bytes of workspace the backward calls need (no GPU needed)."""
+    lib = _lib.load()
+    return int(lib.e2d2_attn_train_backward_workspace(_dims(batch, q_heads, kv_heads, head_dim, None), L))
+
+
 def _train_backward_ws(lib, B, Hq, Hkv, d, L, scale, device, workspace):
     need = lib.e2d2_attn_train_backward_workspace(_dims(B, Hq, Hkv, d, scale), L)
     if workspace is None:
@@ -141,22 +147,22 @@ def _train_backward_ws(lib, B, Hq, Hkv, d, L, scale, device, workspace):
 
 
 @_device_guard
-def encoder_backward(q, k, v, lse, dout, S: int, scale=None, workspace=None):
+def encoder_backward(q, k, v, out, lse, dout, S: int, scale=None, workspace=None):
     """Gradients of the encoder call: (dq [B,Hq,L,d], dk, dv [B,Hkv,L,d]) bf16, from the forward's
-    lse (fp32) and the output gradient dout."""
+    output out (bf16) and lse (fp32) and the output gradient dout."""
     lib = _lib.load()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _need(t, n)
     _need(lse, "lse", dtype=torch.float32, ndim=3)
     B, Hq, L, d = q.shape
     Hkv = k.shape[1]
-    if k.shape != (B, Hkv, L, d) or v.shape != k.shape or dout.shape != q.shape:
-        raise ValueError("k/v must be [B, Hkv, L, d]; dout must match q")
+    if k.shape != (B, Hkv, L, d) or v.shape != k.shape or dout.shape != q.shape or out.shape != q.shape:
+        raise ValueError("k/v must be [B, Hkv, L, d]; out and dout must match q")
     if lse.shape != (B, Hq, L):
         raise ValueError("lse must be [B, Hq, L]")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = _train_backward_ws(lib, B, Hq, Hkv, d, L, scale, q.device, workspace)
-    st = lib.e2d2_attn_encoder_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), lse.data_ptr(),
+    st = lib.e2d2_attn_encoder_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                         dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                                         _dims(B, Hq, Hkv, d, scale), L, S, ws.data_ptr(),
                                         ws.numel() * ws.element_size(), _stream(q))
@@ -165,11 +171,12 @@ def encoder_backward(q, k, v, lse, dout, S: int, scale=None, workspace=None):
 
 
 @_device_guard
-def decoder_train_backward(q, k_enc, v_enc, k_dec, v_dec, lse, dout, S: int, scale=None, workspace=None):
-    """Gradients of the decoder train call: (dq, dk_enc, dv_enc, dk_dec, dv_dec) bf16."""
+def decoder_train_backward(q, k_enc, v_enc, k_dec, v_dec, out, lse, dout, S: int, scale=None, workspace=None):
+    """Gradients of the decoder train call: (dq, dk_enc, dv_enc, dk_dec, dv_dec) bf16, from the
+    forward's output out and lse and the output gradient dout."""
     lib = _lib.load()
     for t, n in ((q, "q"), (k_enc, "k_enc"), (v_enc, "v_enc"), (k_dec, "k_dec"), (v_dec, "v_dec"),
-                 (dout, "dout")):
+                 (out, "out"), (dout, "dout")):
         _need(t, n)
     _need(lse, "lse", dtype=torch.float32, ndim=3)
     B, Hq, L, d = q.shape
@@ -177,13 +184,13 @@ def decoder_train_backward(q, k_enc, v_enc, k_dec, v_dec, lse, dout, S: int, sca
     for t in (k_enc, v_enc, k_dec, v_dec):
         if t.shape != (B, Hkv, L, d):
             raise ValueError("k_enc/v_enc/k_dec/v_dec must be [B, Hkv, L, d] matching q")
-    if dout.shape != q.shape or lse.shape != (B, Hq, L):
-        raise ValueError("dout must match q and lse must be [B, Hq, L]")
+    if dout.shape != q.shape or out.shape != q.shape or lse.shape != (B, Hq, L):
+        raise ValueError("out and dout must match q and lse must be [B, Hq, L]")
     dq = torch.empty_like(q)
     grads = [torch.empty_like(k_enc) for _ in range(4)]
     ws = _train_backward_ws(lib, B, Hq, Hkv, d, L, scale, q.device, workspace)
     st = lib.e2d2_attn_decoder_train_backward(q.data_ptr(), k_enc.data_ptr(), v_enc.data_ptr(), k_dec.data_ptr(),
-                                              v_dec.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                                              v_dec.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
                                               dq.data_ptr(), *[g.data_ptr() for g in grads],
                                               _dims(B, Hq, Hkv, d, scale), L, S, ws.data_ptr(),
                                               ws.numel() * ws.element_size(), _stream(q))

@@ -1,0 +1,686 @@
+// attn_bwd_sm100.cuh -- backward of the two E2D2 train calls on the B200 tensor cores (sm_100a):
+// the encoder's block-causal self-attention and the decoder's fused self+cross attention over 2L
+// keys ("Encoder-Decoder Diffusion Language Models for Efficient Training and Inference", paper
+// notes, sec. 4: one encoder and one decoder pass with custom masks train all blocks).  The page
+// prints no backward; this is the plain derivative of those two calls.
+//
+// With p_ij = exp(scale q_i.k_j - lse_i) over the pairs the forward's mask allows,
+//     dp_ij = dout_i.v_j,   D_i = sum_j p_ij dp_ij,   ds_ij = p_ij (dp_ij - D_i),
+//     dq_i = scale sum_j ds_ij k_j,   dk_j = scale sum_i ds_ij q_i,   dv_j = sum_i p_ij dout_i.
+// Two launches of one warp-specialised template, deterministic (no atomics; every gradient
+// element is written once by the CTA that owns its row):
+//
+//   kBwdRowsQ   one item = 128 query rows of one head (rows on the TMEM lanes); the keys the
+//               rows see stream past in 64-key sub-tiles.  Per sub-tile
+//                   S  = Q K^T,  dP = dO V^T                        (tcgen05.mma -> TMEM)
+//                   p  = exp2(S scale log2e - lse_i log2e),  u = p (dp - c_i)
+//                   Y += p K,    X += u K                          (A = p / u from TMEM)
+//               with c_i = dout_i.out_i (out = the forward's output).  At the end
+//                   D_i = c_i + sum_j u_ij,   dq_i = scale (X_i - (D_i - c_i) Y_i),
+//               which is the formula above for ANY constant c_i (sum_j p_ij (dp_ij - D_i) k_j =
+//               sum_j p_ij (dp_ij - c_i) k_j - (D_i - c_i) sum_j p_ij k_j); c_i close to D_i keeps
+//               the bf16 operands u small where one key holds a row's weight, so the difference
+//               X - (D - c) Y does not cancel to rounding noise.  D_i and -lse_i log2e go to the
+//               workspace for the second launch.
+//   kBwdRowsKV  one item = 128 keys of one kv head and key source (keys on the TMEM lanes); the
+//               queries of every head of the GQA group that see them stream past in 64-query
+//               sub-tiles.  Per sub-tile
+//                   S^T = K Q^T,  dP^T = V dO^T,  p^T = exp2(...),  ds^T = p^T (dp^T - D)
+//                   dV += p^T dO,  dK += ds^T Q                      (A = p^T / ds^T from TMEM)
+//               and the item writes dk = scale dK and dv = dV.
+//
+// The mask is per TMEM lane an interval of the column index (the keys a query row sees, or the
+// queries that see a key), so sub-tiles outside every lane's interval are never loaded and no
+// mask matrix exists.  Rows past L come in as zeros (TMA out-of-bounds fill) and their interval
+// is empty; queries past L also carry lse = +inf in the workspace (p = 0).
+//
+// CTA = 12 warps: warp 0 issues the TMA loads (row tiles once per item, column sub-tiles through
+// a ring), warp 1 owns tensor memory and issues tcgen05.mma, warps 2..3 are idle, warps 4..7
+// and 8..11 are two softmax warpgroups that take alternate sub-tiles.  Tensor memory holds two
+// (S, dP) sets of 64 + 64 columns, so while one warpgroup turns set 0 into (p, u) the tensor core
+// computes the products of set 1 and the accumulations of the other; the two accumulators
+// (Y, X or dV, dK) take 2 x head_dim columns, double-buffered across items at head_dim <= 64.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "fmha_sm100.cuh"
+#include "ptx_sm100.cuh"
+
+namespace e2d2 {
+
+enum BwdSide : int { kBwdRowsQ = 0, kBwdRowsKV = 1 };
+
+constexpr int kBwdRows = 128;  // rows of an item (TMEM lanes)
+constexpr int kBwdCols = 64;   // columns of a sub-tile
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct alignas(64) BwdTcParams {
+    CUtensorMap tm_r1[2];  // row operand 1 (128-row boxes): rows-Q: Q at [0]; rows-KV: K of key source 0/1
+    CUtensorMap tm_r2[2];  // row operand 2: rows-Q: dO at [0]; rows-KV: V of key source 0/1
+    CUtensorMap tm_c1[2];  // column operand 1 (64-row boxes): rows-Q: K of key source 0/1; rows-KV: Q at [0]
+    CUtensorMap tm_c2[2];  // column operand 2: rows-Q: V of key source 0/1; rows-KV: dO at [0]
+    const float* lse;                 // rows-Q: the forward's lse [B*Hq][L] (natural log)
+    const __nv_bfloat16* out;         // rows-Q: the forward's output [B*Hq][L][D]
+    const __nv_bfloat16* dout;        // rows-Q: [B*Hq][L][D]
+    float* ws_nl2;                    // [B*Hq][Lpad]: -lse*log2(e), -inf past L (rows-Q writes it)
+    float* ws_D;                      // [B*Hq][Lpad]: D_i, 0 past L
+    __nv_bfloat16* g_a[2];            // rows-Q: dq at [0]; rows-KV: dv of key source 0/1
+    __nv_bfloat16* g_b[2];            // rows-KV: dk of key source 0/1
+    unsigned int* err;                // device error word
+    int batch, q_heads, kv_heads, group;
+    int L, S, Lpad, decoder;
+    float scale, scale_log2;
+    int n_row_tiles;                  // ceil(L / 128)
+    int num_items;
+};
+
+template <int D>
+struct BwdCfg {
+    static constexpr int RB = (D * 2 < 128) ? D * 2 : 128;   // bytes per smem row of one chunk
+    static constexpr int NCH = D * 2 / RB;                   // column chunks per row
+    static constexpr uint32_t SWZ = (RB == 128) ? 2u : 4u;   // 128-byte / 64-byte swizzle
+    static constexpr int ROW_CHUNK = kBwdRows * RB;
+    static constexpr int ROW_TILE = kBwdRows * D * 2;
+    static constexpr int COL_CHUNK = kBwdCols * RB;
+    static constexpr int COL_TILE = kBwdCols * D * 2;
+    static constexpr int KSTEPS_PER_CHUNK = RB / 32;         // 16-element k steps per chunk
+    static constexpr int RBUF = (D == 128) ? 1 : 2;          // row-tile buffers (items in flight)
+    static constexpr int NST = (D == 128) ? 4 : (D == 64 ? 6 : 8);  // column stages
+    static constexpr int NACC = (D == 128) ? 1 : 2;          // accumulator sets
+};
+
+template <int D>
+struct BwdSmem {
+    using C = BwdCfg<D>;
+    static constexpr int OFF_R = 0;                                        // [RBUF][2] row tiles
+    static constexpr int OFF_C = OFF_R + C::RBUF * 2 * C::ROW_TILE;        // [NST][2] column tiles
+    static constexpr int OFF_LD = OFF_C + C::NST * 2 * C::COL_TILE;        // [NST][2][64] nl2, D
+    static constexpr int OFF_X = OFF_LD + C::NST * 2 * kBwdCols * 4;       // [2][2][128] sum exchange
+    static constexpr int OFF_BAR = OFF_X + 2 * 2 * kBwdRows * 4;
+    // row_full[RBUF], row_empty[RBUF], col_full[NST], col_empty[NST], s_full[2], p_full[2],
+    // acc_full[NACC], acc_free[NACC], mma_drain, softmax_done
+    static constexpr int NBAR = 2 * C::RBUF + 2 * C::NST + 4 + 2 * C::NACC + 2;
+    static constexpr int OFF_MISC = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;
+    static constexpr int BYTES = OFF_MISC + 64;
+    static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
+};
+
+struct BwdItem {
+    int row_z;    // z of the row tiles: rows-Q b*Hq+h; rows-KV b*Hkv+g
+    int row0;     // first row (query or key index) of the item
+    int src;      // rows-KV: key source of the item (decoder: 0 encoder-side, 1 decoder-side)
+    int nsub;     // column sub-tiles
+    int a1, n1;   // rows-Q: source-1 key sub-tiles [a1, a1+n1), visited first
+    int n0;       // rows-Q: source-0 key sub-tiles [0, n0)
+    int qa, nq;   // rows-KV: query sub-tiles [qa, qa+nq) of each head of the group
+    int col_z0;   // rows-Q: b*Hkv + h/G; rows-KV: b*Hq + g*G (first query head of the group)
+};
+
+// Items in a fixed order that every role walks; longest first (static round robin over CTAs).
+template <int SIDE>
+struct BwdScheduler {
+    const BwdTcParams& p;
+    int k;
+    __device__ explicit BwdScheduler(const BwdTcParams& prm) : p(prm), k(blockIdx.x) {}
+
+    __device__ bool next(BwdItem& it) {
+        if (k >= p.num_items) return false;
+        const int L = p.L, S = p.S;
+        if (SIDE == kBwdRowsQ) {
+            const int BH = p.batch * p.q_heads;
+            const int qt = p.n_row_tiles - 1 - k / BH;  // later query tiles see more keys
+            const int bh = k % BH;
+            k += gridDim.x;
+            const int b = bh / p.q_heads, h = bh % p.q_heads;
+            it.row_z = bh;
+            it.row0 = qt * kBwdRows;
+            it.src = 0;
+            it.col_z0 = b * p.kv_heads + h / p.group;
+            const int r_last = min(L, it.row0 + kBwdRows) - 1;
+            const int blk0 = it.row0 / S, blkl = r_last / S;
+            const int hi = min(L, (blkl + 1) * S);
+            if (!p.decoder) {
+                it.a1 = 0;
+                it.n1 = 0;
+                it.n0 = ceil_div_i(hi, kBwdCols);
+            } else {
+                it.a1 = (blk0 * S) / kBwdCols;
+                it.n1 = ceil_div_i(hi, kBwdCols) - it.a1;
+                it.n0 = ceil_div_i(blkl * S, kBwdCols);
+            }
+            it.nsub = it.n1 + it.n0;
+            it.qa = it.nq = 0;
+        } else {
+            const int BH = p.batch * p.kv_heads;
+            const int per_src = BH * p.n_row_tiles;
+            const int src = k / per_src;  // decoder: encoder-side keys first (they see more queries)
+            const int kk = k % per_src;
+            const int kt = kk / BH, z = kk % BH;
+            k += gridDim.x;
+            it.row_z = z;
+            it.row0 = kt * kBwdRows;
+            it.src = src;
+            const int b = z / p.kv_heads, g = z % p.kv_heads;
+            it.col_z0 = b * p.q_heads + g * p.group;
+            const int k_last = min(L, it.row0 + kBwdRows) - 1;
+            const int blk0 = it.row0 / S, blkl = k_last / S;
+            int lo, hi;
+            if (!p.decoder) {
+                lo = blk0 * S;
+                hi = L;
+            } else if (src == 0) {
+                lo = min(L, (blk0 + 1) * S);
+                hi = L;
+            } else {
+                lo = blk0 * S;
+                hi = min(L, (blkl + 1) * S);
+            }
+            it.qa = lo / kBwdCols;
+            it.nq = (hi > lo) ? ceil_div_i(hi, kBwdCols) - it.qa : 0;
+            it.nsub = it.nq * p.group;
+            it.a1 = it.n1 = it.n0 = 0;
+        }
+        return true;
+    }
+};
+
+// Column sub-tile t of an item: key source (rows-Q), first column (key or query index) and the
+// z coordinate of its tensor map (and of the workspace row, rows-KV).
+struct BwdCol {
+    int src, y, z;
+};
+
+template <int SIDE>
+__device__ __forceinline__ BwdCol bwd_col(const BwdItem& it, int t) {
+    BwdCol r;
+    if (SIDE == kBwdRowsQ) {
+        if (t < it.n1) {
+            r.src = 1;
+            r.y = (it.a1 + t) * kBwdCols;
+        } else {
+            r.src = 0;
+            r.y = (t - it.n1) * kBwdCols;
+        }
+        r.z = it.col_z0;
+    } else {
+        const int hh = t / it.nq;
+        r.src = 0;
+        r.y = (it.qa + t - hh * it.nq) * kBwdCols;
+        r.z = it.col_z0 + hh;
+    }
+    return r;
+}
+
+// The allowed columns of this lane's row in source `src`: [lo, hi).
+//   rows-Q (row = query i):  encoder keys [0, end(i)); decoder encoder-side keys [0, start(i)),
+//                            decoder-side keys [start(i), end(i))
+//   rows-KV (row = key j):   encoder queries [start(j), L); decoder encoder-side keys are seen by
+//                            queries [end(j), L), decoder-side keys by [start(j), end(j))
+// with start(x) = floor(x/S) S and end(x) = min(L, start(x) + S); an invalid row (>= L) sees nothing.
+template <int SIDE>
+__device__ __forceinline__ void bwd_interval(const BwdTcParams& p, int row, int src, int& lo, int& hi) {
+    if (row >= p.L) {
+        lo = 0;
+        hi = 0;
+        return;
+    }
+    const int start = (row / p.S) * p.S;
+    const int end = min(p.L, start + p.S);
+    if (SIDE == kBwdRowsQ) {
+        if (!p.decoder) {
+            lo = 0;
+            hi = end;
+        } else if (src == 0) {
+            lo = 0;
+            hi = start;
+        } else {
+            lo = start;
+            hi = end;
+        }
+    } else {
+        if (!p.decoder) {
+            lo = start;
+            hi = p.L;
+        } else if (src == 0) {
+            lo = end;
+            hi = p.L;
+        } else {
+            lo = start;
+            hi = end;
+        }
+    }
+}
+
+// One sub-tile of one warpgroup, one lane = one row: reads the 64 S and 64 dP columns of its set,
+// writes p (bf16, packed over S columns 0..31) and u / ds (over dP columns 0..31), and returns
+// sum(u) (rows-Q).  Columns outside [cmin, cmax) get p = 0.
+//   rows-Q:  exponent argument s*sl2 + nl2_row, u = p (dp - c_row)
+//   rows-KV: exponent argument s*sl2 + nl2_col[c], u = p (dp - d_col[c])
+template <int SIDE>
+__device__ __forceinline__ float bwd_subtile(uint32_t set_tmem, int cmin, int cmax, float sl2, float nl2_row,
+                                             float c_row, const float* nl2_col, const float* d_col) {
+    uint32_t sr[64], dr[64];
+    ptx::tmem_ld32(set_tmem, sr);
+    ptx::tmem_ld32(set_tmem + 32, sr + 32);
+    ptx::tmem_ld32(set_tmem + 64, dr);
+    ptx::tmem_ld32(set_tmem + 96, dr + 32);
+    ptx::tmem_wait_ld();
+    ptx::reg_fence<64>(sr);
+    ptx::reg_fence<64>(dr);
+    float usum[2] = {0.f, 0.f};
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+        const bool mine = (cmin < 32 * a + 32) && (cmax > 32 * a);
+        const bool live = __any_sync(0xffffffffu, mine);
+        const bool whole = __all_sync(0xffffffffu, (cmin <= 32 * a) && (cmax >= 32 * a + 32));
+        uint32_t pk[16], uk[16];
+        if (live) {
+#pragma unroll
+            for (int c4 = 0; c4 < 32; c4 += 4) {
+                float nl[4], dd[4];
+                if (SIDE == kBwdRowsKV) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(nl2_col + 32 * a + c4);
+                    const float4 b4 = *reinterpret_cast<const float4*>(d_col + 32 * a + c4);
+                    nl[0] = a4.x; nl[1] = a4.y; nl[2] = a4.z; nl[3] = a4.w;
+                    dd[0] = b4.x; dd[1] = b4.y; dd[2] = b4.z; dd[3] = b4.w;
+                } else {
+                    nl[0] = nl[1] = nl[2] = nl[3] = nl2_row;
+                    dd[0] = dd[1] = dd[2] = dd[3] = c_row;
+                }
+                float pv[4], uv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = 32 * a + c4 + e;
+                    float pe = ptx::ex2(fmaf(__uint_as_float(sr[col]), sl2, nl[e]));
+                    if (!whole) pe = (col >= cmin && col < cmax) ? pe : 0.f;
+                    pv[e] = pe;
+                    uv[e] = pe * (__uint_as_float(dr[col]) - dd[e]);
+                }
+                usum[(c4 >> 2) & 1] += (uv[0] + uv[1]) + (uv[2] + uv[3]);
+                pk[c4 / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
+                pk[c4 / 2 + 1] = ptx::pack_bf16x2(pv[2], pv[3]);
+                uk[c4 / 2] = ptx::pack_bf16x2(uv[0], uv[1]);
+                uk[c4 / 2 + 1] = ptx::pack_bf16x2(uv[2], uv[3]);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk[c] = uk[c] = 0u;
+        }
+        ptx::tmem_st16(set_tmem + 16 * a, pk);
+        ptx::tmem_st16(set_tmem + 64 + 16 * a, uk);
+    }
+    return usum[0] + usum[1];
+}
+
+// Dot product of two bf16 rows of length D (16-byte loads), fp32.
+template <int D>
+__device__ __forceinline__ float row_dot_bf16(const __nv_bfloat16* a, const __nv_bfloat16* b) {
+    const uint4* a4 = reinterpret_cast<const uint4*>(a);
+    const uint4* b4 = reinterpret_cast<const uint4*>(b);
+    float s[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+        const uint4 x = __ldg(a4 + i), y = __ldg(b4 + i);
+        const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[j]));
+            const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[j]));
+            s[j & 1] = fmaf(xf.x, yf.x, s[j & 1]);
+            s[j & 1] = fmaf(xf.y, yf.y, s[j & 1]);
+        }
+    }
+    return s[0] + s[1];
+}
+
+// Writes N columns of one gradient row: values * f, bf16, 16-byte stores.
+template <int N>
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float* v, float f) {
+#pragma unroll
+    for (int c = 0; c < N; c += 8) reinterpret_cast<uint4*>(dst)[c / 8] = pack8_bf16(v + c, f);
+}
+
+template <int D, int SIDE>
+__global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __grid_constant__ BwdTcParams p) {
+    using C = BwdCfg<D>;
+    using SM = BwdSmem<D>;
+    constexpr int NST = C::NST, RBUF = C::RBUF, NACC = C::NACC;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+#define E2D2_BWD_SMEM_POINTERS                                                                       \
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &      \
+                                               ~static_cast<uintptr_t>(1023));                       \
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::OFF_BAR);                                \
+    uint64_t* row_full = bars;                                                                       \
+    uint64_t* row_empty = row_full + RBUF;                                                           \
+    uint64_t* col_full = row_empty + RBUF;                                                           \
+    uint64_t* col_empty = col_full + NST;                                                            \
+    uint64_t* s_full = col_empty + NST;                                                              \
+    uint64_t* p_full = s_full + 2;                                                                   \
+    uint64_t* acc_full = p_full + 2;                                                                 \
+    uint64_t* acc_free = acc_full + NACC;                                                            \
+    uint64_t* mma_drain = acc_free + NACC;                                                           \
+    uint64_t* softmax_done = mma_drain + 1;                                                          \
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);                        \
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);             \
+    (void)row_full; (void)row_empty; (void)col_full; (void)col_empty; (void)s_full; (void)p_full;    \
+    (void)acc_full; (void)acc_free; (void)mma_drain; (void)softmax_done; (void)tmem_holder;          \
+    (void)abort_flag;
+    uint32_t tmem_base;
+    {
+        E2D2_BWD_SMEM_POINTERS
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < RBUF; ++i) {
+                ptx::mbar_init(&row_full[i], 1);
+                ptx::mbar_init(&row_empty[i], 1);
+            }
+            for (int i = 0; i < NST; ++i) {
+                ptx::mbar_init(&col_full[i], 1);
+                ptx::mbar_init(&col_empty[i], 1);
+            }
+            for (int i = 0; i < 2; ++i) {
+                ptx::mbar_init(&s_full[i], 1);
+                ptx::mbar_init(&p_full[i], 128);
+            }
+            for (int i = 0; i < NACC; ++i) {
+                ptx::mbar_init(&acc_full[i], 1);
+                ptx::mbar_init(&acc_free[i], kSoftmaxThreads);
+            }
+            ptx::mbar_init(mma_drain, 1);
+            ptx::mbar_init(softmax_done, kSoftmaxThreads);
+            *abort_flag = 0;
+            ptx::fence_mbar_init();
+        }
+        if (warp == 1) {
+            ptx::tmem_alloc(tmem_holder, kTmemCols);
+            ptx::tmem_relinquish();
+        }
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+        tmem_base = *tmem_holder;
+    }
+
+    E2D2_BWD_SMEM_POINTERS
+    const uint32_t smem_base = ptx::smem_u32(smem);
+    const uint32_t sR = smem_base + SM::OFF_R;
+    const uint32_t sC = smem_base + SM::OFF_C;
+
+    if (warp == 0) {
+        ptx::setmaxnreg_dec<kRegsControl>();
+        // ------------------------------------------------------------------ TMA producer
+        const bool leader = ptx::elect_one();
+        if (leader) {
+            for (int i = 0; i < 2; ++i) {
+                ptx::tma_prefetch_desc(&p.tm_r1[i]);
+                ptx::tma_prefetch_desc(&p.tm_r2[i]);
+                ptx::tma_prefetch_desc(&p.tm_c1[i]);
+                ptx::tma_prefetch_desc(&p.tm_c2[i]);
+            }
+        }
+        __syncwarp();
+        BwdScheduler<SIDE> sched(p);
+        BwdItem it;
+        uint32_t n = 0, iw = 0;
+        bool ok = true;
+        while (ok && sched.next(it)) {
+            if (it.nsub == 0) continue;
+            const uint32_t rb = iw % RBUF;
+            ok = wait_bar_warp(&row_empty[rb], ((iw / RBUF) & 1) ^ 1, abort_flag, p.err);
+            if (!ok) break;
+            if (leader) {
+                const int rs = (SIDE == kBwdRowsQ) ? 0 : it.src;
+                ptx::mbar_arrive_expect_tx(&row_full[rb], 2 * C::ROW_TILE);
+                for (int ch = 0; ch < C::NCH; ++ch) {
+                    ptx::tma_load_3d(&p.tm_r1[rs], &row_full[rb],
+                                     smem + SM::OFF_R + (rb * 2 + 0) * C::ROW_TILE + ch * C::ROW_CHUNK,
+                                     ch * (C::RB / 2), it.row0, it.row_z);
+                    ptx::tma_load_3d(&p.tm_r2[rs], &row_full[rb],
+                                     smem + SM::OFF_R + (rb * 2 + 1) * C::ROW_TILE + ch * C::ROW_CHUNK,
+                                     ch * (C::RB / 2), it.row0, it.row_z);
+                }
+            }
+            __syncwarp();
+            ++iw;
+            for (int t = 0; t < it.nsub; ++t) {
+                const uint32_t st = n % NST;
+                ok = wait_bar_warp(&col_empty[st], ((n / NST) & 1) ^ 1, abort_flag, p.err);
+                if (!ok) break;
+                const BwdCol cr = bwd_col<SIDE>(it, t);
+                if (leader) {
+                    const uint32_t bytes = 2 * C::COL_TILE + (SIDE == kBwdRowsKV ? 2 * kBwdCols * 4 : 0);
+                    ptx::mbar_arrive_expect_tx(&col_full[st], bytes);
+                    for (int ch = 0; ch < C::NCH; ++ch) {
+                        ptx::tma_load_3d(&p.tm_c1[cr.src], &col_full[st],
+                                         smem + SM::OFF_C + (st * 2 + 0) * C::COL_TILE + ch * C::COL_CHUNK,
+                                         ch * (C::RB / 2), cr.y, cr.z);
+                        ptx::tma_load_3d(&p.tm_c2[cr.src], &col_full[st],
+                                         smem + SM::OFF_C + (st * 2 + 1) * C::COL_TILE + ch * C::COL_CHUNK,
+                                         ch * (C::RB / 2), cr.y, cr.z);
+                    }
+                    if (SIDE == kBwdRowsKV) {
+                        const size_t off = static_cast<size_t>(cr.z) * p.Lpad + cr.y;
+                        ptx::bulk_load_g2s(smem + SM::OFF_LD + st * 2 * kBwdCols * 4, p.ws_nl2 + off, kBwdCols * 4,
+                                           &col_full[st]);
+                        ptx::bulk_load_g2s(smem + SM::OFF_LD + st * 2 * kBwdCols * 4 + kBwdCols * 4, p.ws_D + off,
+                                           kBwdCols * 4, &col_full[st]);
+                    }
+                }
+                __syncwarp();
+                ++n;
+            }
+        }
+        // Never leave with copies in flight: wait for the last load of every buffer.
+        volatile int no_abort = 0;
+        for (uint32_t i = n > static_cast<uint32_t>(NST) ? n - NST : 0u; i < n; ++i)
+            wait_bar_warp(&col_full[i % NST], (i / NST) & 1u, &no_abort, p.err);
+        for (uint32_t i = iw > static_cast<uint32_t>(RBUF) ? iw - RBUF : 0u; i < iw; ++i)
+            wait_bar_warp(&row_full[i % RBUF], (i / RBUF) & 1u, &no_abort, p.err);
+    } else if (warp == 1) {
+        ptx::setmaxnreg_dec<kRegsControl>();
+        // ------------------------------------------------------------------ MMA issuer
+        const bool leader = ptx::elect_one();
+        const uint64_t kdesc = ptx::smem_desc(0, 16, 8 * C::RB, C::SWZ);              // K-major
+        const uint64_t mndesc = ptx::smem_desc(0, C::COL_CHUNK, 8 * C::RB, C::SWZ);   // MN-major
+        constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(kBwdRows, kBwdCols, false);
+        constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(kBwdRows, D, true);
+        BwdScheduler<SIDE> sched(p);
+        BwdItem it;
+        uint32_t n = 0, iw = 0;
+        // The accumulation of sub-tile n is issued after the products of sub-tile n+1, so the
+        // tensor core works on one set while a softmax warpgroup works on the other.
+        bool have = false;
+        uint32_t pv_n = 0, pv_iw = 0;
+        bool pv_first = false, pv_last = false;
+        auto issue_acc = [&]() -> bool {
+            const uint32_t set = pv_n & 1u, st = pv_n % NST, ab = pv_iw % NACC;
+            if (!wait_bar_warp(&p_full[set], (pv_n >> 1) & 1u, abort_flag, p.err)) return false;
+            if (pv_first && !wait_bar_warp(&acc_free[ab], ((pv_iw / NACC) & 1u) ^ 1u, abort_flag, p.err))
+                return false;
+            ptx::tc_fence_after();
+            if (leader) {
+                const uint32_t c1 = sC + (st * 2 + 0) * C::COL_TILE;
+                const uint32_t c2 = sC + (st * 2 + 1) * C::COL_TILE;
+                const uint32_t ba = (SIDE == kBwdRowsQ) ? c1 : c2;  // Y += p K  |  dV += p^T dO
+                const uint32_t bb = c1;                             // X += u K  |  dK += ds^T Q
+                const uint32_t acc = tmem_base + 256 + ab * 2 * D;
+                const uint32_t pset = tmem_base + set * 128;
+#pragma unroll
+                for (int ks = 0; ks < kBwdCols / 16; ++ks) {
+                    const uint32_t accum = (pv_first && ks == 0) ? 0u : 1u;
+                    ptx::mma_ts(acc, pset + 8 * ks, mndesc | ((ba + ks * 16 * C::RB) >> 4), idesc_o, accum);
+                    ptx::mma_ts(acc + D, pset + 64 + 8 * ks, mndesc | ((bb + ks * 16 * C::RB) >> 4), idesc_o, accum);
+                }
+                ptx::mma_commit(&col_empty[st]);
+                if (pv_last) ptx::mma_commit(&acc_full[ab]);
+            }
+            __syncwarp();
+            return true;
+        };
+        bool ok = true;
+        while (ok && sched.next(it)) {
+            if (it.nsub == 0) continue;
+            const uint32_t rb = iw % RBUF;
+            ok = wait_bar_warp(&row_full[rb], (iw / RBUF) & 1u, abort_flag, p.err);
+            if (!ok) break;
+            const uint32_t r1 = sR + (rb * 2 + 0) * C::ROW_TILE;
+            const uint32_t r2 = sR + (rb * 2 + 1) * C::ROW_TILE;
+            for (int t = 0; t < it.nsub && ok; ++t) {
+                const uint32_t st = n % NST, set = n & 1u;
+                ok = wait_bar_warp(&col_full[st], (n / NST) & 1u, abort_flag, p.err);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                if (leader) {
+                    const uint32_t c1 = sC + (st * 2 + 0) * C::COL_TILE;
+                    const uint32_t c2 = sC + (st * 2 + 1) * C::COL_TILE;
+                    const uint32_t sset = tmem_base + set * 128;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t ro = (ks / C::KSTEPS_PER_CHUNK) * C::ROW_CHUNK + (ks % C::KSTEPS_PER_CHUNK) * 32;
+                        const uint32_t co = (ks / C::KSTEPS_PER_CHUNK) * C::COL_CHUNK + (ks % C::KSTEPS_PER_CHUNK) * 32;
+                        ptx::mma_ss(sset, kdesc | ((r1 + ro) >> 4), kdesc | ((c1 + co) >> 4), idesc_s, ks > 0 ? 1u : 0u);
+                        ptx::mma_ss(sset + 64, kdesc | ((r2 + ro) >> 4), kdesc | ((c2 + co) >> 4), idesc_s,
+                                    ks > 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit(&s_full[set]);
+                    if (t == it.nsub - 1) ptx::mma_commit(&row_empty[rb]);
+                }
+                __syncwarp();
+                if (have) ok = issue_acc();
+                have = true;
+                pv_n = n;
+                pv_iw = iw;
+                pv_first = (t == 0);
+                pv_last = (t == it.nsub - 1);
+                ++n;
+            }
+            ++iw;
+        }
+        if (ok && have) ok = issue_acc();
+        // Drain: every MMA issued by this warp completes, and every softmax thread is done with
+        // tensor memory, before it is released.
+        if (leader) ptx::mma_commit(mma_drain);
+        __syncwarp();
+        volatile int no_abort = 0;
+        wait_bar_warp(mma_drain, 0, &no_abort, p.err);
+        wait_bar_warp(softmax_done, 0, &no_abort, p.err);
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, kTmemCols);
+    } else if (warp < 4) {
+        ptx::setmaxnreg_dec<kRegsControl>();
+    } else {
+        ptx::setmaxnreg_inc<kRegsSoftmax>();
+        // ------------------------------------------------------------------ softmax warpgroups
+        // Warpgroup w (warps 4+4w .. 7+4w) takes the sub-tiles n with n % 2 == w (tensor-memory
+        // set w).  Every thread owns one row (its TMEM lane).  Waits never break these loops, so
+        // every warp takes every named barrier even after a bounded wait gave up.
+        const int w = (warp - 4) >> 2;
+        const int quarter = warp & 3;
+        const int lrow = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const float sl2 = p.scale_log2;
+        float* xch = reinterpret_cast<float*>(smem + SM::OFF_X);  // [2][2][128]
+        BwdScheduler<SIDE> sched(p);
+        BwdItem it;
+        uint32_t n = 0, iw = 0, own = 0;
+        while (sched.next(it)) {
+            const int row = it.row0 + lrow;
+            const bool valid = row < p.L;
+            if (it.nsub == 0) {
+                // rows-KV only (every query row sees a key): keys that no query sees get zero
+                // gradients.
+                if (SIDE == kBwdRowsKV && valid) {
+                    const float zero[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    __nv_bfloat16* dst = (w == 0 ? p.g_a[it.src] : p.g_b[it.src]) +
+                                         (static_cast<size_t>(it.row_z) * p.L + row) * D;
+#pragma unroll
+                    for (int c = 0; c < D; c += 8) store_row_bf16<8>(dst + c, zero, 1.f);
+                }
+                continue;
+            }
+            int lo0, hi0, lo1, hi1;
+            bwd_interval<SIDE>(p, row, SIDE == kBwdRowsQ ? 0 : it.src, lo0, hi0);
+            bwd_interval<SIDE>(p, row, 1, lo1, hi1);
+            float nl2_row = 0.f, c_row = 0.f;
+            if (SIDE == kBwdRowsQ && valid) {
+                const size_t r = static_cast<size_t>(it.row_z) * p.L + row;
+                nl2_row = -__ldg(p.lse + r) * kLog2e;
+                c_row = row_dot_bf16<D>(p.dout + r * D, p.out + r * D);
+            }
+            float usum = 0.f;
+            for (int t = 0; t < it.nsub; ++t, ++n) {
+                if (static_cast<int>(n & 1u) != w) continue;
+                wait_bar_warp(&s_full[w], own & 1u, abort_flag, p.err);
+                ptx::tc_fence_after();
+                const BwdCol cr = bwd_col<SIDE>(it, t);
+                const bool s1 = (SIDE == kBwdRowsQ) && cr.src == 1;
+                const int cmin = (s1 ? lo1 : lo0) - cr.y;
+                const int cmax = (s1 ? hi1 : hi0) - cr.y;
+                const float* ld = reinterpret_cast<const float*>(smem + SM::OFF_LD) + (n % NST) * 2 * kBwdCols;
+                // The per-column lse / D of a rows-KV sub-tile come in by bulk copy with the
+                // stage: observe the stage's barrier (already complete) before reading them.
+                if (SIDE == kBwdRowsKV) wait_bar_warp(&col_full[n % NST], (n / NST) & 1u, abort_flag, p.err);
+                usum += bwd_subtile<SIDE>(tmem_base + lane_off + w * 128, cmin, cmax, sl2, nl2_row, c_row, ld,
+                                          ld + kBwdCols);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&p_full[w]);
+                ++own;
+            }
+            // ------------------------------------------------------------ epilogue
+            const uint32_t ab = iw % NACC;
+            const uint32_t acc = tmem_base + lane_off + 256 + ab * 2 * D;
+            if (SIDE == kBwdRowsQ) {
+                // D_i - c_i = the sum of u over both warpgroups' sub-tiles.
+                const int par = iw & 1;
+                xch[(par * 2 + w) * kBwdRows + lrow] = usum;
+                ptx::named_barrier_sync(1, kSoftmaxThreads);
+                const float du = xch[(par * 2 + 0) * kBwdRows + lrow] + xch[(par * 2 + 1) * kBwdRows + lrow];
+                wait_bar_warp(&acc_full[ab], (iw / NACC) & 1u, abort_flag, p.err);
+                ptx::tc_fence_after();
+                constexpr int HALF = D / 2;
+                constexpr int CW = HALF < 32 ? HALF : 32;
+                __nv_bfloat16* dq = p.g_a[0] + (static_cast<size_t>(it.row_z) * p.L + row) * D;
+#pragma unroll
+                for (int c0 = w * HALF; c0 < (w + 1) * HALF; c0 += CW) {
+                    float y[CW], x[CW];
+                    load_tmem_cols<CW>(acc + c0, y);
+                    load_tmem_cols<CW>(acc + D + c0, x);
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) x[c] = fmaf(-du, y[c], x[c]);
+                    if (valid) store_row_bf16<CW>(dq + c0, x, p.scale);
+                }
+                if (w == 0) {
+                    const size_t r = static_cast<size_t>(it.row_z) * p.Lpad + row;
+                    p.ws_nl2[r] = valid ? nl2_row : -INFINITY;
+                    p.ws_D[r] = valid ? c_row + du : 0.f;
+                }
+            } else {
+                wait_bar_warp(&acc_full[ab], (iw / NACC) & 1u, abort_flag, p.err);
+                ptx::tc_fence_after();
+                constexpr int CW = D < 32 ? D : 32;
+                __nv_bfloat16* dst = (w == 0 ? p.g_a[it.src] : p.g_b[it.src]) +
+                                     (static_cast<size_t>(it.row_z) * p.L + row) * D;
+                const float f = (w == 0) ? 1.f : p.scale;
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += CW) {
+                    float v[CW];
+                    load_tmem_cols<CW>(acc + w * D + c0, v);
+                    if (valid) store_row_bf16<CW>(dst + c0, v, f);
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&acc_free[ab]);
+            ++iw;
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(softmax_done);
+    }
+#undef E2D2_BWD_SMEM_POINTERS
+}
+
+}  // namespace e2d2

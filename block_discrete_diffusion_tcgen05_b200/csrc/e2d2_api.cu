@@ -9,7 +9,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "attn_bwd_simple.cuh"
+#include "attn_bwd_sm100.cuh"
 #include "e2d2_attn.h"
 #include "fmha_keyrow_sm100.cuh"
 #include "fmha_sm100.cuh"
@@ -213,58 +213,117 @@ e2d2_status train_common(int mode, const void* q, const void* k0, const void* v0
                             : dispatch_fmha<kDecoderTrain>(D, prm, grid, st);
 }
 
-// Backward of the train calls: dq (and D_i = sum_j p_ij dout_i.v_j into the workspace), then dk/dv.
-e2d2_status train_backward(bool decoder, const BwdParams& base, const e2d2_dims& dm, int L, int S,
-                           void* workspace, size_t ws_bytes, cudaStream_t st) {
+// Backward of the train calls: two launches of attn_bwd_sm100_kernel on the stream, rows-Q
+// (dq, and D_i / -lse_i log2e into the workspace), then rows-KV (dk, dv).
+struct BwdArgs {
+    const void *q, *k0, *v0, *k1, *v1, *out, *dout;
+    const float* lse;
+    void *dq, *dk0, *dv0, *dk1, *dv1;
+};
+
+long long bwd_lpad(int L) { return (static_cast<long long>(L) + kBwdRows - 1) / kBwdRows * kBwdRows; }
+
+template <int D, int SIDE>
+e2d2_status launch_bwd(const BwdTcParams& prm, int grid, cudaStream_t st) {
+    using SM = BwdSmem<D>;
+    static_assert(SM::ALLOC <= 232448, "shared memory budget");
+    auto kern = attn_bwd_sm100_kernel<D, SIDE>;
+    const int smem = SM::ALLOC > 118784 ? SM::ALLOC : 118784;
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return E2D2_ERR_CUDA;
+        configured_dev = dev;
+    }
+    kern<<<grid, kThreads, smem, st>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+}
+
+template <int SIDE>
+e2d2_status dispatch_bwd(int D, const BwdTcParams& prm, int grid, cudaStream_t st) {
+    switch (D) {
+        case 32: return launch_bwd<32, SIDE>(prm, grid, st);
+        case 64: return launch_bwd<64, SIDE>(prm, grid, st);
+        case 128: return launch_bwd<128, SIDE>(prm, grid, st);
+        default: return E2D2_ERR_UNSUPPORTED;
+    }
+}
+
+e2d2_status train_backward(bool decoder, const BwdArgs& a, const e2d2_dims& dm, int L, int S, void* workspace,
+                           size_t ws_bytes, cudaStream_t st) {
     e2d2_status s = check_dims(dm);
     if (s != E2D2_OK) return s;
     s = check_train_shape(dm, L, S);
     if (s != E2D2_OK) return s;
-    const size_t need = static_cast<size_t>(dm.batch) * dm.q_heads * L * sizeof(float);
+    const long long Lpad = bwd_lpad(L);
+    const size_t need = 2 * static_cast<size_t>(dm.batch) * dm.q_heads * Lpad * sizeof(float);
     if (!workspace || ws_bytes < need) return E2D2_ERR_WORKSPACE;
-    const void* ptrs[] = {base.q, base.k0, base.v0, base.dout, base.dq, base.dk0, base.dv0, workspace};
+    const void* ptrs[] = {a.q, a.k0, a.v0, a.out, a.dout, a.dq, a.dk0, a.dv0, workspace};
     for (const void* ptr : ptrs)
         if (!aligned16(ptr)) return E2D2_ERR_ALIGNMENT;
-    if (decoder && (!aligned16(base.k1) || !aligned16(base.v1) || !aligned16(base.dk1) || !aligned16(base.dv1)))
+    if (decoder && (!aligned16(a.k1) || !aligned16(a.v1) || !aligned16(a.dk1) || !aligned16(a.dv1)))
         return E2D2_ERR_ALIGNMENT;
-    if (reinterpret_cast<uintptr_t>(base.lse) & 3u) return E2D2_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(a.lse) & 3u) return E2D2_ERR_ALIGNMENT;
     DeviceInfo* di = nullptr;
     s = device_info(&di);
     if (s != E2D2_OK) return s;
 
-    BwdParams prm = base;
-    prm.dsum = static_cast<float*>(workspace);
+    const int D = dm.head_dim;
+    const long long BHq = static_cast<long long>(dm.batch) * dm.q_heads;
+    const long long BHkv = static_cast<long long>(dm.batch) * dm.kv_heads;
+    BwdTcParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.lse = a.lse;
+    prm.out = static_cast<const __nv_bfloat16*>(a.out);
+    prm.dout = static_cast<const __nv_bfloat16*>(a.dout);
+    prm.ws_nl2 = static_cast<float*>(workspace);
+    prm.ws_D = static_cast<float*>(workspace) + BHq * Lpad;
+    prm.err = di->err;
     prm.batch = dm.batch;
     prm.q_heads = dm.q_heads;
     prm.kv_heads = dm.kv_heads;
     prm.group = dm.q_heads / dm.kv_heads;
     prm.L = L;
     prm.S = S;
+    prm.Lpad = static_cast<int>(Lpad);
+    prm.decoder = decoder ? 1 : 0;
     prm.scale = static_cast<float>(dm.scale > 0.f ? static_cast<double>(dm.scale)
                                                   : 1.0 / std::sqrt(static_cast<double>(dm.head_dim)));
-    prm.decoder = decoder ? 1 : 0;
-    constexpr int kWarpsPerBlock = 8;
-    const long long cap = static_cast<long long>(di->sms) * 16;  // 16 blocks of 8 warps per SM
-    const long long rows = static_cast<long long>(dm.batch) * dm.q_heads * L;
-    const long long keys = static_cast<long long>(dm.batch) * dm.kv_heads * L * (decoder ? 2 : 1);
-    const unsigned g1 = static_cast<unsigned>(std::min(cap, (rows + kWarpsPerBlock - 1) / kWarpsPerBlock));
-    const unsigned g2 = static_cast<unsigned>(std::min(cap, (keys + kWarpsPerBlock - 1) / kWarpsPerBlock));
-    switch (dm.head_dim) {
-        case 32:
-            attn_bwd_dq_kernel<32><<<g1, 32 * kWarpsPerBlock, 0, st>>>(prm);
-            attn_bwd_dkv_kernel<32><<<g2, 32 * kWarpsPerBlock, 0, st>>>(prm);
-            break;
-        case 64:
-            attn_bwd_dq_kernel<64><<<g1, 32 * kWarpsPerBlock, 0, st>>>(prm);
-            attn_bwd_dkv_kernel<64><<<g2, 32 * kWarpsPerBlock, 0, st>>>(prm);
-            break;
-        case 128:
-            attn_bwd_dq_kernel<128><<<g1, 32 * kWarpsPerBlock, 0, st>>>(prm);
-            attn_bwd_dkv_kernel<128><<<g2, 32 * kWarpsPerBlock, 0, st>>>(prm);
-            break;
-        default: return E2D2_ERR_UNSUPPORTED;
-    }
-    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+    prm.scale_log2 = scale_log2(dm);
+    prm.n_row_tiles = (L + kBwdRows - 1) / kBwdRows;
+    const void* k1 = decoder ? a.k1 : a.k0;
+    const void* v1 = decoder ? a.v1 : a.v0;
+
+    // rows-Q: row tiles Q, dO (128 rows); column sub-tiles K, V of each key source (64 rows).
+    BwdTcParams pq = prm;
+    bool ok = map_3d(&pq.tm_r1[0], a.q, D, L, BHq, L, kBwdRows) && map_3d(&pq.tm_r2[0], a.dout, D, L, BHq, L, kBwdRows) &&
+              map_3d(&pq.tm_c1[0], a.k0, D, L, BHkv, L, kBwdCols) && map_3d(&pq.tm_c2[0], a.v0, D, L, BHkv, L, kBwdCols) &&
+              map_3d(&pq.tm_c1[1], k1, D, L, BHkv, L, kBwdCols) && map_3d(&pq.tm_c2[1], v1, D, L, BHkv, L, kBwdCols);
+    pq.tm_r1[1] = pq.tm_r1[0];
+    pq.tm_r2[1] = pq.tm_r2[0];
+    pq.g_a[0] = pq.g_a[1] = static_cast<__nv_bfloat16*>(a.dq);
+    pq.num_items = static_cast<int>(BHq * prm.n_row_tiles);
+    // rows-KV: row tiles K, V of each key source (128 rows); column sub-tiles Q, dO (64 rows).
+    BwdTcParams pk = prm;
+    ok = ok && map_3d(&pk.tm_r1[0], a.k0, D, L, BHkv, L, kBwdRows) && map_3d(&pk.tm_r2[0], a.v0, D, L, BHkv, L, kBwdRows) &&
+         map_3d(&pk.tm_r1[1], k1, D, L, BHkv, L, kBwdRows) && map_3d(&pk.tm_r2[1], v1, D, L, BHkv, L, kBwdRows) &&
+         map_3d(&pk.tm_c1[0], a.q, D, L, BHq, L, kBwdCols) && map_3d(&pk.tm_c2[0], a.dout, D, L, BHq, L, kBwdCols);
+    if (!ok) return E2D2_ERR_CUDA;
+    pk.tm_c1[1] = pk.tm_c1[0];
+    pk.tm_c2[1] = pk.tm_c2[0];
+    pk.g_a[0] = static_cast<__nv_bfloat16*>(a.dv0);
+    pk.g_b[0] = static_cast<__nv_bfloat16*>(a.dk0);
+    pk.g_a[1] = static_cast<__nv_bfloat16*>(decoder ? a.dv1 : a.dv0);
+    pk.g_b[1] = static_cast<__nv_bfloat16*>(decoder ? a.dk1 : a.dk0);
+    pk.num_items = static_cast<int>((decoder ? 2 : 1) * BHkv * prm.n_row_tiles);
+
+    const int gq = pq.num_items < di->sms ? pq.num_items : di->sms;
+    const int gk = pk.num_items < di->sms ? pk.num_items : di->sms;
+    s = dispatch_bwd<kBwdRowsQ>(D, pq, gq, st);
+    if (s != E2D2_OK) return s;
+    return dispatch_bwd<kBwdRowsKV>(D, pk, gk, st);
 }
 
 struct SampleLayout {
@@ -332,11 +391,20 @@ SamplePlan plan_sample(const e2d2_dims& dims, int S, int P, int sms) {
     return pl;
 }
 
-// The sampling call; `append` (encoder block step) also writes the block's K/V to cache rows
-// P..P+S-1 from inside the same launch.
-e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, const void* v_cache, int capacity,
-                        int P, const void* k_blk, const void* v_blk, void* out, float* lse, e2d2_dims dims, int S,
-                        void* workspace, size_t ws_bytes, cudaStream_t stream) {
+// A sampling call, checked and encoded but not yet launched.
+struct SampleLaunch {
+    FmhaParams prm;
+    int keyrow_n;
+    int head_dim;
+    long long grid;
+};
+
+// Every check of a sampling call and the kernel parameters; launches and enqueues nothing, so an
+// error return leaves the stream untouched.  `append` (encoder block step) also writes the block's
+// K/V to cache rows P..P+S-1 from inside the same launch.
+e2d2_status sample_prepare(bool append, const void* q_blk, const void* k_cache, const void* v_cache, int capacity,
+                           int P, const void* k_blk, const void* v_blk, void* out, float* lse, e2d2_dims dims,
+                           int S, void* workspace, size_t ws_bytes, SampleLaunch* sl) {
     if (!q_blk || !k_cache || !v_cache || !k_blk || !v_blk || !out) return E2D2_ERR_INVALID_ARG;
     e2d2_status s = check_dims(dims);
     if (s != E2D2_OK) return s;
@@ -357,7 +425,7 @@ e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, con
 
     const int D = dims.head_dim;
     const int G = dims.q_heads / dims.kv_heads;
-    FmhaParams prm;
+    FmhaParams& prm = sl->prm;
     std::memset(&prm, 0, sizeof(prm));
     const long long BHkv = static_cast<long long>(dims.batch) * dims.kv_heads;
     const int S16 = (S + 15) / 16 * 16;
@@ -405,13 +473,29 @@ e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, con
     prm.whole_units = plan.whole_units;
     prm.split_ctas = plan.split_ctas;
     prm.total_tiles = plan.total_tiles;
-    const long long grid = plan.grid;
-    switch (keyrow_n) {
-        case 16: return launch_keyrow<16>(prm, static_cast<int>(grid), stream);
-        case 32: return launch_keyrow<32>(prm, static_cast<int>(grid), stream);
-        case 64: return launch_keyrow<64>(prm, static_cast<int>(grid), stream);
-        default: return dispatch_fmha<kDecoderSample>(D, prm, static_cast<int>(grid), stream);
+    sl->keyrow_n = keyrow_n;
+    sl->head_dim = D;
+    sl->grid = plan.grid;
+    return E2D2_OK;
+}
+
+e2d2_status sample_launch(const SampleLaunch& sl, cudaStream_t stream) {
+    const int grid = static_cast<int>(sl.grid);
+    switch (sl.keyrow_n) {
+        case 16: return launch_keyrow<16>(sl.prm, grid, stream);
+        case 32: return launch_keyrow<32>(sl.prm, grid, stream);
+        case 64: return launch_keyrow<64>(sl.prm, grid, stream);
+        default: return dispatch_fmha<kDecoderSample>(sl.head_dim, sl.prm, grid, stream);
     }
+}
+
+e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, const void* v_cache, int capacity,
+                        int P, const void* k_blk, const void* v_blk, void* out, float* lse, e2d2_dims dims, int S,
+                        void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    SampleLaunch sl;
+    const e2d2_status s = sample_prepare(append, q_blk, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims,
+                                         S, workspace, ws_bytes, &sl);
+    return s != E2D2_OK ? s : sample_launch(sl, stream);
 }
 
 }  // namespace
@@ -454,49 +538,52 @@ e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_enc, const 
 
 size_t e2d2_attn_train_backward_workspace(e2d2_dims dims, int L) {
     if (check_dims(dims) != E2D2_OK || L <= 0) return 0;
-    return static_cast<size_t>(dims.batch) * dims.q_heads * L * sizeof(float);
+    return 2 * static_cast<size_t>(dims.batch) * dims.q_heads * bwd_lpad(L) * sizeof(float);
 }
 
-e2d2_status e2d2_attn_encoder_backward(const void* q, const void* k, const void* v, const float* lse,
-                                       const void* dout, void* dq, void* dk, void* dv, e2d2_dims dims, int L,
-                                       int S, void* workspace, size_t ws_bytes, cudaStream_t stream) {
-    if (!q || !k || !v || !lse || !dout || !dq || !dk || !dv) return E2D2_ERR_INVALID_ARG;
-    BwdParams b;
-    std::memset(&b, 0, sizeof(b));
-    b.q = static_cast<const __nv_bfloat16*>(q);
-    b.k0 = static_cast<const __nv_bfloat16*>(k);
-    b.v0 = static_cast<const __nv_bfloat16*>(v);
-    b.lse = lse;
-    b.dout = static_cast<const __nv_bfloat16*>(dout);
-    b.dq = static_cast<__nv_bfloat16*>(dq);
-    b.dk0 = static_cast<__nv_bfloat16*>(dk);
-    b.dv0 = static_cast<__nv_bfloat16*>(dv);
-    return train_backward(false, b, dims, L, S, workspace, ws_bytes, stream);
+e2d2_status e2d2_attn_encoder_backward(const void* q, const void* k, const void* v, const void* out,
+                                       const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                       e2d2_dims dims, int L, int S, void* workspace, size_t ws_bytes,
+                                       cudaStream_t stream) {
+    if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return E2D2_ERR_INVALID_ARG;
+    BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.k0 = k;
+    a.v0 = v;
+    a.out = out;
+    a.lse = lse;
+    a.dout = dout;
+    a.dq = dq;
+    a.dk0 = dk;
+    a.dv0 = dv;
+    return train_backward(false, a, dims, L, S, workspace, ws_bytes, stream);
 }
 
 e2d2_status e2d2_attn_decoder_train_backward(const void* q_dec, const void* k_enc, const void* v_enc,
-                                             const void* k_dec, const void* v_dec, const float* lse,
-                                             const void* dout, void* dq, void* dk_enc, void* dv_enc, void* dk_dec,
-                                             void* dv_dec, e2d2_dims dims, int L, int S, void* workspace,
-                                             size_t ws_bytes, cudaStream_t stream) {
-    if (!q_dec || !k_enc || !v_enc || !k_dec || !v_dec || !lse || !dout || !dq || !dk_enc ||
+                                             const void* k_dec, const void* v_dec, const void* out,
+                                             const float* lse, const void* dout, void* dq, void* dk_enc,
+                                             void* dv_enc, void* dk_dec, void* dv_dec, e2d2_dims dims, int L,
+                                             int S, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!q_dec || !k_enc || !v_enc || !k_dec || !v_dec || !out || !lse || !dout || !dq || !dk_enc ||
         !dv_enc || !dk_dec || !dv_dec)
         return E2D2_ERR_INVALID_ARG;
-    BwdParams b;
-    std::memset(&b, 0, sizeof(b));
-    b.q = static_cast<const __nv_bfloat16*>(q_dec);
-    b.k0 = static_cast<const __nv_bfloat16*>(k_enc);
-    b.v0 = static_cast<const __nv_bfloat16*>(v_enc);
-    b.k1 = static_cast<const __nv_bfloat16*>(k_dec);
-    b.v1 = static_cast<const __nv_bfloat16*>(v_dec);
-    b.lse = lse;
-    b.dout = static_cast<const __nv_bfloat16*>(dout);
-    b.dq = static_cast<__nv_bfloat16*>(dq);
-    b.dk0 = static_cast<__nv_bfloat16*>(dk_enc);
-    b.dv0 = static_cast<__nv_bfloat16*>(dv_enc);
-    b.dk1 = static_cast<__nv_bfloat16*>(dk_dec);
-    b.dv1 = static_cast<__nv_bfloat16*>(dv_dec);
-    return train_backward(true, b, dims, L, S, workspace, ws_bytes, stream);
+    BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = q_dec;
+    a.k0 = k_enc;
+    a.v0 = v_enc;
+    a.k1 = k_dec;
+    a.v1 = v_dec;
+    a.out = out;
+    a.lse = lse;
+    a.dout = dout;
+    a.dq = dq;
+    a.dk0 = dk_enc;
+    a.dv0 = dv_enc;
+    a.dk1 = dk_dec;
+    a.dv1 = dv_dec;
+    return train_backward(true, a, dims, L, S, workspace, ws_bytes, stream);
 }
 
 size_t e2d2_attn_decoder_sample_workspace(e2d2_dims dims, int S, int capacity) {
@@ -642,10 +729,14 @@ e2d2_status e2d2_attn_decoder_sample_noalloc(const void* q_blk, const void* k_ca
     void* scratch = nullptr;
     e2d2_status s = noalloc_scratch(&scratch);
     if (s != E2D2_OK) return s;
+    // Every check first: an error return must leave nothing queued on the stream.
+    SampleLaunch sl;
+    s = sample_prepare(false, q_blk, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims, S, scratch,
+                       kNoAllocScratchBytes, &sl);
+    if (s != E2D2_OK) return s;
     // Ticket words must start at zero; they occupy the first kSampleMaxCtas ints.
     if (cudaMemsetAsync(scratch, 0, kSampleMaxCtas * sizeof(int), stream) != cudaSuccess) return E2D2_ERR_CUDA;
-    return e2d2_attn_decoder_sample(q_blk, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims, S,
-                                    scratch, kNoAllocScratchBytes, stream);
+    return sample_launch(sl, stream);
 }
 
 }  // extern "C"

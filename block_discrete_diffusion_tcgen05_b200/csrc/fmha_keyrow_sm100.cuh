@@ -660,10 +660,12 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                         for (int c = c_first; c <= c_last; ++c)
                             ptx::bulk_load_g2s(region + (c - c_first) * slot_bytes, slot_of(c), slot_bytes, merge_full);
                     }
-                    wait_bar_warp(merge_full, 0, abort_flag, p.err);
+                    // If the copies never landed (bounded wait gave up: error word set), the
+                    // slots are not merged and out / lse are left untouched.
+                    const bool landed = wait_bar_warp(merge_full, 0, abort_flag, p.err);
                     const int dq = (wtid & 3) * 32;
 #pragma unroll 1
-                    for (int col = wtid >> 2; col < cap; col += 32) {
+                    for (int col = wtid >> 2; landed && col < cap; col += 32) {
                         float mm = -INFINITY, ll = 0.f, acc[32];
 #pragma unroll
                         for (int i = 0; i < 32; ++i) acc[i] = 0.f;

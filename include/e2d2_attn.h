@@ -102,34 +102,42 @@ E2D2_API e2d2_status e2d2_attn_decoder_train(const void* q_dec, const void* k_en
  * of the two calls that a gradient step through them needs).  Gradients of
  * sum(dout * out) with respect to every input, the probabilities recomputed from the forward's
  * lse:  p_ij = exp(scale q_i.k_j - lse_i) over the keys the forward's mask lets row i see,
- * dp_ij = dout_i.v_j,  D_i = sum_j p_ij dp_ij (dout_i.out_i in exact arithmetic, formed here
- * from the probabilities, so the forward's bf16 out is not needed and its rounding does not
- * reach the gradients),  dq_i = scale sum_j p_ij (dp_ij - D_i) k_j,  dv_j = sum_i p_ij dout_i,
+ * dp_ij = dout_i.v_j,  D_i = sum_j p_ij dp_ij (formed from the probabilities, not from out),
+ * dq_i = scale sum_j p_ij (dp_ij - D_i) k_j,  dv_j = sum_i p_ij dout_i,
  * dk_j = scale sum_i p_ij (dp_ij - D_i) q_i, the sums over i running over every query head
  * that shares k_j's kv head (GQA).
  *   q, k, v (or q_dec, k_enc, v_enc, k_dec, v_dec), dims, L, S: exactly as passed to the
- *   forward call; lse (NOT NULL) is that call's lse; dout [batch][q_heads][L][d] bf16.
+ *   forward call; out and lse (both NOT NULL) are that call's outputs; dout
+ *   [batch][q_heads][L][d] bf16.  out serves only as a reference value: dq is accumulated as
+ *   sum_j p_ij (dp_ij - c_i) k_j - (D_i - c_i) sum_j p_ij k_j with c_i = dout_i.out_i, which is
+ *   the same gradient for any c_i and keeps its bf16 operands small where one key carries a
+ *   row's weight; any finite out gives the derivative of the forward, the forward's own out the
+ *   smallest rounding error.
  *   dq [batch][q_heads][L][d]; dk, dv (dk_enc, dv_enc, dk_dec, dv_dec) [batch][kv_heads][L][d],
- *   bf16, every element written (no accumulation into them).
+ *   bf16, every element written (no accumulation into them, no atomics: two calls with the same
+ *   inputs give the same bits).
  *   workspace: device memory of at least e2d2_attn_train_backward_workspace(dims, L) bytes
- *   (batch * q_heads * L floats; the query returns 0 for invalid dims or L <= 0 and needs no
- *   GPU), 16-byte aligned, contents ignored (holds D_i between the two launches of the call);
- *   calls that may run at the same time (different streams) need different workspaces.
- *   Launches two kernels on `stream`: dq with D_i, then dk/dv.  Errors as for the forward
- *   calls; a NULL lse is E2D2_ERR_INVALID_ARG; a small workspace is E2D2_ERR_WORKSPACE.
+ *   (2 * batch * q_heads * ceil(L/128)*128 floats; the query returns 0 for invalid dims or
+ *   L <= 0 and needs no GPU), 16-byte aligned, contents ignored (holds D_i and the scaled lse
+ *   between the two launches of the call); calls that may run at the same time (different
+ *   streams) need different workspaces.
+ *   Launches two kernels on `stream`: dq with D_i (query rows on the tensor-memory lanes),
+ *   then dk/dv (keys on the lanes).  Errors as for the forward calls; a NULL out or lse is
+ *   E2D2_ERR_INVALID_ARG; a small workspace is E2D2_ERR_WORKSPACE.
  */
 E2D2_API size_t e2d2_attn_train_backward_workspace(e2d2_dims dims, int L);
 
-E2D2_API e2d2_status e2d2_attn_encoder_backward(const void* q, const void* k, const void* v, const float* lse,
-                                                const void* dout, void* dq, void* dk, void* dv, e2d2_dims dims,
-                                                int L, int S, void* workspace, size_t ws_bytes,
+E2D2_API e2d2_status e2d2_attn_encoder_backward(const void* q, const void* k, const void* v, const void* out,
+                                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                                e2d2_dims dims, int L, int S, void* workspace, size_t ws_bytes,
                                                 cudaStream_t stream);
 
 E2D2_API e2d2_status e2d2_attn_decoder_train_backward(const void* q_dec, const void* k_enc, const void* v_enc,
-                                                      const void* k_dec, const void* v_dec, const float* lse,
-                                                      const void* dout, void* dq, void* dk_enc, void* dv_enc,
-                                                      void* dk_dec, void* dv_dec, e2d2_dims dims, int L, int S,
-                                                      void* workspace, size_t ws_bytes, cudaStream_t stream);
+                                                      const void* k_dec, const void* v_dec, const void* out,
+                                                      const float* lse, const void* dout, void* dq, void* dk_enc,
+                                                      void* dv_enc, void* dk_dec, void* dv_dec, e2d2_dims dims,
+                                                      int L, int S, void* workspace, size_t ws_bytes,
+                                                      cudaStream_t stream);
 
 /*
  * Bytes of scratch workspace that e2d2_attn_decoder_sample needs for these dims and block

@@ -61,13 +61,14 @@ class Oracle:
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_num_threads.restype = None
-        for name in ("oracle_mask_encoder", "oracle_mask_decoder"):
+        for name in ("oracle_mask_encoder", "oracle_mask_decoder", "oracle_mask_bd3lm"):
             getattr(lib, name).argtypes = [ctypes.c_int, ctypes.c_int, _u8p]
         lib.oracle_mask_sample.argtypes = [ctypes.c_int, ctypes.c_int, _u8p]
         ii = ctypes.c_int
         lib.oracle_encoder.argtypes = [_f32p, _f32p, _f32p, ii, ii, ii, ii, ii, ii,
                                        ctypes.c_double, _f64p, _f64p]
         lib.oracle_decoder_train.argtypes = [_f32p] * 5 + [ii] * 6 + [ctypes.c_double, _f64p, _f64p]
+        lib.oracle_bd3lm_train.argtypes = [_f32p] * 3 + [ii] * 6 + [ctypes.c_double, _f64p, _f64p]
         lib.oracle_decoder_sample.argtypes = [_f32p, _f32p, _f32p, ii, ii, _f32p, _f32p,
                                               ii, ii, ii, ii, ii, ctypes.c_double, _f64p, _f64p]
         lib.oracle_decoder_sample_ragged.argtypes = [_f32p, _f32p, _f32p, ii, ctypes.POINTER(ctypes.c_int),
@@ -76,7 +77,7 @@ class Oracle:
         lib.oracle_kv_append.argtypes = [_u16p, _u16p, ii, ii, _u16p, _u16p, ii, ii, ii, ii]
         lib.oracle_encoder_backward.argtypes = [_f32p] * 4 + [ii] * 6 + [ctypes.c_double] + [_f64p] * 3
         lib.oracle_decoder_train_backward.argtypes = [_f32p] * 6 + [ii] * 6 + [ctypes.c_double] + [_f64p] * 5
-        for name in ("oracle_encoder", "oracle_decoder_train", "oracle_decoder_sample",
+        for name in ("oracle_encoder", "oracle_decoder_train", "oracle_bd3lm_train", "oracle_decoder_sample",
                      "oracle_kv_append", "oracle_encoder_backward", "oracle_decoder_train_backward",
                      "oracle_decoder_sample_ragged"):
             getattr(lib, name).restype = ctypes.c_int
@@ -103,6 +104,12 @@ class Oracle:
     def mask_decoder(self, L: int, S: int) -> np.ndarray:
         m = np.zeros((L, 2 * L), dtype=np.uint8)
         self.lib.oracle_mask_decoder(L, S, m.ctypes.data_as(_u8p))
+        return m.astype(bool)
+
+    def mask_bd3lm(self, L: int, S: int) -> np.ndarray:
+        """BD3LM's [2L, 2L] training mask (noised positions first, then clean)."""
+        m = np.zeros((2 * L, 2 * L), dtype=np.uint8)
+        self.lib.oracle_mask_bd3lm(L, S, m.ctypes.data_as(_u8p))
         return m.astype(bool)
 
     def mask_sample(self, S: int, P: int) -> np.ndarray:
@@ -144,6 +151,23 @@ class Oracle:
         return out, lse
 
     # ---- backward of the train calls ----------------------------------------------
+    def bd3lm_train(self, q, k, v, S: int, scale: float = 0.0):
+        """BD3LM's attention over 2L tokens (noised copy first, then clean): q [B,Hq,2L,d],
+        k/v [B,Hkv,2L,d] -> (out [B,Hq,2L,d] f64, lse [B,Hq,2L] f64)."""
+        B, Hq, W, d = q.shape
+        Hkv = k.shape[1]
+        assert W % 2 == 0 and k.shape == (B, Hkv, W, d) and v.shape == k.shape
+        q, qp = self._f32(q)
+        k, kp = self._f32(k)
+        v, vp = self._f32(v)
+        out = np.zeros((B, Hq, W, d), dtype=np.float64)
+        lse = np.zeros((B, Hq, W), dtype=np.float64)
+        rc = self.lib.oracle_bd3lm_train(qp, kp, vp, B, Hq, Hkv, W // 2, S, d, float(scale),
+                                         out.ctypes.data_as(_f64p), lse.ctypes.data_as(_f64p))
+        if rc:
+            raise RuntimeError(f"oracle_bd3lm_train failed ({rc})")
+        return out, lse
+
     def encoder_backward(self, q, k, v, dout, S: int, scale: float = 0.0):
         """Gradients of sum(dout * encoder(q, k, v)) -> (dq [B,Hq,L,d], dk, dv [B,Hkv,L,d]), fp64."""
         B, Hq, L, d = q.shape

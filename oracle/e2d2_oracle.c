@@ -207,6 +207,59 @@ int oracle_decoder_train(const float* q, const float* k_enc, const float* v_enc,
     return rc ? -1 : 0;
 }
 
+/* BD3LM's training attention over 2L tokens, the comparison point of [E2D2 notes, sec. 1 and 4]:
+ * a decoder-only block diffusion model whose training forward takes the noised and the clean copy
+ * of the sequence together (2L tokens; attention cost 4ND(L^2 + LS) in the FLOPs table).
+ * Positions 0..L-1 hold the noised copy, L..2L-1 the clean copy.  The pages give the cost, not the
+ * mask; the reading taken: a noised token sees the noised tokens of its own block and the clean
+ * tokens of the blocks strictly before its own, a clean token the clean tokens of its own and
+ * earlier blocks; no clean token sees a noised one.  mask: [2L][2L]. */
+void oracle_mask_bd3lm(int L, int S, uint8_t* mask) {
+    const size_t W = (size_t)2 * L;
+    for (int i = 0; i < 2 * L; ++i) {
+        const int noised_row = i < L;
+        const int bi = block_of(noised_row ? i : i - L, S);
+        for (int j = 0; j < 2 * L; ++j) {
+            const int noised_col = j < L;
+            const int bj = block_of(noised_col ? j : j - L, S);
+            uint8_t a;
+            if (noised_row) a = noised_col ? (bj == bi) : (bj < bi);
+            else a = noised_col ? 0 : (bj <= bi);
+            mask[(size_t)i * W + j] = a;
+        }
+    }
+}
+
+/* q, k, v: [B][H][2L][d] (noised rows first); out [B][Hq][2L][d]; lse [B][Hq][2L]. */
+int oracle_bd3lm_train(const float* q, const float* k, const float* v, int B, int Hq, int Hkv, int L, int S,
+                       int d, double scale, double* out, double* lse) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L < 0 || S <= 0 || d <= 0) return -3;
+    const int G = Hq / Hkv;
+    scale = resolve_scale(scale, d);
+    const size_t W = (size_t)2 * L;
+    uint8_t* mask = (uint8_t*)malloc(W * W + 1);
+    if (!mask) return -2;
+    oracle_mask_bd3lm(L, S, mask);
+    int rc = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : rc)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < Hq; ++h) {
+            const int g = h / G;
+            double* kd = (double*)malloc(sizeof(double) * (W * d + 1));
+            double* vd = (double*)malloc(sizeof(double) * (W * d + 1));
+            if (!kd || !vd) { rc |= 2; free(kd); free(vd); continue; }
+            rows_to_double(k + ((size_t)b * Hkv + g) * W * d, (int)W, d, kd);
+            rows_to_double(v + ((size_t)b * Hkv + g) * W * d, (int)W, d, vd);
+            const size_t qo = ((size_t)b * Hq + h) * W;
+            if (attend(q + qo * d, kd, vd, mask, (int)W, (int)W, d, scale, out + qo * d, lse + qo)) rc |= 1;
+            free(kd);
+            free(vd);
+        }
+    }
+    free(mask);
+    return rc ? -1 : 0;
+}
+
 /* Decoder sampling step ([E2D2 notes, sec. 3]): the S noised queries of the current block
  * attend to the cached clean prefix (first P rows of the cache) and to their own block.
  * q: [B][Hq][S][d]; k_cache, v_cache: [B][Hkv][capacity][d]; k_blk, v_blk: [B][Hkv][S][d]. */

@@ -373,6 +373,49 @@ def pin_bd3lm_vectorized_mask(orc):
 
 
 # ---------------------------------------------------------------------------------------
+# 13b. BD3LM's attention over its 2L training tokens as its own oracle function (the comparison
+#      point of the FLOPs table): (a) pair count L^2 + LS, the table's 4ND(L^2+LS) per layer over
+#      4D; (b) the mask equals one built here from numpy block ids; (c) the output equals torch's
+#      SDPA in fp64 on that mask (GQA through repeated kv heads); (d) the noised rows equal the
+#      decoder-train call and the clean rows the encoder call on the same tensors (two definitions
+#      that must agree); (e) S = L: every row attends bidirectionally within its own copy.
+# ---------------------------------------------------------------------------------------
+def _bd3lm_mask(L, S):
+    blk = np.arange(L) // S
+    return np.block([[blk[:, None] == blk[None, :], blk[None, :] < blk[:, None]],
+                     [np.zeros((L, L), dtype=bool), blk[None, :] <= blk[:, None]]])
+
+
+def pin_bd3lm_train(orc):
+    for L, S in ((8, 1), (8, 2), (12, 3), (16, 4), (64, 8), (48, 16), (32, 32)):
+        m = orc.mask_bd3lm(L, S)
+        assert int(m.sum()) == L * L + L * S, (L, S)
+        assert (m == _bd3lm_mask(L, S)).all(), (L, S)
+    B, Hq, Hkv, L, S, d, scale = 2, 4, 2, 20, 5, 8, 0.4
+    G = Hq // Hkv
+    qn, qc = (_rand((B, Hq, L, d), 1200 + t) for t in range(2))
+    kn, vn, kc, vc = (_rand((B, Hkv, L, d), 1202 + t) for t in range(4))
+    q2, k2, v2 = (np.concatenate(x, axis=2) for x in ((qn, qc), (kn, kc), (vn, vc)))
+    out, lse = orc.bd3lm_train(q2, k2, v2, S, scale=scale)
+    m = _bd3lm_mask(L, S)
+    kr, vr = np.repeat(k2, G, axis=1), np.repeat(v2, G, axis=1)
+    np.testing.assert_allclose(out, _sdpa(q2, kr, vr, scale, mask=m), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, _torch_lse(q2, kr, scale, np.broadcast_to(m, lse.shape + (2 * L,))),
+                               rtol=0, atol=1e-12)
+    on, ln = orc.decoder_train(qn, kc, vc, kn, vn, S=S, scale=scale)
+    oc, lc = orc.encoder(qc, kc, vc, S=S, scale=scale)
+    np.testing.assert_allclose(out[:, :, :L], on, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(out[:, :, L:], oc, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[:, :, :L], ln, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[:, :, L:], lc, rtol=0, atol=1e-13)
+    out, _ = orc.bd3lm_train(q2, k2, v2, L, scale=scale)
+    np.testing.assert_allclose(out[:, :, :L], _sdpa(qn, np.repeat(kn, G, 1), np.repeat(vn, G, 1), scale),
+                               rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out[:, :, L:], _sdpa(qc, np.repeat(kc, G, 1), np.repeat(vc, G, 1), scale),
+                               rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
 # 14. Backward of the train calls ([E2D2 notes, sec. 4]: one encoder and one decoder pass, forward
 #     and backward).  (a) torch autograd in fp64 through SDPA on masks built here from the block
 #     rule (GQA through repeated kv heads, whose gradients autograd sums; a short last block);
@@ -482,5 +525,5 @@ ALL_PINS = [pin_pair_count, pin_golden_pairs, pin_block_size_one_is_causal,
             pin_block_size_L_is_bidirectional, pin_masked_against_torch, pin_brute_force,
             pin_zero_keys_closed_form, pin_constant_values, pin_gqa_is_repeated_heads,
             pin_sample_is_train_slice, pin_append_is_concatenation, pin_short_last_block,
-            pin_bd3lm_vectorized_mask, pin_backward_against_autograd, pin_backward_finite_differences,
-            pin_ragged_prefix_against_torch]
+            pin_bd3lm_vectorized_mask, pin_bd3lm_train, pin_backward_against_autograd,
+            pin_backward_finite_differences, pin_ragged_prefix_against_torch]

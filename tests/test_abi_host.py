@@ -82,8 +82,9 @@ def test_encoder_block_step_argument_errors(lib):
 
 
 def test_train_backward_workspace_query_needs_no_gpu(lib):
-    # one float (D_i = dout_i . out_i) per query row
-    assert lib.e2d2_attn_train_backward_workspace(DIMS, 64) == 2 * 4 * 64 * 4
+    # two floats (D_i and the scaled lse) per query row, rows padded to a multiple of 128
+    assert lib.e2d2_attn_train_backward_workspace(DIMS, 64) == 2 * 2 * 4 * 128 * 4
+    assert lib.e2d2_attn_train_backward_workspace(DIMS, 129) == 2 * 2 * 4 * 256 * 4
     assert lib.e2d2_attn_train_backward_workspace(_lib.Dims(2, 4, 2, 96, 0.0), 64) == 0
     assert lib.e2d2_attn_train_backward_workspace(DIMS, 0) == 0
 
@@ -91,31 +92,34 @@ def test_train_backward_workspace_query_needs_no_gpu(lib):
 def test_encoder_backward_argument_errors(lib):
     f = lib.e2d2_attn_encoder_backward
     ws = lib.e2d2_attn_train_backward_workspace(DIMS, 64)
-    # (q, k, v, lse, dout, dq, dk, dv, dims, L, S, workspace, ws_bytes, stream)
-    a = [P16] * 8
-    assert f(*a[:3], None, *a[4:], DIMS, 64, 8, P16, ws, None) == 1                 # lse is required
-    assert f(*a[:7], None, DIMS, 64, 8, P16, ws, None) == 1                         # null dv
+    # (q, k, v, out, lse, dout, dq, dk, dv, dims, L, S, workspace, ws_bytes, stream)
+    a = [P16] * 9
+    assert f(*a[:4], None, *a[5:], DIMS, 64, 8, P16, ws, None) == 1                 # lse is required
+    assert f(*a[:3], None, *a[4:], DIMS, 64, 8, P16, ws, None) == 1                 # out is required
+    assert f(*a[:8], None, DIMS, 64, 8, P16, ws, None) == 1                         # null dv
     assert f(*a, DIMS, 64, 8, P16, ws - 1, None) == 6                               # small workspace
     assert f(*a, DIMS, 64, 8, None, ws, None) == 6                                  # no workspace
     assert f(P16 + 8, *a[1:], DIMS, 64, 8, P16, ws, None) == 4                      # misaligned q
-    assert f(*a[:3], P16 + 2, *a[4:], DIMS, 64, 8, P16, ws, None) == 4              # misaligned lse
+    assert f(*a[:3], P16 + 8, *a[4:], DIMS, 64, 8, P16, ws, None) == 4              # misaligned out
+    assert f(*a[:4], P16 + 2, *a[5:], DIMS, 64, 8, P16, ws, None) == 4              # misaligned lse
     assert f(*a, DIMS, 64, 8, P16 + 4, ws, None) == 4                               # misaligned workspace
     assert f(*a, DIMS, 64, 0, P16, ws, None) == 1                                   # S = 0
     assert f(*a, _lib.Dims(2, 4, 2, 96, 0.0), 64, 8, P16, ws, None) == 2            # head_dim
     assert f(*a, _lib.Dims(2, 4, 3, 64, 0.0), 64, 8, P16, ws, None) == 1            # GQA ratio
     # a short last block passes the shape checks (stopped here by the misaligned lse)
-    assert f(*a[:3], P16 + 2, *a[4:], DIMS, 60, 8, P16, ws, None) == 4
+    assert f(*a[:4], P16 + 2, *a[5:], DIMS, 60, 8, P16, ws, None) == 4
 
 
 def test_decoder_train_backward_argument_errors(lib):
     f = lib.e2d2_attn_decoder_train_backward
     ws = lib.e2d2_attn_train_backward_workspace(DIMS, 64)
-    # (q, k_enc, v_enc, k_dec, v_dec, lse, dout, dq, dk_enc, dv_enc, dk_dec, dv_dec, dims, L, S,
+    # (q, k_enc, v_enc, k_dec, v_dec, out, lse, dout, dq, dk_enc, dv_enc, dk_dec, dv_dec, dims, L, S,
     #  workspace, ws_bytes, stream)
-    a = [P16] * 12
-    assert f(*a[:11], None, DIMS, 64, 8, P16, ws, None) == 1                        # null dv_dec
-    assert f(*a[:5], None, *a[6:], DIMS, 64, 8, P16, ws, None) == 1                 # lse is required
-    assert f(*a[:10], P16 + 8, a[11], DIMS, 64, 8, P16, ws, None) == 4              # misaligned dk_dec
+    a = [P16] * 13
+    assert f(*a[:12], None, DIMS, 64, 8, P16, ws, None) == 1                        # null dv_dec
+    assert f(*a[:6], None, *a[7:], DIMS, 64, 8, P16, ws, None) == 1                 # lse is required
+    assert f(*a[:5], None, *a[6:], DIMS, 64, 8, P16, ws, None) == 1                 # out is required
+    assert f(*a[:11], P16 + 8, a[12], DIMS, 64, 8, P16, ws, None) == 4              # misaligned dk_dec
     assert f(*a, DIMS, 64, 8, P16, ws - 4, None) == 6
     assert f(*a, DIMS, -1, 8, P16, ws, None) == 1
 

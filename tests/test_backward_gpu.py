@@ -49,8 +49,8 @@ def run_encoder_backward(orc, B, Hq, Hkv, L, S, d, seed0=700):
     q, ks = H.train_inputs(B, Hq, Hkv, L, d, 1.0, seed0)
     (k, kt), (v, vt) = ks[0], ks[1]
     g = H.gen((B, Hq, L, d), seed0 + 9)
-    _, lse = attn.encoder_blockcausal(q[1], kt, vt, S)
-    dq, dk, dv = attn.encoder_backward(q[1], kt, vt, lse, g[1], S)
+    o, lse = attn.encoder_blockcausal(q[1], kt, vt, S)
+    dq, dk, dv = attn.encoder_backward(q[1], kt, vt, o, lse, g[1], S)
     torch.cuda.synchronize()
     ref = orc.encoder_backward(q[0].f32, k.f32, v.f32, g[0].f32, S)
     tag = f"encoder bwd B{B} Hq{Hq} Hkv{Hkv} L{L} S{S} d{d}"
@@ -63,8 +63,8 @@ def run_decoder_backward(orc, B, Hq, Hkv, L, S, d, seed0=800):
     q, ks = H.train_inputs(B, Hq, Hkv, L, d, 1.0, seed0)
     (ke, ket), (ve, vet), (kd, kdt), (vd, vdt) = ks
     g = H.gen((B, Hq, L, d), seed0 + 9)
-    _, lse = attn.decoder_train(q[1], ket, vet, kdt, vdt, S)
-    grads = attn.decoder_train_backward(q[1], ket, vet, kdt, vdt, lse, g[1], S)
+    o, lse = attn.decoder_train(q[1], ket, vet, kdt, vdt, S)
+    grads = attn.decoder_train_backward(q[1], ket, vet, kdt, vdt, o, lse, g[1], S)
     torch.cuda.synchronize()
     ref = orc.decoder_train_backward(q[0].f32, ke.f32, ve.f32, kd.f32, vd.f32, g[0].f32, S)
     tag = f"decoder bwd B{B} Hq{Hq} Hkv{Hkv} L{L} S{S} d{d}"
@@ -91,10 +91,11 @@ def test_backward_deterministic_and_fully_written(oracle):
     q, ks = H.train_inputs(B, Hq, Hkv, L, d, 1.0, 900)
     g = H.gen((B, Hq, L, d), 909)
     ket, vet, kdt, vdt = (t[1] for t in ks)
-    _, lse = attn.decoder_train(q[1], ket, vet, kdt, vdt, S)
-    first = attn.decoder_train_backward(q[1], ket, vet, kdt, vdt, lse, g[1], S)
-    ws = torch.full((B * Hq * L,), float("nan"), dtype=torch.float32, device="cuda")
-    second = attn.decoder_train_backward(q[1], ket, vet, kdt, vdt, lse, g[1], S, workspace=ws)
+    o, lse = attn.decoder_train(q[1], ket, vet, kdt, vdt, S)
+    first = attn.decoder_train_backward(q[1], ket, vet, kdt, vdt, o, lse, g[1], S)
+    n_ws = attn.train_backward_workspace_bytes(B, Hq, Hkv, d, L) // 4
+    ws = torch.full((n_ws,), float("nan"), dtype=torch.float32, device="cuda")
+    second = attn.decoder_train_backward(q[1], ket, vet, kdt, vdt, o, lse, g[1], S, workspace=ws)
     torch.cuda.synchronize()
     for a, b in zip(first, second):
         assert torch.isfinite(a.float()).all()
@@ -115,10 +116,10 @@ def test_train_pass_backward_full_size_sampled_heads(oracle):
     ke = H.gen((B, Hq, L, d), synth.seed_for(2, 0, "k_enc"), w.sigma)
     ve = H.gen((B, Hq, L, d), synth.seed_for(2, 0, "v_enc"), w.sigma)
     g = H.gen((B, Hq, L, d), synth.seed_for(2, 0, "dout"))
-    _, lse_e = attn.encoder_blockcausal(q[1], k[1], v[1], S)
-    enc = attn.encoder_backward(q[1], k[1], v[1], lse_e, g[1], S)
-    _, lse_d = attn.decoder_train(q[1], ke[1], ve[1], k[1], v[1], S)
-    dec = attn.decoder_train_backward(q[1], ke[1], ve[1], k[1], v[1], lse_d, g[1], S)
+    o_e, lse_e = attn.encoder_blockcausal(q[1], k[1], v[1], S)
+    enc = attn.encoder_backward(q[1], k[1], v[1], o_e, lse_e, g[1], S)
+    o_d, lse_d = attn.decoder_train(q[1], ke[1], ve[1], k[1], v[1], S)
+    dec = attn.decoder_train_backward(q[1], ke[1], ve[1], k[1], v[1], o_d, lse_d, g[1], S)
     torch.cuda.synchronize()
     for b, h in ((0, 0), (5, 11)):
         sl = (slice(b, b + 1), slice(h, h + 1))

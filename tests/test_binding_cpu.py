@@ -19,9 +19,11 @@ CALLS = [
                                                              bf16(B, Hkv, L, d), S)),
     ("decoder_train", lambda: attn.decoder_train(bf16(B, Hq, L, d), *(bf16(B, Hkv, L, d) for _ in range(4)), S)),
     ("encoder_backward", lambda: attn.encoder_backward(bf16(B, Hq, L, d), bf16(B, Hkv, L, d), bf16(B, Hkv, L, d),
-                                                       torch.zeros(B, Hq, L), bf16(B, Hq, L, d), S)),
+                                                       bf16(B, Hq, L, d), torch.zeros(B, Hq, L), bf16(B, Hq, L, d),
+                                                       S)),
     ("decoder_train_backward", lambda: attn.decoder_train_backward(
-        bf16(B, Hq, L, d), *(bf16(B, Hkv, L, d) for _ in range(4)), torch.zeros(B, Hq, L), bf16(B, Hq, L, d), S)),
+        bf16(B, Hq, L, d), *(bf16(B, Hkv, L, d) for _ in range(4)), bf16(B, Hq, L, d), torch.zeros(B, Hq, L),
+        bf16(B, Hq, L, d), S)),
     ("decoder_sample", lambda: attn.decoder_sample(bf16(B, Hq, S, d), bf16(B, Hkv, 64, d), bf16(B, Hkv, 64, d), 16,
                                                    bf16(B, Hkv, S, d), bf16(B, Hkv, S, d))),
     ("encoder_block_step", lambda: attn.encoder_block_step(bf16(B, Hq, S, d), bf16(B, Hkv, 64, d),

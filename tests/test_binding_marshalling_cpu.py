@@ -113,10 +113,12 @@ def test_decoder_train(rec):
 
 def test_encoder_backward(rec):
     q, k, v, g = bf16(B, Hq, L, d), bf16(B, Hkv, L, d), bf16(B, Hkv, L, d), bf16(B, Hq, L, d)
+    o = bf16(B, Hq, L, d)
     lse = torch.zeros(B, Hq, L)
-    dq, dk, dv = attn.encoder_backward(q, k, v, lse, g, S, scale=0.25)
+    dq, dk, dv = attn.encoder_backward(q, k, v, o, lse, g, S, scale=0.25)
     a = rec.call("e2d2_attn_encoder_backward")
-    assert (a["q"], a["k"], a["v"], a["lse"], a["dout"]) == tuple(t.data_ptr() for t in (q, k, v, lse, g))
+    assert (a["q"], a["k"], a["v"], a["out"], a["lse"], a["dout"]) == tuple(
+        t.data_ptr() for t in (q, k, v, o, lse, g))
     assert (a["dq"], a["dk"], a["dv"]) == (dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
     assert dq.shape == q.shape and dk.shape == k.shape and dv.shape == v.shape
     check_dims(a["dims"], B, Hq, Hkv, d, 0.25)
@@ -128,14 +130,14 @@ def test_encoder_backward(rec):
 
 
 def test_decoder_train_backward(rec):
-    q, g = bf16(B, Hq, L, d), bf16(B, Hq, L, d)
+    q, g, o = bf16(B, Hq, L, d), bf16(B, Hq, L, d), bf16(B, Hq, L, d)
     ke, ve, kd, vd = (bf16(B, Hkv, L, d) for _ in range(4))
     lse = torch.zeros(B, Hq, L)
     ws = torch.zeros(B * Hq * L)
-    dq, dke, dve, dkd, dvd = attn.decoder_train_backward(q, ke, ve, kd, vd, lse, g, S, workspace=ws)
+    dq, dke, dve, dkd, dvd = attn.decoder_train_backward(q, ke, ve, kd, vd, o, lse, g, S, workspace=ws)
     a = rec.call("e2d2_attn_decoder_train_backward")
-    assert (a["q_dec"], a["k_enc"], a["v_enc"], a["k_dec"], a["v_dec"], a["lse"], a["dout"]) == tuple(
-        t.data_ptr() for t in (q, ke, ve, kd, vd, lse, g))
+    assert (a["q_dec"], a["k_enc"], a["v_enc"], a["k_dec"], a["v_dec"], a["out"], a["lse"], a["dout"]) == tuple(
+        t.data_ptr() for t in (q, ke, ve, kd, vd, o, lse, g))
     assert (a["dq"], a["dk_enc"], a["dv_enc"], a["dk_dec"], a["dv_dec"]) == tuple(
         t.data_ptr() for t in (dq, dke, dve, dkd, dvd))
     assert a["workspace"] == ws.data_ptr() and a["ws_bytes"] == ws.numel() * 4

@@ -44,6 +44,12 @@ MUTANTS = [
     ("append-off-by-one", "capacity + P + r) * d;", "capacity + P + r + 1) * d;"),
     ("append-swaps-k-and-v", "memcpy(v_cache + dst, v_new + src, sizeof(uint16_t) * d);",
      "memcpy(v_cache + dst, k_new + src, sizeof(uint16_t) * d);"),
+    # BD3LM's 2L-token attention
+    ("bd3lm-noised-sees-own-clean-block", "if (noised_row) a = noised_col ? (bj == bi) : (bj < bi);",
+     "if (noised_row) a = noised_col ? (bj == bi) : (bj <= bi);"),
+    ("bd3lm-clean-sees-noised", "else a = noised_col ? 0 : (bj <= bi);", "else a = noised_col ? (bj < bi) : (bj <= bi);"),
+    ("bd3lm-clean-rows-read-noised-keys", "rows_to_double(k + ((size_t)b * Hkv + g) * W * d, (int)W, d, kd);",
+     "rows_to_double(k + ((size_t)b * Hkv + g) * W * d, (int)W / 2, d, kd);\n            rows_to_double(k + ((size_t)b * Hkv + g) * W * d, (int)W / 2, d, kd + (size_t)L * d);"),
     # backward of the train calls
     ("bwd-drops-row-term", "const double ds = exp(s[j] - lse) * (dp[j] - dsum);",
      "const double ds = exp(s[j] - lse) * dp[j];"),

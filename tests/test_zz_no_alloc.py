@@ -4,8 +4,9 @@ It serves callers that cannot allocate device memory -- an engine that hands all
 own pool and gives plugins no allocator, or a hot path that may not call cudaMalloc because it
 can synchronise the device.  Its split-KV scratch is a fixed device array inside the library.
 These tests call it through the C ABI and check it against the workspace-taking entry point
-(e2d2_attn_decoder_sample) within the parity tolerances, on two calls in a row (the array keeps
-the previous call's contents), and check that a shape too large for the array is refused.
+(e2d2_attn_decoder_sample) within the parity tolerances, on consecutive calls (the array keeps
+the previous call's contents) that reach both sampling kernels and split their work over
+different CTA counts, and check that a shape too large for the array is refused.
 This file is collected last on purpose."""
 import ctypes
 
@@ -31,10 +32,21 @@ def _noalloc(lib, q, kc, vc, P, kb, vb):
     return out, lse
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
+# Consecutive calls with different work plans: the keys-on-lanes kernel (head_dim 128, G*S <= 64),
+# then the generic kernel (head_dim 64) with its units split over a different number of CTAs, so
+# the second and third calls find the array holding the previous call's partials and tickets.
+CALLS = [(4, 16, 8, 16, 700, 800, 128, 4100),
+         (2, 16, 4, 16, 1000, 1040, 64, 4300),
+         (2, 32, 8, 16, 2048, 2064, 128, 4200)]
+
+
+def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
     lib = _lib.load()
-    for call, (B, Hq, Hkv, S, P, cap, d, seed) in enumerate([(4, 16, 8, 16, 700, 800, 128, 4100),
-                                                             (2, 32, 8, 16, 2048, 2064, 128, 4200)]):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plans = [attn.sample_plan(B, Hq, Hkv, d, S, P, sms) for (B, Hq, Hkv, S, P, cap, d, _) in CALLS]
+    assert plans[1]["kernel"] == 0 and plans[1]["split_units"] > 0, plans[1]
+    assert plans[0]["split_ctas"] != plans[1]["split_ctas"], plans
+    for call, (B, Hq, Hkv, S, P, cap, d, seed) in enumerate(CALLS):
         q, kc, vc, kb, vb = H.sample_inputs(B, Hq, Hkv, S, cap, d, 1.0, seed)
         ref_o, ref_l = attn.decoder_sample(q[1], kc[1], vc[1], P, kb[1], vb[1])
         out, lse = _noalloc(lib, q[1], kc[1], vc[1], P, kb[1], vb[1])
