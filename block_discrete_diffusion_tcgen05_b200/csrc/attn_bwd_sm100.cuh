@@ -35,11 +35,15 @@
 // is empty; queries past L also carry lse = +inf in the workspace (p = 0).
 //
 // CTA = 12 warps: warp 0 issues the TMA loads (row tiles once per item, column sub-tiles through
-// a ring), warp 1 owns tensor memory and issues tcgen05.mma, warps 2..3 are idle, warps 4..7
-// and 8..11 are two softmax warpgroups that take alternate sub-tiles.  Tensor memory holds two
-// (S, dP) sets of 64 + 64 columns, so while one warpgroup turns set 0 into (p, u) the tensor core
-// computes the products of set 1 and the accumulations of the other; the two accumulators
-// (Y, X or dV, dK) take 2 x head_dim columns, double-buffered across items at head_dim <= 64.
+// a ring), warp 1 owns tensor memory and issues the S / dP products, warp 2 issues the
+// accumulations (two issuing threads, so neither stream waits behind the other), warp 3 fetches
+// the per-row constants of the next item (rows-Q), warps 4..7 and 8..11 are two softmax
+// warpgroups that take alternate sub-tiles and write the gradient tiles (through shared memory
+// and one TMA store per tile, so the accumulator is free again at once).  Tensor memory holds three
+// (S, dP) sets of 64 + 64 columns (two at head_dim 128), used round robin: while the warpgroups
+// turn two sets into (p, u) the tensor core computes the products of the third and the
+// accumulations of the sets already done, so a warpgroup normally finds its next S ready.  The two
+// accumulators (Y, X or dV, dK) take the remaining 2 x head_dim columns.
 #pragma once
 
 #include <cstdint>
@@ -58,6 +62,8 @@ constexpr int kBwdCols = 64;   // columns of a sub-tile
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct alignas(64) BwdTcParams {
+    CUtensorMap tm_ga[2];  // gradient stores (128-row boxes): rows-Q: dq at [0]; rows-KV: dv of key source 0/1
+    CUtensorMap tm_gb[2];  // rows-KV: dk of key source 0/1
     CUtensorMap tm_r1[2];  // row operand 1 (128-row boxes): rows-Q: Q at [0]; rows-KV: K of key source 0/1
     CUtensorMap tm_r2[2];  // row operand 2: rows-Q: dO at [0]; rows-KV: V of key source 0/1
     CUtensorMap tm_c1[2];  // column operand 1 (64-row boxes): rows-Q: K of key source 0/1; rows-KV: Q at [0]
@@ -88,8 +94,12 @@ struct BwdCfg {
     static constexpr int COL_TILE = kBwdCols * D * 2;
     static constexpr int KSTEPS_PER_CHUNK = RB / 32;         // 16-element k steps per chunk
     static constexpr int RBUF = (D == 128) ? 1 : 2;          // row-tile buffers (items in flight)
-    static constexpr int NST = (D == 128) ? 4 : (D == 64 ? 6 : 8);  // column stages
-    static constexpr int NACC = (D == 128) ? 1 : 2;          // accumulator sets
+    static constexpr int NST = (D == 128) ? 2 : (D == 64 ? 6 : 8);  // column stages
+    // (S, dP) sets of 128 TMEM columns and accumulator sets of 2 D columns, within 512 columns.
+    // A third set lets the products of sub-tile n+2 run while sub-tile n's p is still consumed.
+    static constexpr int NSET = (D == 128) ? 2 : 3;
+    static constexpr int NACC = (D == 32) ? 2 : 1;
+    static_assert(NSET * 128 + NACC * 2 * D <= 512, "tensor memory budget");
 };
 
 template <int D>
@@ -99,10 +109,13 @@ struct BwdSmem {
     static constexpr int OFF_C = OFF_R + C::RBUF * 2 * C::ROW_TILE;        // [NST][2] column tiles
     static constexpr int OFF_LD = OFF_C + C::NST * 2 * C::COL_TILE;        // [NST][2][64] nl2, D
     static constexpr int OFF_X = OFF_LD + C::NST * 2 * kBwdCols * 4;       // [2][2][128] sum exchange
-    static constexpr int OFF_BAR = OFF_X + 2 * 2 * kBwdRows * 4;
-    // row_full[RBUF], row_empty[RBUF], col_full[NST], col_empty[NST], s_full[2], p_full[2],
-    // acc_full[NACC], acc_free[NACC], mma_drain, softmax_done
-    static constexpr int NBAR = 2 * C::RBUF + 2 * C::NST + 4 + 2 * C::NACC + 2;
+    static constexpr int OFF_ROWD = OFF_X + 2 * 2 * kBwdRows * 4;         // [2][2][128] rows-Q: c_i, -lse_i log2e
+    static constexpr int OFF_STG = ((OFF_ROWD + 2 * 2 * kBwdRows * 4 + 1023) / 1024) * 1024;  // [2] gradient tiles
+    static constexpr int OFF_BAR = OFF_STG + 2 * C::ROW_TILE;
+    // row_full[RBUF], row_empty[RBUF], col_full[NST], col_empty[NST], s_full[NSET], p_full[NSET],
+    // set_free[NSET], acc_full[NACC], acc_free[NACC], rowd_full[2], rowd_empty[2], mma_drain,
+    // acc_drain, softmax_done
+    static constexpr int NBAR = 2 * C::RBUF + 2 * C::NST + 3 * C::NSET + 2 * C::NACC + 4 + 3;
     static constexpr int OFF_MISC = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
@@ -347,7 +360,8 @@ template <int D, int SIDE>
 __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __grid_constant__ BwdTcParams p) {
     using C = BwdCfg<D>;
     using SM = BwdSmem<D>;
-    constexpr int NST = C::NST, RBUF = C::RBUF, NACC = C::NACC;
+    constexpr int NST = C::NST, RBUF = C::RBUF, NACC = C::NACC, NSET = C::NSET;
+    constexpr uint32_t ACC0 = NSET * 128;  // first accumulator column
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -360,15 +374,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
     uint64_t* col_full = row_empty + RBUF;                                                           \
     uint64_t* col_empty = col_full + NST;                                                            \
     uint64_t* s_full = col_empty + NST;                                                              \
-    uint64_t* p_full = s_full + 2;                                                                   \
-    uint64_t* acc_full = p_full + 2;                                                                 \
+    uint64_t* p_full = s_full + NSET;                                                                \
+    uint64_t* set_free = p_full + NSET;                                                              \
+    uint64_t* acc_full = set_free + NSET;                                                            \
     uint64_t* acc_free = acc_full + NACC;                                                            \
-    uint64_t* mma_drain = acc_free + NACC;                                                           \
-    uint64_t* softmax_done = mma_drain + 1;                                                          \
+    uint64_t* rowd_full = acc_free + NACC;                                                           \
+    uint64_t* rowd_empty = rowd_full + 2;                                                            \
+    uint64_t* mma_drain = rowd_empty + 2;                                                            \
+    uint64_t* acc_drain = mma_drain + 1;                                                             \
+    uint64_t* softmax_done = acc_drain + 1;                                                          \
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);                        \
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);             \
     (void)row_full; (void)row_empty; (void)col_full; (void)col_empty; (void)s_full; (void)p_full;    \
     (void)acc_full; (void)acc_free; (void)mma_drain; (void)softmax_done; (void)tmem_holder;          \
+    (void)set_free; (void)acc_drain; (void)rowd_full; (void)rowd_empty;                              \
     (void)abort_flag;
     uint32_t tmem_base;
     {
@@ -382,15 +401,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                 ptx::mbar_init(&col_full[i], 1);
                 ptx::mbar_init(&col_empty[i], 1);
             }
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < NSET; ++i) {
                 ptx::mbar_init(&s_full[i], 1);
                 ptx::mbar_init(&p_full[i], 128);
+                ptx::mbar_init(&set_free[i], 1);
             }
             for (int i = 0; i < NACC; ++i) {
                 ptx::mbar_init(&acc_full[i], 1);
                 ptx::mbar_init(&acc_free[i], kSoftmaxThreads);
             }
+            for (int i = 0; i < 2; ++i) {
+                ptx::mbar_init(&rowd_full[i], 32);
+                ptx::mbar_init(&rowd_empty[i], kSoftmaxThreads);
+            }
             ptx::mbar_init(mma_drain, 1);
+            ptx::mbar_init(acc_drain, 1);
             ptx::mbar_init(softmax_done, kSoftmaxThreads);
             *abort_flag = 0;
             ptx::fence_mbar_init();
@@ -482,45 +507,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             wait_bar_warp(&row_full[i % RBUF], (i / RBUF) & 1u, &no_abort, p.err);
     } else if (warp == 1) {
         ptx::setmaxnreg_dec<kRegsControl>();
-        // ------------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------------ product issuer
+        // S = R1 C1^T and dP = R2 C2^T of every sub-tile into its set, once the set's previous
+        // accumulation (sub-tile n - NSET, issued by warp 2) has read it.  Also owns tensor memory.
         const bool leader = ptx::elect_one();
-        const uint64_t kdesc = ptx::smem_desc(0, 16, 8 * C::RB, C::SWZ);              // K-major
-        const uint64_t mndesc = ptx::smem_desc(0, C::COL_CHUNK, 8 * C::RB, C::SWZ);   // MN-major
+        const uint64_t kdesc = ptx::smem_desc(0, 16, 8 * C::RB, C::SWZ);  // K-major
         constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(kBwdRows, kBwdCols, false);
-        constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(kBwdRows, D, true);
         BwdScheduler<SIDE> sched(p);
         BwdItem it;
         uint32_t n = 0, iw = 0;
-        // The accumulation of sub-tile n is issued after the products of sub-tile n+1, so the
-        // tensor core works on one set while a softmax warpgroup works on the other.
-        bool have = false;
-        uint32_t pv_n = 0, pv_iw = 0;
-        bool pv_first = false, pv_last = false;
-        auto issue_acc = [&]() -> bool {
-            const uint32_t set = pv_n & 1u, st = pv_n % NST, ab = pv_iw % NACC;
-            if (!wait_bar_warp(&p_full[set], (pv_n >> 1) & 1u, abort_flag, p.err)) return false;
-            if (pv_first && !wait_bar_warp(&acc_free[ab], ((pv_iw / NACC) & 1u) ^ 1u, abort_flag, p.err))
-                return false;
-            ptx::tc_fence_after();
-            if (leader) {
-                const uint32_t c1 = sC + (st * 2 + 0) * C::COL_TILE;
-                const uint32_t c2 = sC + (st * 2 + 1) * C::COL_TILE;
-                const uint32_t ba = (SIDE == kBwdRowsQ) ? c1 : c2;  // Y += p K  |  dV += p^T dO
-                const uint32_t bb = c1;                             // X += u K  |  dK += ds^T Q
-                const uint32_t acc = tmem_base + 256 + ab * 2 * D;
-                const uint32_t pset = tmem_base + set * 128;
-#pragma unroll
-                for (int ks = 0; ks < kBwdCols / 16; ++ks) {
-                    const uint32_t accum = (pv_first && ks == 0) ? 0u : 1u;
-                    ptx::mma_ts(acc, pset + 8 * ks, mndesc | ((ba + ks * 16 * C::RB) >> 4), idesc_o, accum);
-                    ptx::mma_ts(acc + D, pset + 64 + 8 * ks, mndesc | ((bb + ks * 16 * C::RB) >> 4), idesc_o, accum);
-                }
-                ptx::mma_commit(&col_empty[st]);
-                if (pv_last) ptx::mma_commit(&acc_full[ab]);
-            }
-            __syncwarp();
-            return true;
-        };
         bool ok = true;
         while (ok && sched.next(it)) {
             if (it.nsub == 0) continue;
@@ -529,9 +524,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             if (!ok) break;
             const uint32_t r1 = sR + (rb * 2 + 0) * C::ROW_TILE;
             const uint32_t r2 = sR + (rb * 2 + 1) * C::ROW_TILE;
-            for (int t = 0; t < it.nsub && ok; ++t) {
-                const uint32_t st = n % NST, set = n & 1u;
-                ok = wait_bar_warp(&col_full[st], (n / NST) & 1u, abort_flag, p.err);
+            for (int t = 0; t < it.nsub && ok; ++t, ++n) {
+                const uint32_t st = n % NST, set = n % NSET;
+                ok = wait_bar_warp(&col_full[st], (n / NST) & 1u, abort_flag, p.err) &&
+                     wait_bar_warp(&set_free[set], ((n / NSET) & 1u) ^ 1u, abort_flag, p.err);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 if (leader) {
@@ -550,28 +546,96 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                     if (t == it.nsub - 1) ptx::mma_commit(&row_empty[rb]);
                 }
                 __syncwarp();
-                if (have) ok = issue_acc();
-                have = true;
-                pv_n = n;
-                pv_iw = iw;
-                pv_first = (t == 0);
-                pv_last = (t == it.nsub - 1);
-                ++n;
             }
             ++iw;
         }
-        if (ok && have) ok = issue_acc();
-        // Drain: every MMA issued by this warp completes, and every softmax thread is done with
-        // tensor memory, before it is released.
+        // Drain: this warp's and warp 2's MMAs have completed and every softmax thread is done with
+        // tensor memory before it is released.
         if (leader) ptx::mma_commit(mma_drain);
         __syncwarp();
         volatile int no_abort = 0;
         wait_bar_warp(mma_drain, 0, &no_abort, p.err);
+        wait_bar_warp(acc_drain, 0, &no_abort, p.err);
         wait_bar_warp(softmax_done, 0, &no_abort, p.err);
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, kTmemCols);
-    } else if (warp < 4) {
+    } else if (warp == 2) {
         ptx::setmaxnreg_dec<kRegsControl>();
+        // ------------------------------------------------------------------ accumulation issuer
+        // Y += p C1, X += u C1 (rows-Q) or dV += p^T C2, dK += ds^T C1 (rows-KV) of every sub-tile,
+        // in order, once its softmax has written p and u into the set; then the set and the column
+        // stage are free.
+        const bool leader = ptx::elect_one();
+        const uint64_t mndesc = ptx::smem_desc(0, C::COL_CHUNK, 8 * C::RB, C::SWZ);  // MN-major
+        constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(kBwdRows, D, true);
+        BwdScheduler<SIDE> sched(p);
+        BwdItem it;
+        uint32_t n = 0, iw = 0;
+        bool ok = true;
+        while (ok && sched.next(it)) {
+            if (it.nsub == 0) continue;
+            const uint32_t ab = iw % NACC;
+            for (int t = 0; t < it.nsub && ok; ++t, ++n) {
+                const uint32_t set = n % NSET, st = n % NST;
+                ok = wait_bar_warp(&p_full[set], (n / NSET) & 1u, abort_flag, p.err) &&
+                     (t != 0 || wait_bar_warp(&acc_free[ab], ((iw / NACC) & 1u) ^ 1u, abort_flag, p.err));
+                if (!ok) break;
+                ptx::tc_fence_after();
+                if (leader) {
+                    const uint32_t c1 = sC + (st * 2 + 0) * C::COL_TILE;
+                    const uint32_t c2 = sC + (st * 2 + 1) * C::COL_TILE;
+                    const uint32_t ba = (SIDE == kBwdRowsQ) ? c1 : c2;
+                    const uint32_t acc = tmem_base + ACC0 + ab * 2 * D;
+                    const uint32_t pset = tmem_base + set * 128;
+#pragma unroll
+                    for (int ks = 0; ks < kBwdCols / 16; ++ks) {
+                        const uint32_t accum = (t == 0 && ks == 0) ? 0u : 1u;
+                        ptx::mma_ts(acc, pset + 8 * ks, mndesc | ((ba + ks * 16 * C::RB) >> 4), idesc_o, accum);
+                        ptx::mma_ts(acc + D, pset + 64 + 8 * ks, mndesc | ((c1 + ks * 16 * C::RB) >> 4), idesc_o,
+                                    accum);
+                    }
+                    ptx::mma_commit(&col_empty[st]);
+                    ptx::mma_commit(&set_free[set]);
+                    if (t == it.nsub - 1) ptx::mma_commit(&acc_full[ab]);
+                }
+                __syncwarp();
+            }
+            ++iw;
+        }
+        if (leader) ptx::mma_commit(acc_drain);  // the thread that issued this warp's MMAs
+        __syncwarp();
+    } else if (warp == 3) {
+        ptx::setmaxnreg_dec<kRegsControl>();
+        // ------------------------------------------------------------------ row data (rows-Q)
+        // c_i = dout_i.out_i and -lse_i log2(e) of the next item's 128 query rows into shared
+        // memory, ahead of the softmax warpgroups (their global-load latency is off the critical
+        // path); double-buffered by item.
+        if (SIDE == kBwdRowsQ) {
+            float* rowd = reinterpret_cast<float*>(smem + SM::OFF_ROWD);
+            BwdScheduler<SIDE> sched(p);
+            BwdItem it;
+            uint32_t iw = 0;
+            while (sched.next(it)) {
+                if (it.nsub == 0) continue;
+                const uint32_t par = iw & 1u;
+                wait_bar_warp(&rowd_empty[par], ((iw >> 1) & 1u) ^ 1u, abort_flag, p.err);
+#pragma unroll
+                for (int j = 0; j < kBwdRows / 32; ++j) {
+                    const int lr = j * 32 + lane;
+                    const int row = it.row0 + lr;
+                    float c = 0.f, nl = 0.f;
+                    if (row < p.L) {
+                        const size_t r = static_cast<size_t>(it.row_z) * p.L + row;
+                        c = row_dot_bf16<D>(p.dout + r * D, p.out + r * D);
+                        nl = -__ldg(p.lse + r) * kLog2e;
+                    }
+                    rowd[(par * 2 + 0) * kBwdRows + lr] = c;
+                    rowd[(par * 2 + 1) * kBwdRows + lr] = nl;
+                }
+                ptx::mbar_arrive(&rowd_full[par]);
+                ++iw;
+            }
+        }
     } else {
         ptx::setmaxnreg_inc<kRegsSoftmax>();
         // ------------------------------------------------------------------ softmax warpgroups
@@ -586,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
         float* xch = reinterpret_cast<float*>(smem + SM::OFF_X);  // [2][2][128]
         BwdScheduler<SIDE> sched(p);
         BwdItem it;
-        uint32_t n = 0, iw = 0, own = 0;
+        uint32_t n = 0, iw = 0;
         while (sched.next(it)) {
             const int row = it.row0 + lrow;
             const bool valid = row < p.L;
@@ -606,15 +670,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             bwd_interval<SIDE>(p, row, SIDE == kBwdRowsQ ? 0 : it.src, lo0, hi0);
             bwd_interval<SIDE>(p, row, 1, lo1, hi1);
             float nl2_row = 0.f, c_row = 0.f;
-            if (SIDE == kBwdRowsQ && valid) {
-                const size_t r = static_cast<size_t>(it.row_z) * p.L + row;
-                nl2_row = -__ldg(p.lse + r) * kLog2e;
-                c_row = row_dot_bf16<D>(p.dout + r * D, p.out + r * D);
+            if (SIDE == kBwdRowsQ) {
+                const uint32_t par = iw & 1u;
+                const float* rowd = reinterpret_cast<const float*>(smem + SM::OFF_ROWD);
+                wait_bar_warp(&rowd_full[par], (iw >> 1) & 1u, abort_flag, p.err);
+                c_row = rowd[(par * 2 + 0) * kBwdRows + lrow];
+                nl2_row = rowd[(par * 2 + 1) * kBwdRows + lrow];
+                ptx::mbar_arrive(&rowd_empty[par]);
             }
             float usum = 0.f;
             for (int t = 0; t < it.nsub; ++t, ++n) {
                 if (static_cast<int>(n & 1u) != w) continue;
-                wait_bar_warp(&s_full[w], own & 1u, abort_flag, p.err);
+                const uint32_t set = n % NSET;
+                wait_bar_warp(&s_full[set], (n / NSET) & 1u, abort_flag, p.err);
                 ptx::tc_fence_after();
                 const BwdCol cr = bwd_col<SIDE>(it, t);
                 const bool s1 = (SIDE == kBwdRowsQ) && cr.src == 1;
@@ -624,17 +692,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                 // The per-column lse / D of a rows-KV sub-tile come in by bulk copy with the
                 // stage: observe the stage's barrier (already complete) before reading them.
                 if (SIDE == kBwdRowsKV) wait_bar_warp(&col_full[n % NST], (n / NST) & 1u, abort_flag, p.err);
-                usum += bwd_subtile<SIDE>(tmem_base + lane_off + w * 128, cmin, cmax, sl2, nl2_row, c_row, ld,
+                usum += bwd_subtile<SIDE>(tmem_base + lane_off + set * 128, cmin, cmax, sl2, nl2_row, c_row, ld,
                                           ld + kBwdCols);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(&p_full[w]);
-                ++own;
+                ptx::mbar_arrive(&p_full[set]);
             }
             // ------------------------------------------------------------ epilogue
+            // The gradient tile goes to shared memory in the swizzled layout of its tensor map, the
+            // accumulator is released, and one thread stores the tile with TMA (rows past L are
+            // clipped by the map).
             const uint32_t ab = iw % NACC;
-            const uint32_t acc = tmem_base + lane_off + 256 + ab * 2 * D;
+            const uint32_t acc = tmem_base + lane_off + ACC0 + ab * 2 * D;
+            const int wtid = threadIdx.x - 128 - 128 * w;  // 0..127 within the warpgroup
+            constexpr int UNITS_PER_CHUNK = C::RB / 16;
             if (SIDE == kBwdRowsQ) {
+                uint8_t* stage = smem + SM::OFF_STG;
+                // the previous item's store has finished reading the stage
+                if (w == 0 && wtid == 0) ptx::tma_store_wait_read_all();
                 // D_i - c_i = the sum of u over both warpgroups' sub-tiles.
                 const int par = iw & 1;
                 xch[(par * 2 + w) * kBwdRows + lrow] = usum;
@@ -644,7 +719,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                 ptx::tc_fence_after();
                 constexpr int HALF = D / 2;
                 constexpr int CW = HALF < 32 ? HALF : 32;
-                __nv_bfloat16* dq = p.g_a[0] + (static_cast<size_t>(it.row_z) * p.L + row) * D;
 #pragma unroll
                 for (int c0 = w * HALF; c0 < (w + 1) * HALF; c0 += CW) {
                     float y[CW], x[CW];
@@ -652,31 +726,65 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                     load_tmem_cols<CW>(acc + D + c0, x);
 #pragma unroll
                     for (int c = 0; c < CW; ++c) x[c] = fmaf(-du, y[c], x[c]);
-                    if (valid) store_row_bf16<CW>(dq + c0, x, p.scale);
+#pragma unroll
+                    for (int g = 0; g < CW / 8; ++g) {
+                        const int unit = (c0 + 8 * g) / 8;
+                        *reinterpret_cast<uint4*>(stage + (unit / UNITS_PER_CHUNK) * C::ROW_CHUNK +
+                                                  swz_offset<C::RB>(lrow, unit % UNITS_PER_CHUNK)) =
+                            pack8_bf16(&x[8 * g], p.scale);
+                    }
                 }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&acc_free[ab]);
                 if (w == 0) {
                     const size_t r = static_cast<size_t>(it.row_z) * p.Lpad + row;
                     p.ws_nl2[r] = valid ? nl2_row : -INFINITY;
                     p.ws_D[r] = valid ? c_row + du : 0.f;
                 }
+                ptx::fence_proxy_async_smem();
+                ptx::named_barrier_sync(1, kSoftmaxThreads);
+                if (w == 0 && wtid == 0) {
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        ptx::tma_store_3d(&p.tm_ga[0], stage + ch * C::ROW_CHUNK, ch * (C::RB / 2), it.row0,
+                                          it.row_z);
+                    ptx::tma_store_commit();
+                }
             } else {
+                // warpgroup 0 writes dv = dV, warpgroup 1 dk = scale dK, each from its own stage
+                uint8_t* stage = smem + SM::OFF_STG + w * C::ROW_TILE;
+                if (wtid == 0) ptx::tma_store_wait_read_all();
+                ptx::named_barrier_sync(2 + w, 128);
                 wait_bar_warp(&acc_full[ab], (iw / NACC) & 1u, abort_flag, p.err);
                 ptx::tc_fence_after();
                 constexpr int CW = D < 32 ? D : 32;
-                __nv_bfloat16* dst = (w == 0 ? p.g_a[it.src] : p.g_b[it.src]) +
-                                     (static_cast<size_t>(it.row_z) * p.L + row) * D;
                 const float f = (w == 0) ? 1.f : p.scale;
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += CW) {
                     float v[CW];
                     load_tmem_cols<CW>(acc + w * D + c0, v);
-                    if (valid) store_row_bf16<CW>(dst + c0, v, f);
+#pragma unroll
+                    for (int g = 0; g < CW / 8; ++g) {
+                        const int unit = (c0 + 8 * g) / 8;
+                        *reinterpret_cast<uint4*>(stage + (unit / UNITS_PER_CHUNK) * C::ROW_CHUNK +
+                                                  swz_offset<C::RB>(lrow, unit % UNITS_PER_CHUNK)) =
+                            pack8_bf16(&v[8 * g], f);
+                    }
+                }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&acc_free[ab]);
+                ptx::fence_proxy_async_smem();
+                ptx::named_barrier_sync(2 + w, 128);
+                if (wtid == 0) {
+                    const CUtensorMap* m = (w == 0) ? &p.tm_ga[it.src] : &p.tm_gb[it.src];
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        ptx::tma_store_3d(m, stage + ch * C::ROW_CHUNK, ch * (C::RB / 2), it.row0, it.row_z);
+                    ptx::tma_store_commit();
                 }
             }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&acc_free[ab]);
             ++iw;
         }
+        // every issued store has completed before the CTA exits
+        if (threadIdx.x == 128 || (SIDE == kBwdRowsKV && threadIdx.x == 256)) ptx::tma_store_wait_all();
         ptx::tc_fence_before();
         ptx::mbar_arrive(softmax_done);
     }
