@@ -20,7 +20,7 @@
 //               which is the formula above for ANY constant c_i (sum_j p_ij (dp_ij - D_i) k_j =
 //               sum_j p_ij (dp_ij - c_i) k_j - (D_i - c_i) sum_j p_ij k_j); c_i close to D_i keeps
 //               the bf16 operands u small where one key holds a row's weight, so the difference
-//               X - (D - c) Y does not cancel to rounding noise.  D_i and -lse_i log2e go to the
+//               X - (D - c) Y does not cancel to rounding noise.  -D_i and -lse_i log2e go to the
 //               workspace for the second launch.
 //   kBwdRowsKV  one item = 128 keys of one kv head and key source (keys on the TMEM lanes); the
 //               queries of every head of the GQA group that see them stream past in 64-query
@@ -72,7 +72,7 @@ struct alignas(64) BwdTcParams {
     const __nv_bfloat16* out;         // rows-Q: the forward's output [B*Hq][L][D]
     const __nv_bfloat16* dout;        // rows-Q: [B*Hq][L][D]
     float* ws_nl2;                    // [B*Hq][Lpad]: -lse*log2(e), -inf past L (rows-Q writes it)
-    float* ws_D;                      // [B*Hq][Lpad]: D_i, 0 past L
+    float* ws_D;                      // [B*Hq][Lpad]: -D_i, 0 past L
     __nv_bfloat16* g_a[2];            // rows-Q: dq at [0]; rows-KV: dv of key source 0/1
     __nv_bfloat16* g_b[2];            // rows-KV: dk of key source 0/1
     unsigned int* err;                // device error word
@@ -107,7 +107,7 @@ struct BwdSmem {
     using C = BwdCfg<D>;
     static constexpr int OFF_R = 0;                                        // [RBUF][2] row tiles
     static constexpr int OFF_C = OFF_R + C::RBUF * 2 * C::ROW_TILE;        // [NST][2] column tiles
-    static constexpr int OFF_LD = OFF_C + C::NST * 2 * C::COL_TILE;        // [NST][2][64] nl2, D
+    static constexpr int OFF_LD = OFF_C + C::NST * 2 * C::COL_TILE;        // [NST][2][64] nl2, -D
     static constexpr int OFF_X = OFF_LD + C::NST * 2 * kBwdCols * 4;       // [2][2][128] sum exchange
     static constexpr int OFF_ROWD = OFF_X + 2 * 2 * kBwdRows * 4;         // [2][2][128] rows-Q: c_i, -lse_i log2e
     static constexpr int OFF_STG = ((OFF_ROWD + 2 * 2 * kBwdRows * 4 + 1023) / 1024) * 1024;  // [2] gradient tiles
@@ -269,12 +269,14 @@ __device__ __forceinline__ void bwd_interval(const BwdTcParams& p, int row, int 
 
 // One sub-tile of one warpgroup, one lane = one row: reads the 64 S and 64 dP columns of its set,
 // writes p (bf16, packed over S columns 0..31) and u / ds (over dP columns 0..31), and returns
-// sum(u) (rows-Q).  Columns outside [cmin, cmax) get p = 0.
+// sum(u) (rows-Q).  Columns outside [cmin, cmax) get p = 0.  The arithmetic runs on column pairs
+// (packed fp32x2 FMA / add / multiply of sm_100), the exponentials one by one.
 //   rows-Q:  exponent argument s*sl2 + nl2_row, u = p (dp - c_row)
-//   rows-KV: exponent argument s*sl2 + nl2_col[c], u = p (dp - d_col[c])
+//   rows-KV: exponent argument s*sl2 + nl2[c], ds = p (dp - D[c]); nl2 and -D of the sub-tile's 64
+//            columns sit in shared memory at ld_saddr (64 floats, then 64 floats)
 template <int SIDE>
 __device__ __forceinline__ float bwd_subtile(uint32_t set_tmem, int cmin, int cmax, float sl2, float nl2_row,
-                                             float c_row, const float* nl2_col, const float* d_col) {
+                                             float c_row, uint32_t ld_saddr) {
     uint32_t sr[64], dr[64];
     ptx::tmem_ld32(set_tmem, sr);
     ptx::tmem_ld32(set_tmem + 32, sr + 32);
@@ -283,7 +285,8 @@ __device__ __forceinline__ float bwd_subtile(uint32_t set_tmem, int cmin, int cm
     ptx::tmem_wait_ld();
     ptx::reg_fence<64>(sr);
     ptx::reg_fence<64>(dr);
-    float usum[2] = {0.f, 0.f};
+    const float2 sl2v = make_float2(sl2, sl2);
+    float2 usum = make_float2(0.f, 0.f);
 #pragma unroll
     for (int a = 0; a < 2; ++a) {
         const bool mine = (cmin < 32 * a + 32) && (cmax > 32 * a);
@@ -293,30 +296,35 @@ __device__ __forceinline__ float bwd_subtile(uint32_t set_tmem, int cmin, int cm
         if (live) {
 #pragma unroll
             for (int c4 = 0; c4 < 32; c4 += 4) {
-                float nl[4], dd[4];
+                const int col = 32 * a + c4;
+                float2 nl[2], nd[2];
                 if (SIDE == kBwdRowsKV) {
-                    const float4 a4 = *reinterpret_cast<const float4*>(nl2_col + 32 * a + c4);
-                    const float4 b4 = *reinterpret_cast<const float4*>(d_col + 32 * a + c4);
-                    nl[0] = a4.x; nl[1] = a4.y; nl[2] = a4.z; nl[3] = a4.w;
-                    dd[0] = b4.x; dd[1] = b4.y; dd[2] = b4.z; dd[3] = b4.w;
+                    const float4 a4 = ptx::lds_f4(ld_saddr + col * 4);
+                    const float4 b4 = ptx::lds_f4(ld_saddr + (kBwdCols + col) * 4);
+                    nl[0] = make_float2(a4.x, a4.y);
+                    nl[1] = make_float2(a4.z, a4.w);
+                    nd[0] = make_float2(b4.x, b4.y);
+                    nd[1] = make_float2(b4.z, b4.w);
                 } else {
-                    nl[0] = nl[1] = nl[2] = nl[3] = nl2_row;
-                    dd[0] = dd[1] = dd[2] = dd[3] = c_row;
+                    nl[0] = nl[1] = make_float2(nl2_row, nl2_row);
+                    nd[0] = nd[1] = make_float2(-c_row, -c_row);
                 }
-                float pv[4], uv[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int col = 32 * a + c4 + e;
-                    float pe = ptx::ex2(fmaf(__uint_as_float(sr[col]), sl2, nl[e]));
-                    if (!whole) pe = (col >= cmin && col < cmax) ? pe : 0.f;
-                    pv[e] = pe;
-                    uv[e] = pe * (__uint_as_float(dr[col]) - dd[e]);
+                for (int h = 0; h < 2; ++h) {
+                    const int c = col + 2 * h;
+                    const float2 sv = make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                    const float2 dv = make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1]));
+                    const float2 x = __ffma2_rn(sv, sl2v, nl[h]);
+                    float2 pv = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+                    if (!whole) {
+                        pv.x = (c >= cmin && c < cmax) ? pv.x : 0.f;
+                        pv.y = (c + 1 >= cmin && c + 1 < cmax) ? pv.y : 0.f;
+                    }
+                    const float2 uv = __fmul2_rn(pv, __fadd2_rn(dv, nd[h]));
+                    if (SIDE == kBwdRowsQ) usum = __fadd2_rn(usum, uv);
+                    pk[(c4 >> 1) + h] = ptx::pack_bf16x2(pv.x, pv.y);
+                    uk[(c4 >> 1) + h] = ptx::pack_bf16x2(uv.x, uv.y);
                 }
-                usum[(c4 >> 2) & 1] += (uv[0] + uv[1]) + (uv[2] + uv[3]);
-                pk[c4 / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
-                pk[c4 / 2 + 1] = ptx::pack_bf16x2(pv[2], pv[3]);
-                uk[c4 / 2] = ptx::pack_bf16x2(uv[0], uv[1]);
-                uk[c4 / 2 + 1] = ptx::pack_bf16x2(uv[2], uv[3]);
             }
         } else {
 #pragma unroll
@@ -325,7 +333,7 @@ __device__ __forceinline__ float bwd_subtile(uint32_t set_tmem, int cmin, int cm
         ptx::tmem_st16(set_tmem + 16 * a, pk);
         ptx::tmem_st16(set_tmem + 64 + 16 * a, uk);
     }
-    return usum[0] + usum[1];
+    return usum.x + usum.y;
 }
 
 // Dot product of two bf16 rows of length D (16-byte loads), fp32.
@@ -688,12 +696,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                 const bool s1 = (SIDE == kBwdRowsQ) && cr.src == 1;
                 const int cmin = (s1 ? lo1 : lo0) - cr.y;
                 const int cmax = (s1 ? hi1 : hi0) - cr.y;
-                const float* ld = reinterpret_cast<const float*>(smem + SM::OFF_LD) + (n % NST) * 2 * kBwdCols;
+                const uint32_t ld_saddr = smem_base + SM::OFF_LD + (n % NST) * 2 * kBwdCols * 4;
                 // The per-column lse / D of a rows-KV sub-tile come in by bulk copy with the
                 // stage: observe the stage's barrier (already complete) before reading them.
                 if (SIDE == kBwdRowsKV) wait_bar_warp(&col_full[n % NST], (n / NST) & 1u, abort_flag, p.err);
-                usum += bwd_subtile<SIDE>(tmem_base + lane_off + set * 128, cmin, cmax, sl2, nl2_row, c_row, ld,
-                                          ld + kBwdCols);
+                usum += bwd_subtile<SIDE>(tmem_base + lane_off + set * 128, cmin, cmax, sl2, nl2_row, c_row,
+                                          ld_saddr);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&p_full[set]);
@@ -739,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                 if (w == 0) {
                     const size_t r = static_cast<size_t>(it.row_z) * p.Lpad + row;
                     p.ws_nl2[r] = valid ? nl2_row : -INFINITY;
-                    p.ws_D[r] = valid ? c_row + du : 0.f;
+                    p.ws_D[r] = valid ? -(c_row + du) : 0.f;
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::named_barrier_sync(1, kSoftmaxThreads);
