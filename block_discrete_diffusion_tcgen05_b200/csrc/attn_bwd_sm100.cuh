@@ -68,6 +68,7 @@ struct alignas(64) BwdTcParams {
     CUtensorMap tm_r2[2];  // row operand 2: rows-Q: dO at [0]; rows-KV: V of key source 0/1
     CUtensorMap tm_c1[2];  // column operand 1 (64-row boxes): rows-Q: K of key source 0/1; rows-KV: Q at [0]
     CUtensorMap tm_c2[2];  // column operand 2: rows-Q: V of key source 0/1; rows-KV: dO at [0]
+    CUtensorMap tm_out;    // rows-Q: the forward's output (128-row boxes), for c_i
     const float* lse;                 // rows-Q: the forward's lse [B*Hq][L] (natural log)
     const __nv_bfloat16* out;         // rows-Q: the forward's output [B*Hq][L][D]
     const __nv_bfloat16* dout;        // rows-Q: [B*Hq][L][D]
@@ -111,11 +112,13 @@ struct BwdSmem {
     static constexpr int OFF_X = OFF_LD + C::NST * 2 * kBwdCols * 4;       // [2][2][128] sum exchange
     static constexpr int OFF_ROWD = OFF_X + 2 * 2 * kBwdRows * 4;         // [2][2][128] rows-Q: c_i, -lse_i log2e
     static constexpr int OFF_STG = ((OFF_ROWD + 2 * 2 * kBwdRows * 4 + 1023) / 1024) * 1024;  // [2] gradient tiles
+    // rows-Q stores one gradient tile: the second stage buffer holds the forward's out tile
+    static constexpr int OFF_OUT = OFF_STG + C::ROW_TILE;
     static constexpr int OFF_BAR = OFF_STG + 2 * C::ROW_TILE;
     // row_full[RBUF], row_empty[RBUF], col_full[NST], col_empty[NST], s_full[NSET], p_full[NSET],
-    // set_free[NSET], acc_full[NACC], acc_free[NACC], rowd_full[2], rowd_empty[2], mma_drain,
-    // acc_drain, softmax_done
-    static constexpr int NBAR = 2 * C::RBUF + 2 * C::NST + 3 * C::NSET + 2 * C::NACC + 4 + 3;
+    // set_free[NSET], acc_full[NACC], acc_free[NACC], rowd_full[2], rowd_empty[2], out_full,
+    // out_empty, acc_issued, mma_drain, acc_drain, softmax_done
+    static constexpr int NBAR = 2 * C::RBUF + 2 * C::NST + 3 * C::NSET + 2 * C::NACC + 4 + 3 + 3;
     static constexpr int OFF_MISC = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
@@ -133,20 +136,24 @@ struct BwdItem {
 };
 
 // Items in a fixed order that every role walks; longest first (static round robin over CTAs).
+// Rounds of gridDim.x items go to the CTAs alternately forwards and backwards (boustrophedon), so
+// the per-CTA sums of the decreasing item costs stay level.
 template <int SIDE>
 struct BwdScheduler {
     const BwdTcParams& p;
-    int k;
-    __device__ explicit BwdScheduler(const BwdTcParams& prm) : p(prm), k(blockIdx.x) {}
+    int r;  // round
+    __device__ explicit BwdScheduler(const BwdTcParams& prm) : p(prm), r(0) {}
 
     __device__ bool next(BwdItem& it) {
+        const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+        const int k = r * G + ((r & 1) ? G - 1 - c : c);
         if (k >= p.num_items) return false;
+        ++r;
         const int L = p.L, S = p.S;
         if (SIDE == kBwdRowsQ) {
             const int BH = p.batch * p.q_heads;
             const int qt = p.n_row_tiles - 1 - k / BH;  // later query tiles see more keys
             const int bh = k % BH;
-            k += gridDim.x;
             const int b = bh / p.q_heads, h = bh % p.q_heads;
             it.row_z = bh;
             it.row0 = qt * kBwdRows;
@@ -172,7 +179,6 @@ struct BwdScheduler {
             const int src = k / per_src;  // decoder: encoder-side keys first (they see more queries)
             const int kk = k % per_src;
             const int kt = kk / BH, z = kk % BH;
-            k += gridDim.x;
             it.row_z = z;
             it.row0 = kt * kBwdRows;
             it.src = src;
@@ -388,14 +394,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
     uint64_t* acc_free = acc_full + NACC;                                                            \
     uint64_t* rowd_full = acc_free + NACC;                                                           \
     uint64_t* rowd_empty = rowd_full + 2;                                                            \
-    uint64_t* mma_drain = rowd_empty + 2;                                                            \
+    uint64_t* out_full = rowd_empty + 2;                                                             \
+    uint64_t* out_empty = out_full + 1;                                                              \
+    uint64_t* acc_issued = out_empty + 1;                                                            \
+    uint64_t* mma_drain = acc_issued + 1;                                                            \
     uint64_t* acc_drain = mma_drain + 1;                                                             \
     uint64_t* softmax_done = acc_drain + 1;                                                          \
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);                        \
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);             \
     (void)row_full; (void)row_empty; (void)col_full; (void)col_empty; (void)s_full; (void)p_full;    \
     (void)acc_full; (void)acc_free; (void)mma_drain; (void)softmax_done; (void)tmem_holder;          \
-    (void)set_free; (void)acc_drain; (void)rowd_full; (void)rowd_empty;                              \
+    (void)set_free; (void)acc_drain; (void)rowd_full; (void)rowd_empty; (void)out_full;              \
+    (void)out_empty; (void)acc_issued;                                                               \
     (void)abort_flag;
     uint32_t tmem_base;
     {
@@ -403,7 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
         if (threadIdx.x == 0) {
             for (int i = 0; i < RBUF; ++i) {
                 ptx::mbar_init(&row_full[i], 1);
-                ptx::mbar_init(&row_empty[i], 1);
+                // rows-Q: warp 3 also reads the dO tile (for c_i) before the buffer is reused
+                ptx::mbar_init(&row_empty[i], SIDE == kBwdRowsQ ? 2 : 1);
             }
             for (int i = 0; i < NST; ++i) {
                 ptx::mbar_init(&col_full[i], 1);
@@ -422,6 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                 ptx::mbar_init(&rowd_full[i], 32);
                 ptx::mbar_init(&rowd_empty[i], kSoftmaxThreads);
             }
+            ptx::mbar_init(out_full, 1);
+            ptx::mbar_init(out_empty, 1);
+            ptx::mbar_init(acc_issued, 1);
             ptx::mbar_init(mma_drain, 1);
             ptx::mbar_init(acc_drain, 1);
             ptx::mbar_init(softmax_done, kSoftmaxThreads);
@@ -478,6 +492,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                 }
             }
             __syncwarp();
+            if (SIDE == kBwdRowsQ) {
+                // the forward's out tile of the item's rows (one buffer; warp 3 frees it)
+                ok = wait_bar_warp(out_empty, (iw & 1u) ^ 1u, abort_flag, p.err);
+                if (!ok) break;
+                if (leader) {
+                    ptx::mbar_arrive_expect_tx(out_full, C::ROW_TILE);
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        ptx::tma_load_3d(&p.tm_out, out_full, smem + SM::OFF_OUT + ch * C::ROW_CHUNK, ch * (C::RB / 2),
+                                         it.row0, it.row_z);
+                }
+                __syncwarp();
+            }
             ++iw;
             for (int t = 0; t < it.nsub; ++t) {
                 const uint32_t st = n % NST;
@@ -513,6 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             wait_bar_warp(&col_full[i % NST], (i / NST) & 1u, &no_abort, p.err);
         for (uint32_t i = iw > static_cast<uint32_t>(RBUF) ? iw - RBUF : 0u; i < iw; ++i)
             wait_bar_warp(&row_full[i % RBUF], (i / RBUF) & 1u, &no_abort, p.err);
+        if (SIDE == kBwdRowsQ && iw > 0) wait_bar_warp(out_full, (iw - 1) & 1u, &no_abort, p.err);
     } else if (warp == 1) {
         ptx::setmaxnreg_dec<kRegsControl>();
         // ------------------------------------------------------------------ product issuer
@@ -530,6 +557,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             const uint32_t rb = iw % RBUF;
             ok = wait_bar_warp(&row_full[rb], (iw / RBUF) & 1u, abort_flag, p.err);
             if (!ok) break;
+            // The previous item's last accumulation goes to the tensor core before this item's
+            // products, so its epilogue is not held up behind them.
+            if (iw > 0) {
+                ok = wait_bar_warp(acc_issued, (iw - 1) & 1u, abort_flag, p.err);
+                if (!ok) break;
+            }
             const uint32_t r1 = sR + (rb * 2 + 0) * C::ROW_TILE;
             const uint32_t r2 = sR + (rb * 2 + 1) * C::ROW_TILE;
             for (int t = 0; t < it.nsub && ok; ++t, ++n) {
@@ -604,7 +637,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                     }
                     ptx::mma_commit(&col_empty[st]);
                     ptx::mma_commit(&set_free[set]);
-                    if (t == it.nsub - 1) ptx::mma_commit(&acc_full[ab]);
+                    if (t == it.nsub - 1) {
+                        ptx::mma_commit(&acc_full[ab]);
+                        ptx::mbar_arrive(acc_issued);
+                    }
                 }
                 __syncwarp();
             }
@@ -623,22 +659,47 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             BwdScheduler<SIDE> sched(p);
             BwdItem it;
             uint32_t iw = 0;
+            constexpr int UNITS_PER_CHUNK = C::RB / 16;
             while (sched.next(it)) {
                 if (it.nsub == 0) continue;
-                const uint32_t par = iw & 1u;
+                const uint32_t par = iw & 1u, rb = iw % RBUF;
+                // -lse log2(e) of this lane's four rows (global loads issued first)
+                float nl[kBwdRows / 32];
+#pragma unroll
+                for (int j = 0; j < kBwdRows / 32; ++j) {
+                    const int row = it.row0 + j * 32 + lane;
+                    nl[j] = row < p.L ? -__ldg(p.lse + static_cast<size_t>(it.row_z) * p.L + row) * kLog2e : 0.f;
+                }
                 wait_bar_warp(&rowd_empty[par], ((iw >> 1) & 1u) ^ 1u, abort_flag, p.err);
+                wait_bar_warp(&row_full[rb], (iw / RBUF) & 1u, abort_flag, p.err);
+                wait_bar_warp(out_full, iw & 1u, abort_flag, p.err);
+                const uint8_t* tdo = smem + SM::OFF_R + (rb * 2 + 1) * C::ROW_TILE;
+                const uint8_t* tout = smem + SM::OFF_OUT;
 #pragma unroll
                 for (int j = 0; j < kBwdRows / 32; ++j) {
                     const int lr = j * 32 + lane;
-                    const int row = it.row0 + lr;
-                    float c = 0.f, nl = 0.f;
-                    if (row < p.L) {
-                        const size_t r = static_cast<size_t>(it.row_z) * p.L + row;
-                        c = row_dot_bf16<D>(p.dout + r * D, p.out + r * D);
-                        nl = -__ldg(p.lse + r) * kLog2e;
+                    float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int unit = 0; unit < D / 8; ++unit) {
+                        const uint32_t off = (unit / UNITS_PER_CHUNK) * C::ROW_CHUNK +
+                                             swz_offset<C::RB>(lr, unit % UNITS_PER_CHUNK);
+                        const uint4 x = *reinterpret_cast<const uint4*>(tdo + off);
+                        const uint4 y = *reinterpret_cast<const uint4*>(tout + off);
+                        const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            acc2 = __ffma2_rn(__bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[e])),
+                                              __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[e])),
+                                              acc2);
                     }
-                    rowd[(par * 2 + 0) * kBwdRows + lr] = c;
-                    rowd[(par * 2 + 1) * kBwdRows + lr] = nl;
+                    // rows past L: zero tiles (out-of-bounds fill), so c = 0
+                    rowd[(par * 2 + 0) * kBwdRows + lr] = acc2.x + acc2.y;
+                    rowd[(par * 2 + 1) * kBwdRows + lr] = nl[j];
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(out_empty);
+                    ptx::mbar_arrive(&row_empty[rb]);
                 }
                 ptx::mbar_arrive(&rowd_full[par]);
                 ++iw;

@@ -301,7 +301,7 @@ e2d2_status train_backward(bool decoder, const BwdArgs& a, const e2d2_dims& dm, 
     bool ok = map_3d(&pq.tm_r1[0], a.q, D, L, BHq, L, kBwdRows) && map_3d(&pq.tm_r2[0], a.dout, D, L, BHq, L, kBwdRows) &&
               map_3d(&pq.tm_c1[0], a.k0, D, L, BHkv, L, kBwdCols) && map_3d(&pq.tm_c2[0], a.v0, D, L, BHkv, L, kBwdCols) &&
               map_3d(&pq.tm_c1[1], k1, D, L, BHkv, L, kBwdCols) && map_3d(&pq.tm_c2[1], v1, D, L, BHkv, L, kBwdCols);
-    ok = ok && map_3d(&pq.tm_ga[0], a.dq, D, L, BHq, L, kBwdRows);
+    ok = ok && map_3d(&pq.tm_ga[0], a.dq, D, L, BHq, L, kBwdRows) && map_3d(&pq.tm_out, a.out, D, L, BHq, L, kBwdRows);
     pq.tm_ga[1] = pq.tm_gb[0] = pq.tm_gb[1] = pq.tm_ga[0];
     pq.tm_r1[1] = pq.tm_r1[0];
     pq.tm_r2[1] = pq.tm_r2[0];
@@ -318,6 +318,7 @@ e2d2_status train_backward(bool decoder, const BwdArgs& a, const e2d2_dims& dm, 
     if (!ok) return E2D2_ERR_CUDA;
     pk.tm_c1[1] = pk.tm_c1[0];
     pk.tm_c2[1] = pk.tm_c2[0];
+    pk.tm_out = pk.tm_ga[0];  // unused on this side
     pk.g_a[0] = static_cast<__nv_bfloat16*>(a.dv0);
     pk.g_b[0] = static_cast<__nv_bfloat16*>(a.dk0);
     pk.g_a[1] = static_cast<__nv_bfloat16*>(decoder ? a.dv1 : a.dv0);
