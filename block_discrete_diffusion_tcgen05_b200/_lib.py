@@ -19,7 +19,8 @@ EXPORTS = ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
            "e2d2_kv_cache_append", "e2d2_status_string", "e2d2_last_device_error", "e2d2_version",
            "e2d2_attn_decoder_sample_noalloc", "e2d2_attn_encoder_block_step",
            "e2d2_attn_train_backward_workspace", "e2d2_attn_encoder_backward",
-           "e2d2_attn_decoder_train_backward", "e2d2_attn_decoder_sample_plan")
+           "e2d2_attn_decoder_train_backward", "e2d2_attn_decoder_sample_plan",
+           "e2d2_attn_decoder_sample_ragged", "e2d2_attn_decoder_sample_ragged_plan")
 
 # E2D2_SAMPLE_NOALLOC_MAX_BYTES of include/e2d2_attn.h
 SAMPLE_NOALLOC_MAX_BYTES = 32 << 20
@@ -38,6 +39,13 @@ class SamplePlan(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int), ("units", ctypes.c_int), ("tiles_per_unit", ctypes.c_int),
                 ("split_units", ctypes.c_int), ("split_ctas", ctypes.c_int), ("whole_units", ctypes.c_int),
                 ("grid", ctypes.c_int)]
+
+
+class RaggedPlan(ctypes.Structure):
+    """e2d2_ragged_plan."""
+
+    _fields_ = [("kernel", ctypes.c_int), ("units", ctypes.c_int), ("units_per_entry", ctypes.c_int),
+                ("total_tiles", ctypes.c_longlong), ("grid", ctypes.c_int)]
 
 
 class E2D2Error(RuntimeError):
@@ -80,6 +88,12 @@ def load(path: Path | str | None = None):
                                                      Dims, ci, ci, vp, ctypes.c_size_t, st]
     lib.e2d2_attn_decoder_sample_plan.argtypes = [Dims, ci, ci, ci, ctypes.POINTER(SamplePlan)]
     lib.e2d2_attn_decoder_sample_plan.restype = ctypes.c_int
+    lib.e2d2_attn_decoder_sample_ragged.argtypes = [vp, vp, vp, ci, vp, vp, vp, vp, fp, Dims, ci, vp,
+                                                    ctypes.c_size_t, st]
+    lib.e2d2_attn_decoder_sample_ragged.restype = ctypes.c_int
+    lib.e2d2_attn_decoder_sample_ragged_plan.argtypes = [Dims, ci, ctypes.POINTER(ctypes.c_int), ci, ci,
+                                                         ctypes.POINTER(RaggedPlan)]
+    lib.e2d2_attn_decoder_sample_ragged_plan.restype = ctypes.c_int
     lib.e2d2_status_string.argtypes = [ci]
     lib.e2d2_status_string.restype = ctypes.c_char_p
     lib.e2d2_last_device_error.argtypes = [st]

@@ -249,6 +249,48 @@ def decoder_sample(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=None
     return out, lse_t
 
 
+def sample_ragged_plan(batch, q_heads, kv_heads, head_dim, S, P, capacity, num_sms) -> dict:
+    """Work plan of a ragged sampling call for host prefix lengths P (a sequence of batch ints)."""
+    lib = _lib.load()
+    P = [int(x) for x in P]
+    if len(P) != batch:
+        raise ValueError("P must hold one prefix length per batch entry")
+    arr = (ctypes.c_int * max(batch, 1))(*P)
+    plan = _lib.RaggedPlan()
+    st = lib.e2d2_attn_decoder_sample_ragged_plan(_dims(batch, q_heads, kv_heads, head_dim, None), S, arr, capacity,
+                                                  num_sms, ctypes.byref(plan))
+    _lib.check(st, "e2d2_attn_decoder_sample_ragged_plan")
+    return {name: getattr(plan, name) for name, _ in _lib.RaggedPlan._fields_}
+
+
+@_device_guard
+def decoder_sample_ragged(q_blk, k_cache, v_cache, P, k_blk, v_blk, workspace=None, scale=None, out=None, lse=True):
+    """Sampling step with one prefix length per batch entry: P is a CUDA int32 tensor [B]; entry b
+    attends to k_cache[b, :, :P[b]] and its own block."""
+    lib = _lib.load()
+    for t, n in ((q_blk, "q_blk"), (k_cache, "k_cache"), (v_cache, "v_cache"), (k_blk, "k_blk"),
+                 (v_blk, "v_blk")):
+        _need(t, n)
+    _need(P, "P", dtype=torch.int32, ndim=1)
+    B, Hq, S, d = q_blk.shape
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, cap, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [B, Hkv, capacity, d]")
+    if k_blk.shape != (B, Hkv, S, d) or v_blk.shape != k_blk.shape:
+        raise ValueError("k_blk/v_blk must be [B, Hkv, S, d]")
+    if P.shape != (B,):
+        raise ValueError("P must be [B]")
+    ws = sample_workspace(q_blk, k_cache) if workspace is None else _need_workspace(workspace)
+    out = _out_tensor(out, q_blk)
+    lse_t = _lse_tensor(lse, (B, Hq, S), q_blk.device)
+    st = lib.e2d2_attn_decoder_sample_ragged(q_blk.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cap,
+                                             P.data_ptr(), k_blk.data_ptr(), v_blk.data_ptr(), out.data_ptr(),
+                                             _ptr(lse_t), _dims(B, Hq, Hkv, d, scale), S, ws.data_ptr(),
+                                             ws.numel() * ws.element_size(), _stream(q_blk))
+    _lib.check(st, "e2d2_attn_decoder_sample_ragged")
+    return out, lse_t
+
+
 @_device_guard
 def encoder_block_step(q_blk, k_cache, v_cache, P: int, k_blk, v_blk, workspace=None, scale=None,
                        out=None, lse=True):

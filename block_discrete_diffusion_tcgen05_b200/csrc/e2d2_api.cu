@@ -409,8 +409,8 @@ struct SampleLaunch {
 // error return leaves the stream untouched.  `append` (encoder block step) also writes the block's
 // K/V to cache rows P..P+S-1 from inside the same launch.
 e2d2_status sample_prepare(bool append, const void* q_blk, const void* k_cache, const void* v_cache, int capacity,
-                           int P, const void* k_blk, const void* v_blk, void* out, float* lse, e2d2_dims dims,
-                           int S, void* workspace, size_t ws_bytes, SampleLaunch* sl) {
+                           int P, const int* P_dev, const void* k_blk, const void* v_blk, void* out, float* lse,
+                           e2d2_dims dims, int S, void* workspace, size_t ws_bytes, SampleLaunch* sl) {
     if (!q_blk || !k_cache || !v_cache || !k_blk || !v_blk || !out) return E2D2_ERR_INVALID_ARG;
     e2d2_status s = check_dims(dims);
     if (s != E2D2_OK) return s;
@@ -419,6 +419,14 @@ e2d2_status sample_prepare(bool append, const void* q_blk, const void* k_cache, 
     const long long rows = static_cast<long long>(dims.batch) * dims.q_heads * S;
     if (rows > kMaxI32 / 8 || static_cast<long long>(capacity) * dims.batch * dims.kv_heads > kMaxI32)
         return E2D2_ERR_SHAPE;
+    if (P_dev != nullptr) {
+        if (reinterpret_cast<uintptr_t>(P_dev) & 3u) return E2D2_ERR_ALIGNMENT;
+        if (dims.batch > kRaggedMaxBatch) return E2D2_ERR_SHAPE;
+        // every tile index of the stream fits in an int
+        const long long units = static_cast<long long>(dims.batch) * dims.kv_heads *
+                                ((static_cast<long long>(dims.q_heads / dims.kv_heads) * S + kBlockM - 1) / kBlockM);
+        if (units * ((capacity + kBlockN - 1) / kBlockN + (S + kBlockN - 1) / kBlockN) > kMaxI32) return E2D2_ERR_SHAPE;
+    }
     if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_blk) ||
         !aligned16(v_blk) || !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return E2D2_ERR_ALIGNMENT;
@@ -443,9 +451,12 @@ e2d2_status sample_prepare(bool append, const void* q_blk, const void* k_cache, 
     const int q_chunk = kBlockM / 4;
     const SamplePlan plan = plan_sample(dims, S, P, di->sms);
     const int keyrow_n = plan.keyrow_n;
+    // Single prefix: cache rows >= P lie outside the map (zeros, never read).  Ragged prefixes: the
+    // map spans the capacity; the kernels mask keys past each entry's P and zero those V rows.
+    const int map_rows = P_dev != nullptr ? capacity : P;
     bool ok = map_2d(&prm.tm_q, q_blk, D, rows, keyrow_n ? keyrow_n : q_chunk) &&
-              map_3d(&prm.tm_k0, k_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
-              map_3d(&prm.tm_v0, v_cache, D, P > 0 ? P : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
+              map_3d(&prm.tm_k0, k_cache, D, map_rows > 0 ? map_rows : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
+              map_3d(&prm.tm_v0, v_cache, D, map_rows > 0 ? map_rows : 1, BHkv, capacity > 0 ? capacity : 1, kBlockN) &&
               map_3d(&prm.tm_k1, k_blk, D, S, BHkv, S, box1) && map_3d(&prm.tm_v1, v_blk, D, S, BHkv, S, box1);
     if (!ok) return E2D2_ERR_CUDA;
     prm.out = out;
@@ -482,6 +493,18 @@ e2d2_status sample_prepare(bool append, const void* q_blk, const void* k_cache, 
     sl->keyrow_n = keyrow_n;
     sl->head_dim = D;
     sl->grid = plan.grid;
+    if (P_dev != nullptr) {
+        // one stream-K stream over every unit's tiles, cut over a full grid (the tile count is
+        // known only on the device)
+        const int grid = di->sms < kSampleMaxCtas ? di->sms : kSampleMaxCtas;
+        prm.P_dev = P_dev;
+        prm.rg_capacity = capacity;
+        prm.rg_units_per_entry = dims.kv_heads * plan.num_qtiles;
+        prm.split_units = prm.whole_units = 0;
+        prm.total_tiles = 0;
+        prm.split_ctas = grid;
+        sl->grid = grid;
+    }
     return E2D2_OK;
 }
 
@@ -499,8 +522,8 @@ e2d2_status sample_call(bool append, const void* q_blk, const void* k_cache, con
                         int P, const void* k_blk, const void* v_blk, void* out, float* lse, e2d2_dims dims, int S,
                         void* workspace, size_t ws_bytes, cudaStream_t stream) {
     SampleLaunch sl;
-    const e2d2_status s = sample_prepare(append, q_blk, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims,
-                                         S, workspace, ws_bytes, &sl);
+    const e2d2_status s = sample_prepare(append, q_blk, k_cache, v_cache, capacity, P, nullptr, k_blk, v_blk, out, lse,
+                                         dims, S, workspace, ws_bytes, &sl);
     return s != E2D2_OK ? s : sample_launch(sl, stream);
 }
 
@@ -629,6 +652,36 @@ e2d2_status e2d2_attn_encoder_block_step(const void* q_blk, void* k_cache, void*
                        ws_bytes, stream);
 }
 
+e2d2_status e2d2_attn_decoder_sample_ragged(const void* q_blk, const void* k_cache, const void* v_cache, int capacity,
+                                            const int* P_dev, const void* k_blk, const void* v_blk, void* out,
+                                            float* lse, e2d2_dims dims, int S, void* workspace, size_t ws_bytes,
+                                            cudaStream_t stream) {
+    if (!P_dev) return E2D2_ERR_INVALID_ARG;
+    SampleLaunch sl;
+    const e2d2_status s = sample_prepare(false, q_blk, k_cache, v_cache, capacity, 0, P_dev, k_blk, v_blk, out, lse,
+                                         dims, S, workspace, ws_bytes, &sl);
+    return s != E2D2_OK ? s : sample_launch(sl, stream);
+}
+
+e2d2_status e2d2_attn_decoder_sample_ragged_plan(e2d2_dims dims, int S, const int* P_host, int capacity, int num_sms,
+                                                 e2d2_ragged_plan* plan) {
+    if (!plan || !P_host) return E2D2_ERR_INVALID_ARG;
+    e2d2_status s = check_dims(dims);
+    if (s != E2D2_OK) return s;
+    if (S <= 0 || capacity < 0 || num_sms <= 0) return E2D2_ERR_INVALID_ARG;
+    if (dims.batch > kRaggedMaxBatch) return E2D2_ERR_SHAPE;
+    const SamplePlan pl = plan_sample(dims, S, 0, num_sms);
+    const int upe = dims.kv_heads * pl.num_qtiles;
+    long long total = 0;
+    for (int b = 0; b < dims.batch; ++b) total += ragged_entry_tiles(ragged_clamp(P_host[b], capacity), S, upe);
+    plan->kernel = pl.keyrow_n;
+    plan->units = dims.batch * upe;
+    plan->units_per_entry = upe;
+    plan->total_tiles = total;
+    plan->grid = num_sms < kSampleMaxCtas ? num_sms : kSampleMaxCtas;
+    return E2D2_OK;
+}
+
 e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int P, const void* k_new,
                                  const void* v_new, int S_new, e2d2_dims dims, cudaStream_t stream) {
     if (!k_cache || !v_cache || !k_new || !v_new) return E2D2_ERR_INVALID_ARG;
@@ -737,7 +790,7 @@ e2d2_status e2d2_attn_decoder_sample_noalloc(const void* q_blk, const void* k_ca
     if (s != E2D2_OK) return s;
     // Every check first: an error return must leave nothing queued on the stream.
     SampleLaunch sl;
-    s = sample_prepare(false, q_blk, k_cache, v_cache, capacity, P, k_blk, v_blk, out, lse, dims, S, scratch,
+    s = sample_prepare(false, q_blk, k_cache, v_cache, capacity, P, nullptr, k_blk, v_blk, out, lse, dims, S, scratch,
                        kNoAllocScratchBytes, &sl);
     if (s != E2D2_OK) return s;
     // Ticket words must start at zero; they occupy the first kSampleMaxCtas ints.

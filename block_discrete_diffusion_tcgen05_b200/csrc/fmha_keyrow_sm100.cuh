@@ -91,7 +91,9 @@ struct KrSmem {
     static constexpr int OFF_LRED = OFF_CMAX + 2 * 2 * 4 * C::NH * 4;  // float [2 ob][2 wg][4 warps][NH]
     static constexpr int OFF_MROW = OFF_LRED + 2 * 2 * 4 * C::NH * 4;  // float [2 ob][N]
     static constexpr int OFF_MISC = OFF_MROW + 2 * N * 4;
-    static constexpr int BYTES = OFF_MISC + 64 + N * 4;  // + per-column scale of the epilogue
+    // + per-column scale of the epilogue, then the ragged prefix table (+ 8 scan sums)
+    static constexpr int OFF_RG = ((OFF_MISC + 64 + N * 4 + 15) / 16) * 16;
+    static constexpr int BYTES = OFF_RG + (kRaggedMaxBatch + 1 + 8) * 4;
     static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
 };
 
@@ -175,6 +177,8 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);                         \
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);              \
     volatile int* bcast = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 16);                  \
+    int* rg_pre = reinterpret_cast<int*>(smem + SM::OFF_RG);                                          \
+    (void)rg_pre;                                                                                     \
     (void)q_full; (void)q_empty; (void)k_full; (void)k_empty; (void)v_full; (void)v_empty;            \
     (void)s_full; (void)s_free; (void)p_full; (void)pv_done; (void)o_full; (void)o_free;              \
     (void)l_ready; (void)l_free; (void)qk_drain; (void)pv_drain; (void)tmem_done; (void)merge_full;   \
@@ -214,6 +218,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         ptx::tmem_alloc(tmem_holder, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
+    if (p.P_dev != nullptr) ragged_prefix(p, rg_pre, rg_pre + kRaggedMaxBatch + 1);
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -242,7 +247,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         uint64_t* full = is_k ? k_full : v_full;
         uint64_t* empty = is_k ? k_empty : v_empty;
         const uint32_t ring_off = is_k ? SM::OFF_K : SM::OFF_V;
-        Scheduler<kDecoderSample> sched(p);
+        Scheduler<kDecoderSample> sched(p, rg_pre);
         Item it;
         uint32_t iter = 0, item_idx = 0;
         bool ok = true;
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         const uint32_t sQ = smem_base + SM::OFF_Q, sK = smem_base + SM::OFF_K;
         const uint64_t kdesc = ptx::smem_desc(0, 16, 1024, 2u);  // K (A) and Q (B): K-major, 128B swizzle
         constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(kBlockN, N, false, false);
-        Scheduler<kDecoderSample> sched(p);
+        Scheduler<kDecoderSample> sched(p, rg_pre);
         Item it;
         uint32_t kit = 0, item_idx = 0, tc = 0;
         bool ok = true;
@@ -345,7 +350,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         const uint64_t vdesc = ptx::smem_desc(0, C::KV_CHUNK, 1024, 2u);             // V^T: MN-major (d contiguous)
         const uint64_t pdesc = ptx::smem_desc(0, C::P_BYTES, 8 * C::PRB, C::PSWZ);    // P^T: MN-major
         constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(D, N, true, true);
-        Scheduler<kDecoderSample> sched(p);
+        Scheduler<kDecoderSample> sched(p, rg_pre);
         Item it;
         uint32_t vit = 0, item_idx = 0, tc = 0;
         bool ok = true;
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         uint32_t* vote = reinterpret_cast<uint32_t*>(smem + SM::OFF_VOTE) + g * 8;
         float* cmax = reinterpret_cast<float*>(smem + SM::OFF_CMAX) + g * 2 * 4 * NH;
         uint8_t* sP = smem + SM::OFF_P;
-        Scheduler<kDecoderSample> sched(p);
+        Scheduler<kDecoderSample> sched(p, rg_pre);
         Item it;
         uint32_t tc = 0, item_idx = 0;
         while (sched.next(it)) {
@@ -414,7 +419,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 wait_bar_warp(&s_full[sb], use & 1, abort_flag, p.err);
                 ptx::tc_fence_after();
                 const TileRef tr = tile_of<kDecoderSample>(p, it, t);
-                const int len = tr.src ? p.S : p.P;
+                const int len = tr.src ? p.S : it.P;
                 const bool key_ok = key < min(kBlockN, len - tr.kt * kBlockN);
                 float x[NH];
                 {
@@ -496,6 +501,21 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 for (int u = 0; u < NH / 8; ++u)
                     *reinterpret_cast<uint4*>(pbuf + swz_rows<C::PRB>(key, colbase / 8 + u)) =
                         make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                if (g == 0 && p.P_dev != nullptr && tr.src == 0 && it.P - tr.kt * kBlockN < tr.nk16) {
+                    // Ragged prefix: cache rows at or past P[b] in this tile may hold anything (NaN
+                    // included) and O^T += V^T P^T would meet them with p = 0; zero those V rows.
+                    const uint32_t vst = tc % C::NV;
+                    wait_bar_warp(&v_full[vst], (tc / C::NV) & 1u, abort_flag, p.err);
+                    if (key >= it.P - tr.kt * kBlockN && key < tr.nk16) {
+#pragma unroll
+                        for (int ch = 0; ch < 2; ++ch) {
+                            uint4* dst = reinterpret_cast<uint4*>(smem + SM::OFF_V + vst * C::KV_BYTES + ch * C::KV_CHUNK +
+                                                                  key * 128);
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                }
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&p_full[sb]);
@@ -536,7 +556,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         const float* mrow_all = reinterpret_cast<const float*>(smem + SM::OFF_MROW);
         const float* lred_all = reinterpret_cast<const float*>(smem + SM::OFF_LRED);
         uint8_t* stg = smem + SM::OFF_STG;
-        Scheduler<kDecoderSample> sched(p);
+        Scheduler<kDecoderSample> sched(p, rg_pre);
         Item it;
         uint32_t item_idx = 0;
         while (sched.next(it)) {
@@ -547,11 +567,11 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
             wait_bar_warp(&o_full[ob], (item_idx >> 1) & 1, abort_flag, p.err);
             wait_bar_warp(&l_ready[ob], (item_idx >> 1) & 1, abort_flag, p.err);
             ptx::tc_fence_after();
-            const int Tu = p.tiles_per_unit;
+            const int Tu = it.tu;
             const bool whole = (it.t_begin == 0 && it.t_end == Tu);
-            const long long ubeg = static_cast<long long>(it.q_z) * Tu;
-            const long long T = p.total_tiles;
-            const int grid = p.split_ctas;
+            const long long ubeg = it.ubeg;
+            const long long T = it.total;
+            const int grid = it.sgrid;
             const int c_first = whole ? 0 : owner_cta(ubeg, T, grid);
             const int c_last = whole ? 0 : owner_cta(ubeg + Tu - 1, T, grid);
             auto slot_of = [&](int c) -> float* {

@@ -97,7 +97,47 @@ struct alignas(64) FmhaParams {
     uint4* app_dst_k;        // [B*Hkv][capacity][D] bf16
     uint4* app_dst_v;
     int app_capacity;
+    // sample, ragged prefixes only (null otherwise): entry b's queries see cache rows [0, P_dev[b])
+    // (clamped to [0, rg_capacity]); every unit's key tiles form one stream-K stream over all CTAs.
+    const int* P_dev;
+    int rg_capacity;
+    int rg_units_per_entry;  // kv heads x query tiles per kv head
 };
+
+constexpr int kRaggedMaxBatch = 256;  // entries of a ragged sampling call (one per thread of the prefix scan)
+
+__host__ __device__ __forceinline__ int ragged_clamp(int P, int capacity) {
+    return P < 0 ? 0 : (P > capacity ? capacity : P);
+}
+
+// Key tiles of one batch entry of a ragged sampling call: its units' own-block tiles and prefix
+// tiles (128 keys each).
+__host__ __device__ __forceinline__ int ragged_entry_tiles(int P, int S, int units_per_entry) {
+    return units_per_entry * ((S + 127) / 128 + (P + 127) / 128);
+}
+
+// pre[b] = key tiles of entries 0..b-1 (pre[0] = 0, pre[batch] = all tiles), in shared memory.
+// Every thread of the block calls it (one __syncthreads inside); threads 0..255 scan.
+__device__ __forceinline__ void ragged_prefix(const FmhaParams& p, int* pre, int* wsum) {
+    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+    int x = 0;
+    if (t < p.batch) x = ragged_entry_tiles(ragged_clamp(__ldg(p.P_dev + t), p.rg_capacity), p.S, p.rg_units_per_entry);
+    if (t < kRaggedMaxBatch) {
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[wid] = x;
+    }
+    __syncthreads();
+    if (t < kRaggedMaxBatch) {
+        int add = 0;
+        for (int i = 0; i < wid; ++i) add += wsum[i];
+        pre[t + 1] = x + add;
+        if (t == 0) pre[0] = 0;
+    }
+}
 
 // Copies the S block rows of kv head kv_z (K and V) into cache rows P..P+S-1, 16 bytes per
 // thread-step, with `n` threads numbered `tid`.
@@ -146,7 +186,10 @@ struct Smem {
     // s_full[NQ*NSB], p_full[NQ*NSB], pv_done[NQ], o_free[NOB*NQ], mma_drain, softmax_done
     static constexpr int NBAR = 3 * C::NST + 2 * C::QBUF + 2 * C::NQ * C::NSB + C::NQ + C::NOB * C::NQ + 2;
     static constexpr int OFF_MISC = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;
-    static constexpr int BYTES = OFF_MISC + 64;
+    // sampling: ragged prefix table pre[kRaggedMaxBatch + 1] and the scan's 8 warp sums
+    static constexpr int OFF_RG = OFF_MISC + 64;
+    static constexpr int RG_BYTES = C::SAMPLE ? ((kRaggedMaxBatch + 1 + 8) * 4 + 15) / 16 * 16 : 0;
+    static constexpr int BYTES = OFF_RG + RG_BYTES;
     static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
 };
 
@@ -177,6 +220,11 @@ struct Item {
     int n1, a1;     // source-1 tiles (visited first), starting at key tile a1
     int n0;         // source-0 tiles, starting at key tile 0
     int t_begin, t_end;
+    // sample: the unit's prefix length, its key tiles, its first tile in the stream of split
+    // units, and the length of that stream
+    int P, tu;
+    long long ubeg, total;
+    int sgrid;      // sample: CTAs the split stream is cut over
     // What each query tile needs of that stream: source-1 key tiles [a1q, e1q), source-0 key
     // tiles [0, n0q).  Other tiles are skipped for that query tile (no MMA, no softmax).
     int a1q[2], e1q[2], n0q[2];
@@ -210,22 +258,83 @@ __device__ __forceinline__ void train_ranges(int L, int S, int r0, int r_last, i
 }
 
 // Iterates the work items of this CTA.  Every role walks the same sequence.
+//
+// A ragged sampling call (P_dev set) has no whole-unit phase: the key tiles of every unit, entry
+// b's units taking tiles pre[b]..pre[b+1]-1, form one stream cut into equal contiguous ranges for
+// all gridDim.x CTAs; a CTA locates the unit of a tile by binary search over pre.
 template <int MODE>
 struct Scheduler {
     const FmhaParams& p;
+    const int* rg_pre;   // sample, ragged: prefix table in shared memory
     long long pos, end;  // sample: tile range of this CTA
+    long long total;     // sample: tiles of the split stream
+    int sgrid;           // sample: CTAs the split stream is cut over
     int k;               // train: next item index
 
-    __device__ Scheduler(const FmhaParams& prm) : p(prm) {
+    __device__ Scheduler(const FmhaParams& prm, const int* pre = nullptr) : p(prm), rg_pre(pre) {
         k = blockIdx.x;
         if (MODE == kDecoderSample) {
             const int c = static_cast<int>(blockIdx.x);
-            pos = c < p.split_ctas ? range_begin(c, p.total_tiles, p.split_ctas) : 0;
-            end = c < p.split_ctas ? range_begin(c + 1, p.total_tiles, p.split_ctas) : 0;
+            if (p.P_dev != nullptr) {
+                // every CTA of the stream gets at least one tile: CTAs past the tile count stay idle
+                total = rg_pre[p.batch];
+                sgrid = total < static_cast<long long>(gridDim.x) ? static_cast<int>(total) : static_cast<int>(gridDim.x);
+                pos = c < sgrid ? range_begin(c, total, sgrid) : 0;
+                end = c < sgrid ? range_begin(c + 1, total, sgrid) : 0;
+            } else {
+                total = p.total_tiles;
+                sgrid = p.split_ctas;
+                pos = c < p.split_ctas ? range_begin(c, p.total_tiles, p.split_ctas) : 0;
+                end = c < p.split_ctas ? range_begin(c + 1, p.total_tiles, p.split_ctas) : 0;
+            }
         }
     }
 
+    // Fills the sampling fields of unit u (prefix length P, Tu tiles, first stream tile ubeg).
+    __device__ void fill_sample(Item& it, int u, int P, int Tu, long long ubeg, long long seg_begin,
+                                long long seg_end) const {
+        const int qt = u % p.num_qtiles;
+        const int kvz = u / p.num_qtiles;  // b*Hkv + g
+        const int b = kvz / p.kv_heads, g = kvz % p.kv_heads;
+        it.q_z = u;
+        it.kv_z = kvz;
+        it.q_row0 = qt * kBlockM;
+        it.out_row0 = (b * p.q_heads + g * p.group) * p.S + qt * kBlockM;
+        it.q_y = it.out_row0;
+        it.nact = 1;
+        it.n1 = ceil_div_i(p.S, kBlockN);
+        it.a1 = 0;
+        it.n0 = ceil_div_i(P, kBlockN);
+        it.a1q[0] = it.a1q[1] = 0;
+        it.e1q[0] = it.e1q[1] = it.n1;
+        it.n0q[0] = it.n0q[1] = it.n0;
+        it.t_begin = static_cast<int>(seg_begin - ubeg);
+        it.t_end = static_cast<int>(seg_end - ubeg);
+        it.P = P;
+        it.tu = Tu;
+        it.ubeg = ubeg;
+        it.total = total;
+        it.sgrid = sgrid;
+    }
+
     __device__ bool next(Item& it) {
+        if (MODE == kDecoderSample && p.P_dev != nullptr) {
+            if (pos >= end) return false;
+            int lo = 0, hi = p.batch;  // pre[lo] <= pos < pre[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (rg_pre[mid] <= pos) lo = mid;
+                else hi = mid;
+            }
+            const int UB = p.rg_units_per_entry;
+            const int Tu = (rg_pre[lo + 1] - rg_pre[lo]) / UB;
+            const int u_in = static_cast<int>((pos - rg_pre[lo]) / Tu);
+            const long long ubeg = rg_pre[lo] + static_cast<long long>(u_in) * Tu;
+            const long long seg_end = (end < ubeg + Tu) ? end : ubeg + Tu;
+            fill_sample(it, lo * UB + u_in, ragged_clamp(__ldg(p.P_dev + lo), p.rg_capacity), Tu, ubeg, pos, seg_end);
+            pos = seg_end;
+            return true;
+        }
         if (MODE == kDecoderSample) {
             const int Tu = p.tiles_per_unit;
             int u;
@@ -244,23 +353,7 @@ struct Scheduler {
             } else {
                 return false;
             }
-            const int qt = u % p.num_qtiles;
-            const int kvz = u / p.num_qtiles;  // b*Hkv + g
-            const int b = kvz / p.kv_heads, g = kvz % p.kv_heads;
-            it.q_z = u;
-            it.kv_z = kvz;
-            it.q_row0 = qt * kBlockM;
-            it.out_row0 = (b * p.q_heads + g * p.group) * p.S + qt * kBlockM;
-            it.q_y = it.out_row0;
-            it.nact = 1;
-            it.n1 = ceil_div_i(p.S, kBlockN);
-            it.a1 = 0;
-            it.n0 = ceil_div_i(p.P, kBlockN);
-            it.a1q[0] = it.a1q[1] = 0;
-            it.e1q[0] = it.e1q[1] = it.n1;
-            it.n0q[0] = it.n0q[1] = it.n0;
-            it.t_begin = static_cast<int>(pos - ubeg);
-            it.t_end = static_cast<int>(seg_end - ubeg);
+            fill_sample(it, u, p.P, Tu, ubeg, pos, seg_end);
             if (pos < end) pos = seg_end;
             return true;
         } else {
@@ -320,7 +413,7 @@ __device__ __forceinline__ TileRef tile_of(const FmhaParams& p, const Item& it, 
     } else {
         r.src = 0;
         r.kt = t - it.n1;
-        const int len = (MODE == kDecoderSample) ? p.P : p.L;
+        const int len = (MODE == kDecoderSample) ? it.P : p.L;
         r.nk16 = round16(min(kBlockN, len - r.kt * kBlockN));
         r.box_rows = kBlockN;
     }
@@ -542,6 +635,8 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);                        \
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);             \
     volatile int* bcast = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 16);                 \
+    int* rg_pre = reinterpret_cast<int*>(smem + SM::OFF_RG);                                         \
+    (void)rg_pre;                                                                                    \
     (void)k_full; (void)v_full; (void)kv_empty; (void)q_full; (void)q_empty; (void)s_full;           \
     (void)p_full; (void)pv_done; (void)o_free; (void)mma_drain; (void)tmem_holder; (void)abort_flag; \
     (void)softmax_done;                                                                              \
@@ -574,6 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         ptx::tmem_alloc(tmem_holder, kTmemCols);
         ptx::tmem_relinquish();
     }
+    if (MODE == kDecoderSample && p.P_dev != nullptr) ragged_prefix(p, rg_pre, rg_pre + kRaggedMaxBatch + 1);
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -602,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             }
         }
         __syncwarp();
-        Scheduler<MODE> sched(p);
+        Scheduler<MODE> sched(p, rg_pre);
         Item it;
         uint32_t kv_iter = 0, item_idx = 0;
         bool ok = true;
@@ -675,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         // The whole warp walks the schedule, so descriptors and TMEM addresses are warp-uniform;
         // one elected lane issues tcgen05.mma / tcgen05.commit.
         const bool leader = ptx::elect_one();
-        Scheduler<MODE> sched(p);
+        Scheduler<MODE> sched(p, rg_pre);
         Item it;
         uint32_t kv_iter = 0, item_idx = 0;
         uint32_t qtile[NQ], qitem[NQ];
@@ -796,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         ptx::setmaxnreg_dec<kRegsControl>();
         // Warps 2-3: the cache write of an encoder block step (sampling calls only), else idle.
         if (MODE == kDecoderSample && p.app_dst_k != nullptr) {
-            Scheduler<MODE> sched(p);
+            Scheduler<MODE> sched(p, rg_pre);
             Item it;
             while (sched.next(it))
                 if (it.t_begin == 0 && it.q_row0 == 0) append_block_rows(p, D, it.kv_z, threadIdx.x - 64, 64);
@@ -815,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         const uint32_t wg_bar = 1 + q;               // named barrier of this warpgroup
         const float sl2 = p.scale_log2;
         if (q < NQ) {
-            Scheduler<MODE> sched(p);
+            Scheduler<MODE> sched(p, rg_pre);
             Item it;
             uint32_t qtile = 0, qitem = 0;
             while (sched.next(it)) {
@@ -831,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 if (MODE == kDecoderSample) {
                     row_valid = prow < kBlockM && qrow < p.rows_per_unit;
                     lo0 = 0;
-                    hi0 = row_valid ? p.P : 0;
+                    hi0 = row_valid ? it.P : 0;
                     lo1 = 0;
                     hi1 = row_valid ? p.S : 0;
                 } else {
@@ -902,6 +998,23 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         // tcgen05.ld/st are warp-collective: the warp rescales if any row needs it.
                         if (__any_sync(0xffffffffu, rescale)) rescale_tmem_cols<D>(o_tmem, rescale ? alpha : 1.f);
                     }
+                    if (MODE == kDecoderSample && p.P_dev != nullptr && tr.src == 0 && it.P - k0 < tr.nk16) {
+                        // Ragged prefix: cache rows at or past P[b] in this tile may hold anything (NaN
+                        // included) and P.V would meet them with p = 0; zero those V rows of the stage.
+                        const uint32_t vst = qtile % C::NST;
+                        wait_bar_warp(&v_full[vst], (qtile / C::NST) & 1u, abort_flag, p.err);
+                        const int vrow = quarter * 32 + lane;
+                        if (vrow >= it.P - k0 && vrow < tr.nk16) {
+#pragma unroll
+                            for (int ch = 0; ch < C::NCH; ++ch) {
+                                uint4* dst = reinterpret_cast<uint4*>(smem + SM::OFF_V + vst * C::TILE_BYTES +
+                                                                      ch * C::CHUNK_BYTES + vrow * C::RB);
+#pragma unroll
+                                for (int u = 0; u < C::RB / 16; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
+                            }
+                        }
+                        ptx::fence_proxy_async_smem();
+                    }
                     ptx::tmem_wait_st();
                     ptx::tc_fence_before();
                     ptx::mbar_arrive(&p_full[q * NSB + sbuf]);
@@ -915,16 +1028,16 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 const float lse_val = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
                 constexpr int CW = D < 32 ? D : 32;  // columns per step
                 __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
-                const int Tu = p.tiles_per_unit;
+                const int Tu = it.tu;
                 const bool whole = (MODE != kDecoderSample) || (it.t_begin == 0 && it.t_end == Tu);
                 float* slot = nullptr;
                 int c_first = 0, c_last = 0;
                 long long ubeg = 0;
                 if (MODE == kDecoderSample && !whole) {
-                    ubeg = static_cast<long long>(it.q_z) * Tu;
-                    c_first = owner_cta(ubeg, p.total_tiles, p.split_ctas);
-                    c_last = owner_cta(ubeg + Tu - 1, p.total_tiles, p.split_ctas);
-                    const int my_slot = (range_begin(blockIdx.x, p.total_tiles, p.split_ctas) >= ubeg)
+                    ubeg = it.ubeg;
+                    c_first = owner_cta(ubeg, it.total, it.sgrid);
+                    c_last = owner_cta(ubeg + Tu - 1, it.total, it.sgrid);
+                    const int my_slot = (range_begin(blockIdx.x, it.total, it.sgrid) >= ubeg)
                                             ? 2 * blockIdx.x
                                             : 2 * blockIdx.x + 1;
                     slot = p.ws_partial + static_cast<size_t>(my_slot) * p.slot_floats;
@@ -1002,8 +1115,8 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     if (is_last) {
                         __threadfence();
                         if (row_valid && prow < p.rows_cap) {
-                            const long long T = p.total_tiles;
-                            const int grid = p.split_ctas;
+                            const long long T = it.total;
+                            const int grid = it.sgrid;
                             auto slot_ptr = [&](int c) -> const float* {
                                 const int si = (range_begin(c, T, grid) >= ubeg) ? 2 * c : 2 * c + 1;
                                 return p.ws_partial + static_cast<size_t>(si) * p.slot_floats;

@@ -226,6 +226,49 @@ E2D2_API e2d2_status e2d2_attn_encoder_block_step(const void* q_blk, void* k_cac
                                                   size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Sampling step with ragged prefixes: as e2d2_attn_decoder_sample, but batch entry b has decoded
+ * its own number of clean tokens, P_dev[b] ([E2D2 notes, sec. 3]: the cache grows per decoded
+ * block; "Block Diffusion: Interpolating Between Autoregressive and Diffusion Language Models",
+ * sec. 3: sequences of any length, so entries of one batch sit at different block boundaries, or
+ * off them after prompts of different lengths).  Entry b's S queries attend to rows
+ * 0..P_dev[b]-1 of its own cache and to its own block.
+ *   P_dev: DEVICE array of batch ints (4-byte aligned), read by the kernel; each value is clamped
+ *   to [0, capacity].  Cache rows at or past P_dev[b] are never used (they may hold anything).
+ *   Other arguments, layouts and the workspace as for e2d2_attn_decoder_sample; batch <= 256
+ *   (E2D2_ERR_SHAPE otherwise); a NULL P_dev is E2D2_ERR_INVALID_ARG.
+ *   Work split: the key tiles of every (entry, kv head, query tile) unit form one stream cut into
+ *   equal contiguous ranges over min(SMs, 256, tiles) CTAs (entry b's units take
+ *   ceil(S/128) + ceil(P_dev[b]/128) tiles each); partials of units that straddle CTAs are merged
+ *   as in the single-prefix call.
+ */
+E2D2_API e2d2_status e2d2_attn_decoder_sample_ragged(const void* q_blk, const void* k_cache, const void* v_cache,
+                                                     int capacity, const int* P_dev, const void* k_blk,
+                                                     const void* v_blk, void* out, float* lse, e2d2_dims dims, int S,
+                                                     void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Work plan of a ragged sampling call for host copies of the prefix lengths (P_host, batch ints)
+ * on a GPU with num_sms SMs.  Needs no GPU; launches nothing.
+ *   kernel: as in e2d2_sample_plan; units = batch * units_per_entry; total_tiles = the length of
+ *   the stream (sum over entries of units_per_entry * (ceil(S/128) + ceil(P/128)), P clamped to
+ *   [0, capacity]); grid = CTAs launched = min(num_sms, 256).  The stream is cut over
+ *   G = min(grid, total_tiles) CTAs, CTA c < G taking stream tiles [c * total / G, (c + 1) * total / G)
+ *   (so each at least one); CTAs c >= G take nothing.
+ * Returns E2D2_ERR_INVALID_ARG for NULL pointers, bad dims, S <= 0, capacity < 0 or num_sms <= 0,
+ * E2D2_ERR_SHAPE for batch > 256.
+ */
+typedef struct {
+    int kernel;
+    int units;
+    int units_per_entry;
+    long long total_tiles;
+    int grid;
+} e2d2_ragged_plan;
+
+E2D2_API e2d2_status e2d2_attn_decoder_sample_ragged_plan(e2d2_dims dims, int S, const int* P_host, int capacity,
+                                                          int num_sms, e2d2_ragged_plan* plan);
+
+/*
  * KV-cache append ([E2D2 notes, sec. 3]: after a block is decoded the encoder absorbs it and
  * the cache grows by that block): rows P..P+S_new-1 of every (batch, kv head) cache take the
  * rows of k_new / v_new, bit for bit.  k_new, v_new [batch][kv_heads][S_new][d].  The cache

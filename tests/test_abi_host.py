@@ -160,3 +160,17 @@ def test_product_package_never_imports_the_oracle():
         src = p.read_text()
         assert "import block_discrete_diffusion_tcgen05_b200" not in src, p
         assert "from block_discrete_diffusion_tcgen05_b200" not in src, p
+
+
+def test_ragged_sample_argument_errors(lib):
+    f = lib.e2d2_attn_decoder_sample_ragged
+    dims = _lib.Dims(2, 4, 2, 128, 0.0)
+    ws = lib.e2d2_attn_decoder_sample_workspace(dims, 16, 64)
+    # (q_blk, k_cache, v_cache, capacity, P_dev, k_blk, v_blk, out, lse, dims, S, workspace, ws_bytes, stream)
+    assert f(P16, P16, P16, 64, None, P16, P16, P16, None, dims, 16, P16, ws, None) == 1       # P is required
+    assert f(P16, P16, P16, 64, P16 + 2, P16, P16, P16, None, dims, 16, P16, ws, None) == 4   # misaligned P
+    assert f(P16, P16, P16, 64, P16, P16, P16, P16, None, _lib.Dims(257, 4, 2, 128, 0.0), 16, P16, ws, None) == 3
+    assert f(P16, None, P16, 64, P16, P16, P16, P16, None, dims, 16, P16, ws, None) == 1      # null cache
+    assert f(P16, P16, P16, 64, P16, P16, P16, P16, None, dims, 16, P16, ws - 1, None) == 6   # small workspace
+    assert f(P16, P16, P16, -1, P16, P16, P16, P16, None, dims, 16, P16, ws, None) == 1       # capacity < 0
+

@@ -76,7 +76,7 @@ def test_every_wrapped_call_is_declared():
     for name in ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train", "e2d2_attn_encoder_backward",
                  "e2d2_attn_decoder_train_backward", "e2d2_attn_decoder_sample", "e2d2_attn_encoder_block_step",
                  "e2d2_kv_cache_append", "e2d2_attn_train_backward_workspace",
-                 "e2d2_attn_decoder_sample_workspace"):
+                 "e2d2_attn_decoder_sample_workspace", "e2d2_attn_decoder_sample_ragged"):
         assert name in PARAMS, name
 
 
@@ -170,3 +170,19 @@ def test_kv_cache_append(rec):
     assert (a["k_cache"], a["v_cache"], a["k_new"], a["v_new"]) == tuple(t.data_ptr() for t in (kc, vc, kn, vn))
     assert (a["capacity"], a["P"], a["S_new"], a["stream"]) == (cap, P, Sn, STREAM)
     check_dims(a["dims"], B, Hkv, Hkv, d, None)
+
+
+def test_decoder_sample_ragged(rec):
+    Ss, cap = 16, 80
+    qb, kc, vc = bf16(B, Hq, Ss, d), bf16(B, Hkv, cap, d), bf16(B, Hkv, cap, d)
+    kb, vb = bf16(B, Hkv, Ss, d), bf16(B, Hkv, Ss, d)
+    P = torch.tensor([3, 80][:B], dtype=torch.int32)
+    ws = torch.zeros(1024)
+    out, lse = attn.decoder_sample_ragged(qb, kc, vc, P, kb, vb, workspace=ws, scale=0.5)
+    a = rec.call("e2d2_attn_decoder_sample_ragged")
+    assert (a["q_blk"], a["k_cache"], a["v_cache"], a["P_dev"], a["k_blk"], a["v_blk"]) == tuple(
+        t.data_ptr() for t in (qb, kc, vc, P, kb, vb))
+    assert a["capacity"] == cap and a["S"] == Ss and a["stream"] == STREAM
+    assert a["out"] == out.data_ptr() and a["lse"] == lse.data_ptr()
+    assert a["workspace"] == ws.data_ptr() and a["ws_bytes"] == ws.numel() * 4
+    check_dims(a["dims"], B, Hq, Hkv, d, 0.5)

@@ -128,3 +128,95 @@ def test_sample_workspace_holds_two_slots_per_cta():
         ws = attn.sample_workspace_bytes(B, Hkv * G, Hkv, d, S, 4096)
         rows = min(G * S, 128)
         assert ws >= 1024 + 2 * MAX_CTAS * rows * (d + 2) * 4
+
+
+# ---------------------------------------------------------------------------------------------
+# Ragged prefixes (e2d2_attn_decoder_sample_ragged): one stream-K stream over every unit's tiles,
+# entry b's units taking ceil(S/128) + ceil(P[b]/128) tiles each, cut into equal contiguous
+# ranges over all launched CTAs.
+# ---------------------------------------------------------------------------------------------
+def ragged_walk(P, S, upe, cap, grid):
+    """The schedule as the kernels walk it: per-entry prefix, binary search for a tile's entry,
+    unit = entry's units in order, the stream cut over min(grid, tiles) CTAs.  Returns (taken per
+    tile, partial writers per unit, prefix, tiles, CTAs of the stream)."""
+    per_entry = [upe * (-(-S // 128) + -(-min(max(p, 0), cap) // 128)) for p in P]
+    pre = np.concatenate([[0], np.cumsum(per_entry)]).astype(np.int64)
+    T = int(pre[-1])
+    grid = min(grid, T)   # CTAs past the tile count take nothing
+    taken = np.zeros(T, dtype=np.int64)
+    writers = {}
+    for c in range(grid):
+        start, end = range_begin(c, T, grid), range_begin(c + 1, T, grid)
+        pos, slots = start, set()
+        while pos < end:
+            b = int(np.searchsorted(pre, pos, side="right") - 1)   # pre[b] <= pos < pre[b+1]
+            Tu = (int(pre[b + 1]) - int(pre[b])) // upe
+            u_in = (pos - int(pre[b])) // Tu
+            u, ubeg = b * upe + u_in, int(pre[b]) + u_in * Tu
+            seg_end = min(end, ubeg + Tu)
+            taken[pos:seg_end] += 1
+            if not (pos == ubeg and seg_end == ubeg + Tu):
+                slot = 2 * c if start >= ubeg else 2 * c + 1
+                assert slot not in slots, "two partial units of one CTA share a slot"
+                slots.add(slot)
+                writers.setdefault(u, set()).add(c)
+                # the merge ticket arithmetic of the kernels
+                c_first, c_last = owner_cta(ubeg, T, grid), owner_cta(ubeg + Tu - 1, T, grid)
+                assert c_first <= c <= c_last
+            pos = seg_end
+        assert len(slots) <= 2
+    return taken, writers, pre, T, grid
+
+
+RAGGED_CASES = [
+    # B, Hq, Hkv, d, S, cap, P, sms
+    (6, 16, 8, 128, 16, 1040, [0, 1040, 17, 128, 1000, 513], 148),
+    (4, 8, 2, 64, 16, 600, [5, 600, 256, 0], 148),
+    (2, 8, 1, 128, 16, 400, [300, 77], 148),
+    (32, 16, 8, 128, 16, 2064, [(67 * b) % 2065 for b in range(32)], 148),
+    (3, 4, 4, 32, 130, 5000, [4999, 1, 2560], 13),
+    (1, 2, 1, 64, 1, 0, [0], 148),
+    (256, 2, 1, 128, 16, 300, [(7 * b) % 301 for b in range(256)], 148),
+    (5, 32, 8, 128, 16, 8192, [8192, 8176, 0, 16, 4000], 148),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,S,cap,P,sms", RAGGED_CASES)
+def test_ragged_plan_covers_every_tile_once(B, Hq, Hkv, d, S, cap, P, sms):
+    plan = attn.sample_ragged_plan(B, Hq, Hkv, d, S, P, cap, sms)
+    G = Hq // Hkv
+    GS = G * S
+    kernel = 0 if (d != 128 or GS > 64) else (16 if GS <= 16 else 32 if GS <= 32 else 64)
+    qtiles = 1 if kernel else -(-GS // 128)
+    assert plan["kernel"] == kernel
+    assert plan["units_per_entry"] == Hkv * qtiles and plan["units"] == B * Hkv * qtiles
+    assert plan["grid"] == min(sms, MAX_CTAS)
+    taken, writers, pre, T, G = ragged_walk(P, S, plan["units_per_entry"], cap, plan["grid"])
+    assert plan["total_tiles"] == T
+    assert (taken == 1).all(), "a key tile taken twice or never"
+    for u, ctas in writers.items():
+        b, Tu = u // plan["units_per_entry"], None
+        Tu = (int(pre[b + 1]) - int(pre[b])) // plan["units_per_entry"]
+        ubeg = int(pre[b]) + (u % plan["units_per_entry"]) * Tu
+        c_first, c_last = owner_cta(ubeg, T, G), owner_cta(ubeg + Tu - 1, T, G)
+        assert ctas == set(range(c_first, c_last + 1)), "merge ticket count disagrees with the writers"
+
+
+def test_ragged_plan_clamps_and_refuses():
+    lib = _lib.load()
+    # values outside [0, capacity] are clamped
+    a = attn.sample_ragged_plan(2, 4, 2, 128, 16, [-5, 10_000], 300, 148)
+    b = attn.sample_ragged_plan(2, 4, 2, 128, 16, [0, 300], 300, 148)
+    assert a == b
+    plan = _lib.RaggedPlan()
+    ref = _lib.ctypes.byref(plan)
+    arr = (_lib.ctypes.c_int * 2)(1, 2)
+    good = _lib.Dims(2, 4, 2, 128, 0.0)
+    assert lib.e2d2_attn_decoder_sample_ragged_plan(good, 16, None, 64, 148, ref) == 1
+    assert lib.e2d2_attn_decoder_sample_ragged_plan(good, 16, arr, 64, 148, None) == 1
+    assert lib.e2d2_attn_decoder_sample_ragged_plan(good, 0, arr, 64, 148, ref) == 1
+    assert lib.e2d2_attn_decoder_sample_ragged_plan(good, 16, arr, -1, 148, ref) == 1
+    assert lib.e2d2_attn_decoder_sample_ragged_plan(good, 16, arr, 64, 0, ref) == 1
+    big = (_lib.ctypes.c_int * 257)()
+    assert lib.e2d2_attn_decoder_sample_ragged_plan(_lib.Dims(257, 4, 2, 128, 0.0), 16, big, 64, 148, ref) == 3
+    assert lib.e2d2_attn_decoder_sample_ragged_plan(good, 16, arr, 64, 148, ref) == 0
