@@ -4,15 +4,18 @@ library is missing, importing the attention calls fails loudly."""
 from __future__ import annotations
 
 import ctypes
+import os
 from pathlib import Path
 
 PKG = Path(__file__).resolve().parent
 LIBRARY = PKG / "libe2d2_attn.so"
+# E2D2_DEBUG=1 selects the build with device-side bounds checks (E2D2_ERR_DEVICE_CHECK)
+DEBUG_LIBRARY = PKG / "libe2d2_attn_debug.so"
 
 # Names and values of include/e2d2_attn.h's e2d2_status.
 STATUS = {0: "E2D2_OK", 1: "E2D2_ERR_INVALID_ARG", 2: "E2D2_ERR_UNSUPPORTED", 3: "E2D2_ERR_SHAPE",
           4: "E2D2_ERR_ALIGNMENT", 5: "E2D2_ERR_CAPACITY", 6: "E2D2_ERR_WORKSPACE",
-          7: "E2D2_ERR_CUDA", 8: "E2D2_ERR_TIMEOUT"}
+          7: "E2D2_ERR_CUDA", 8: "E2D2_ERR_TIMEOUT", 9: "E2D2_ERR_DEVICE_CHECK"}
 
 EXPORTS = ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
            "e2d2_attn_decoder_sample_workspace", "e2d2_attn_decoder_sample",
@@ -20,7 +23,8 @@ EXPORTS = ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
            "e2d2_attn_decoder_sample_noalloc", "e2d2_attn_encoder_block_step",
            "e2d2_attn_train_backward_workspace", "e2d2_attn_encoder_backward",
            "e2d2_attn_decoder_train_backward", "e2d2_attn_decoder_sample_plan",
-           "e2d2_attn_decoder_sample_ragged", "e2d2_attn_decoder_sample_ragged_plan")
+           "e2d2_attn_decoder_sample_ragged", "e2d2_attn_decoder_sample_ragged_plan",
+           "e2d2_debug_set_wait_test")
 
 # E2D2_SAMPLE_NOALLOC_MAX_BYTES of include/e2d2_attn.h
 SAMPLE_NOALLOC_MAX_BYTES = 32 << 20
@@ -62,7 +66,10 @@ def load(path: Path | str | None = None):
     global _lib
     if _lib is not None and path is None:
         return _lib
-    p = Path(path) if path is not None else LIBRARY
+    if path is not None:
+        p = Path(path)
+    else:
+        p = DEBUG_LIBRARY if os.environ.get("E2D2_DEBUG", "0") not in ("", "0") else LIBRARY
     if not p.exists():
         raise ImportError(f"{p} is missing: build it with `python -m block_discrete_diffusion_tcgen05_b200.build`"
                           " (or __graft_entry__.build()); there is no CPU fallback")
@@ -97,6 +104,8 @@ def load(path: Path | str | None = None):
     lib.e2d2_status_string.argtypes = [ci]
     lib.e2d2_status_string.restype = ctypes.c_char_p
     lib.e2d2_last_device_error.argtypes = [st]
+    lib.e2d2_debug_set_wait_test.argtypes = [ctypes.c_ulonglong, ctypes.c_ulonglong]
+    lib.e2d2_debug_set_wait_test.restype = ctypes.c_int
     for name in ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
                  "e2d2_attn_decoder_sample", "e2d2_kv_cache_append", "e2d2_last_device_error",
                  "e2d2_version", "e2d2_attn_encoder_backward", "e2d2_attn_decoder_train_backward"):

@@ -10,6 +10,8 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIBRARY = PKG / "libe2d2_attn.so"
+# the same library with device-side bounds checks (E2D2_DEBUG): selected by E2D2_DEBUG=1
+DEBUG_LIBRARY = PKG / "libe2d2_attn_debug.so"
 SOURCES = [CSRC / "e2d2_api.cu"]
 HEADERS = sorted(CSRC.glob("*.cuh")) + [ROOT / "include" / "e2d2_attn.h"]
 
@@ -26,24 +28,32 @@ def nvcc() -> str:
     return str(cand) if cand.exists() else "nvcc"
 
 
-def up_to_date() -> bool:
-    if not LIBRARY.exists():
+def up_to_date(lib: Path = LIBRARY) -> bool:
+    if not lib.exists():
         return False
-    t = LIBRARY.stat().st_mtime
+    t = lib.stat().st_mtime
     return all(p.stat().st_mtime <= t for p in SOURCES + HEADERS)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> Path:
-    if not force and up_to_date():
-        return LIBRARY
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", str(ROOT / "include"), "-I", str(CSRC),
-           *map(str, SOURCES), "-o", str(LIBRARY)]
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = False) -> Path:
+    """Builds the library (debug=True: the E2D2_DEBUG variant with device bounds checks)."""
+    lib = DEBUG_LIBRARY if debug else LIBRARY
+    if not force and up_to_date(lib):
+        return lib
+    flags = ["-DE2D2_DEBUG"] if debug else []
+    cmd = [nvcc(), *NVCC_FLAGS, *flags, *extra, "-I", str(ROOT / "include"), "-I", str(CSRC),
+           *map(str, SOURCES), "-o", str(lib)]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    return LIBRARY
+    return lib
+
+
+def build_all(force: bool = False, verbose: bool = False) -> None:
+    build(force=force, verbose=verbose)
+    build(force=force, verbose=verbose, debug=True)
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
+          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [], debug="--debug" in sys.argv)

@@ -470,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             }
         }
         __syncwarp();
+        test_producer_delay();
         BwdScheduler<SIDE> sched(p);
         BwdItem it;
         uint32_t n = 0, iw = 0;
@@ -479,6 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             const uint32_t rb = iw % RBUF;
             ok = wait_bar_warp(&row_empty[rb], ((iw / RBUF) & 1) ^ 1, abort_flag, p.err);
             if (!ok) break;
+            // debug builds: the row tile starts inside the sequence and its head exists
+            E2D2_DCHECK(it.row0 < p.L && it.row_z < p.batch * (SIDE == kBwdRowsQ ? p.q_heads : p.kv_heads), p.err);
             if (leader) {
                 const int rs = (SIDE == kBwdRowsQ) ? 0 : it.src;
                 ptx::mbar_arrive_expect_tx(&row_full[rb], 2 * C::ROW_TILE);
@@ -510,6 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
                 ok = wait_bar_warp(&col_empty[st], ((n / NST) & 1) ^ 1, abort_flag, p.err);
                 if (!ok) break;
                 const BwdCol cr = bwd_col<SIDE>(it, t);
+                E2D2_DCHECK(cr.y < p.L && cr.z < p.batch * (SIDE == kBwdRowsQ ? p.kv_heads : p.q_heads), p.err);
                 if (leader) {
                     const uint32_t bytes = 2 * C::COL_TILE + (SIDE == kBwdRowsKV ? 2 * kBwdCols * 4 : 0);
                     ptx::mbar_arrive_expect_tx(&col_full[st], bytes);
@@ -536,10 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
         // Never leave with copies in flight: wait for the last load of every buffer.
         volatile int no_abort = 0;
         for (uint32_t i = n > static_cast<uint32_t>(NST) ? n - NST : 0u; i < n; ++i)
-            wait_bar_warp(&col_full[i % NST], (i / NST) & 1u, &no_abort, p.err);
+            wait_bar_warp(&col_full[i % NST], (i / NST) & 1u, &no_abort, p.err, true);
         for (uint32_t i = iw > static_cast<uint32_t>(RBUF) ? iw - RBUF : 0u; i < iw; ++i)
-            wait_bar_warp(&row_full[i % RBUF], (i / RBUF) & 1u, &no_abort, p.err);
-        if (SIDE == kBwdRowsQ && iw > 0) wait_bar_warp(out_full, (iw - 1) & 1u, &no_abort, p.err);
+            wait_bar_warp(&row_full[i % RBUF], (i / RBUF) & 1u, &no_abort, p.err, true);
+        if (SIDE == kBwdRowsQ && iw > 0) wait_bar_warp(out_full, (iw - 1) & 1u, &no_abort, p.err, true);
     } else if (warp == 1) {
         ptx::setmaxnreg_dec<kRegsControl>();
         // ------------------------------------------------------------------ product issuer
@@ -595,9 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
         if (leader) ptx::mma_commit(mma_drain);
         __syncwarp();
         volatile int no_abort = 0;
-        wait_bar_warp(mma_drain, 0, &no_abort, p.err);
-        wait_bar_warp(acc_drain, 0, &no_abort, p.err);
-        wait_bar_warp(softmax_done, 0, &no_abort, p.err);
+        wait_bar_warp(mma_drain, 0, &no_abort, p.err, true);
+        wait_bar_warp(acc_drain, 0, &no_abort, p.err, true);
+        wait_bar_warp(softmax_done, 0, &no_abort, p.err, true);
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, kTmemCols);
     } else if (warp == 2) {

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -365,6 +366,16 @@ struct SamplePlan {
     long long grid;      // CTAs launched
 };
 
+// E2D2_SPLITS=n (read once per process): CTAs of the split phase, for tests of split-count
+// independence; clamped to what the schedule supports.  0 or unset: the heuristic below.
+int split_override() {
+    static const int v = [] {
+        const char* e = std::getenv("E2D2_SPLITS");
+        return e ? std::atoi(e) : 0;
+    }();
+    return v;
+}
+
 SamplePlan plan_sample(const e2d2_dims& dims, int S, int P, int sms) {
     SamplePlan pl;
     const int D = dims.head_dim;
@@ -386,6 +397,8 @@ SamplePlan plan_sample(const e2d2_dims& dims, int S, int P, int sms) {
     constexpr long long kMinSplitTiles = 6;
     long long sc = R * 5 < grid ? R * 5 : grid;
     if (sc > R * Tu / kMinSplitTiles) sc = R * Tu / kMinSplitTiles;
+    if (sc < R) sc = R;
+    if (split_override() > 0 && R > 0) sc = split_override() < grid ? split_override() : grid;
     if (sc < R) sc = R;
     if (sc > R * Tu) sc = R * Tu;
     pl.split_ctas = static_cast<int>(sc);
@@ -545,6 +558,7 @@ const char* e2d2_status_string(e2d2_status s) {
         case E2D2_ERR_WORKSPACE: return "E2D2_ERR_WORKSPACE";
         case E2D2_ERR_CUDA: return "E2D2_ERR_CUDA";
         case E2D2_ERR_TIMEOUT: return "E2D2_ERR_TIMEOUT";
+        case E2D2_ERR_DEVICE_CHECK: return "E2D2_ERR_DEVICE_CHECK";
     }
     return "E2D2_ERR_UNKNOWN";
 }
@@ -723,8 +737,19 @@ e2d2_status e2d2_last_device_error(cudaStream_t stream) {
     if (word != 0) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return E2D2_ERR_CUDA;
-        return E2D2_ERR_TIMEOUT;
+        return (word & kErrDeviceCheck) ? E2D2_ERR_DEVICE_CHECK : E2D2_ERR_TIMEOUT;
     }
+    return E2D2_OK;
+}
+
+e2d2_status e2d2_debug_set_wait_test(unsigned long long wait_limit_ns, unsigned long long producer_delay_ns) {
+    DeviceInfo* di = nullptr;
+    const e2d2_status s = device_info(&di);
+    if (s != E2D2_OK) return s;
+    const unsigned long long limit = wait_limit_ns ? wait_limit_ns : kWaitTimeoutNs;
+    if (cudaMemcpyToSymbol(g_wait_limit_ns, &limit, sizeof(limit)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_test_producer_delay_ns, &producer_delay_ns, sizeof(producer_delay_ns)) != cudaSuccess)
+        return E2D2_ERR_CUDA;
     return E2D2_OK;
 }
 

@@ -243,6 +243,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
             }
         }
         __syncwarp();
+        test_producer_delay();
         const int NS = is_k ? C::NK : C::NV;
         uint64_t* full = is_k ? k_full : v_full;
         uint64_t* empty = is_k ? k_empty : v_empty;
@@ -270,6 +271,9 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 ok = wait_bar_warp(&empty[st], ((iter / NS) & 1) ^ 1, abort_flag, p.err);
                 if (!ok) break;
                 const TileRef tr = tile_of<kDecoderSample>(p, it, t);
+                // debug builds: the tile starts inside its source and the kv unit exists
+                E2D2_DCHECK(tr.kt * kBlockN < (tr.src ? p.S : it.P), p.err);
+                E2D2_DCHECK(it.kv_z >= 0 && it.kv_z < p.batch * p.kv_heads, p.err);
                 if (leader) {
                     const CUtensorMap* m = is_k ? (tr.src ? &p.tm_k1 : &p.tm_k0) : (tr.src ? &p.tm_v1 : &p.tm_v0);
                     ptx::mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(tr.box_rows) * D * 2);
@@ -284,10 +288,10 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         // Never leave with copies in flight.
         volatile int no_abort = 0;
         for (uint32_t i = iter > static_cast<uint32_t>(NS) ? iter - NS : 0u; i < iter; ++i)
-            wait_bar_warp(&full[i % NS], (i / NS) & 1u, &no_abort, p.err);
+            wait_bar_warp(&full[i % NS], (i / NS) & 1u, &no_abort, p.err, true);
         if (is_k)
             for (uint32_t i = item_idx > 2u ? item_idx - 2u : 0u; i < item_idx; ++i)
-                wait_bar_warp(&q_full[i & 1], (i >> 1) & 1u, &no_abort, p.err);
+                wait_bar_warp(&q_full[i & 1], (i >> 1) & 1u, &no_abort, p.err, true);
     } else if (warp == 1) {
         ptx::setmaxnreg_dec<kKrRegsControl>();
         E2D2_KR_POINTERS
@@ -335,9 +339,9 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         if (leader) ptx::mma_commit(qk_drain);
         __syncwarp();
         volatile int no_abort = 0;
-        wait_bar_warp(qk_drain, 0, &no_abort, p.err);
-        wait_bar_warp(pv_drain, 0, &no_abort, p.err);
-        wait_bar_warp(tmem_done, 0, &no_abort, p.err);
+        wait_bar_warp(qk_drain, 0, &no_abort, p.err, true);
+        wait_bar_warp(pv_drain, 0, &no_abort, p.err, true);
+        wait_bar_warp(tmem_done, 0, &no_abort, p.err, true);
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
     } else if (warp == 3) {

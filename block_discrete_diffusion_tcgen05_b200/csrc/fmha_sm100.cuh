@@ -57,8 +57,22 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int kSampleMaxCtas = 256;     // upper bound of the sampling grid (workspace sizing)
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 
-// Bit set in the device error word when a bounded wait gives up.
+// Bits of the device error word: a bounded wait gave up; a debug-build bounds check failed.
 constexpr unsigned int kErrWaitTimeout = 1u;
+constexpr unsigned int kErrDeviceCheck = 2u;
+
+// Debug builds (E2D2_DEBUG): device-side bounds checks that record kErrDeviceCheck in the error
+// word and carry on (TMA coordinates past a tensor's extent read zeros, so nothing faults).
+#ifdef E2D2_DEBUG
+#define E2D2_DCHECK(cond, err)                                  \
+    do {                                                        \
+        if (!(cond)) atomicOr((err), e2d2::kErrDeviceCheck);     \
+    } while (0)
+#else
+#define E2D2_DCHECK(cond, err) \
+    do {                       \
+    } while (0)
+#endif
 
 struct alignas(64) FmhaParams {
     CUtensorMap tm_q;   // kEncoder/kDecoderTrain: 3D {D, L, B*Hq}; kDecoderSample: 2D {D, B*Hq*S}
@@ -420,17 +434,28 @@ __device__ __forceinline__ TileRef tile_of(const FmhaParams& p, const Item& it, 
     return r;
 }
 
+// Limit of the pipeline waits (device variable, so that a test can shorten it without a rebuild;
+// see e2d2_debug_set_wait_test) and a delay the producers of the next launches take before their
+// first load (0 outside that test).
+__device__ unsigned long long g_wait_limit_ns = kWaitTimeoutNs;
+__device__ unsigned long long g_test_producer_delay_ns = 0;
+
 // Bounded mbarrier wait.  Returns false (and flags the CTA and the device error word) if the
-// phase does not complete within kWaitTimeoutNs or another role already gave up.  The thread
-// sleeps inside try_wait (up to 1 ms per attempt) rather than spinning.
+// phase does not complete within the limit or another role already gave up.  The thread sleeps
+// inside try_wait (up to 1 ms per attempt) rather than spinning.  Pipeline waits use the
+// (test-adjustable) limit g_wait_limit_ns; drain waits (`drain`: the last copies of a producer,
+// the MMAs and roles that must be done before tensor memory is freed) always allow kWaitTimeoutNs,
+// so a shortened limit never frees resources that are still in use.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         unsigned int* err) {
+                                         unsigned int* err, bool drain = false) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
+    unsigned long long limit = kWaitTimeoutNs + 0ull;
+    if (!drain) limit = *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
     const uint64_t t0 = ptx::globaltimer_ns();
     for (;;) {
         if (ptx::mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
         if (*abort_flag) return false;
-        if (ptx::globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        if (ptx::globaltimer_ns() - t0 > limit) {
             *abort_flag = 1;
             atomicOr(err, kErrWaitTimeout);
             return false;
@@ -441,9 +466,17 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 // Warp-collective form of wait_bar: every lane returns the same answer, so the .sync.aligned
 // tcgen05 instructions that follow are always executed by the whole warp.
 __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              unsigned int* err) {
-    const bool ok = wait_bar(bar, parity, abort_flag, err);
+                                              unsigned int* err, bool drain = false) {
+    const bool ok = wait_bar(bar, parity, abort_flag, err, drain);
     return __all_sync(0xffffffffu, ok);
+}
+
+// Test hook: the producer sleeps for g_test_producer_delay_ns before its first load (bounded).
+__device__ __forceinline__ void test_producer_delay() {
+    const unsigned long long delay = *reinterpret_cast<volatile unsigned long long*>(&g_test_producer_delay_ns);
+    if (delay == 0) return;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (ptx::globaltimer_ns() - t0 < delay) __nanosleep(100000);
 }
 
 // Byte offset of 16-byte unit `u` of row `r` inside one swizzled chunk (row pitch RB bytes).
@@ -698,6 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             }
         }
         __syncwarp();
+        test_producer_delay();
         Scheduler<MODE> sched(p, rg_pre);
         Item it;
         uint32_t kv_iter = 0, item_idx = 0;
@@ -707,6 +741,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             const uint32_t qround = item_idx / C::QBUF;
             ok = wait_bar_warp(&q_empty[qb], (qround & 1) ^ 1, abort_flag, p.err);
             if (!ok) break;
+            E2D2_DCHECK(MODE == kDecoderSample ? (it.q_z < p.batch * p.kv_heads * p.num_qtiles && it.q_row0 < p.rows_per_unit)
+                                               : (it.q_z < p.batch * p.q_heads && it.q_y < p.L),
+                        p.err);
             if (leader) {
                 if (MODE == kDecoderSample) {
                     // The packed rows are spread over the four TMEM lane quarters: rows
@@ -736,6 +773,11 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 ok = wait_bar_warp(&kv_empty[st], (round & 1) ^ 1, abort_flag, p.err);
                 if (!ok) break;
                 const TileRef tr = tile_of<MODE>(p, it, t);
+                // debug builds: the tile starts inside its source and the kv unit exists
+                E2D2_DCHECK(tr.kt * kBlockN < (tr.src ? (MODE == kDecoderSample ? p.S : p.L)
+                                                      : (MODE == kDecoderSample ? it.P : p.L)),
+                            p.err);
+                E2D2_DCHECK(it.kv_z >= 0 && it.kv_z < p.batch * p.kv_heads, p.err);
                 if (leader) {
                     const CUtensorMap* mk = tr.src ? &p.tm_k1 : &p.tm_k0;
                     const CUtensorMap* mv = tr.src ? &p.tm_v1 : &p.tm_v0;
@@ -760,11 +802,11 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         volatile int no_abort = 0;
         const uint32_t first_live = kv_iter > static_cast<uint32_t>(C::NST) ? kv_iter - C::NST : 0u;
         for (uint32_t i = first_live; i < kv_iter; ++i) {
-            wait_bar_warp(&k_full[i % C::NST], (i / C::NST) & 1u, &no_abort, p.err);
-            wait_bar_warp(&v_full[i % C::NST], (i / C::NST) & 1u, &no_abort, p.err);
+            wait_bar_warp(&k_full[i % C::NST], (i / C::NST) & 1u, &no_abort, p.err, true);
+            wait_bar_warp(&v_full[i % C::NST], (i / C::NST) & 1u, &no_abort, p.err, true);
         }
         for (uint32_t i = item_idx > static_cast<uint32_t>(C::QBUF) ? item_idx - C::QBUF : 0u; i < item_idx; ++i)
-            wait_bar_warp(&q_full[i % C::QBUF], (i / C::QBUF) & 1u, &no_abort, p.err);
+            wait_bar_warp(&q_full[i % C::QBUF], (i / C::QBUF) & 1u, &no_abort, p.err, true);
     } else if (warp == 1) {
         ptx::setmaxnreg_dec<kRegsControl>();
         // ------------------------------------------------------------------ MMA issuer
@@ -884,8 +926,8 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         if (leader) ptx::mma_commit(mma_drain);
         __syncwarp();
         volatile int no_abort = 0;
-        wait_bar_warp(mma_drain, 0, &no_abort, p.err);
-        wait_bar_warp(softmax_done, 0, &no_abort, p.err);
+        wait_bar_warp(mma_drain, 0, &no_abort, p.err, true);
+        wait_bar_warp(softmax_done, 0, &no_abort, p.err, true);
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, kTmemCols);
     } else if (warp < 4) {

@@ -58,7 +58,8 @@ typedef enum {
     E2D2_ERR_CAPACITY = 5,    /* P + S_new > capacity, or P > capacity                      */
     E2D2_ERR_WORKSPACE = 6,   /* workspace missing or smaller than the _workspace query     */
     E2D2_ERR_CUDA = 7,        /* a CUDA runtime / driver call failed                        */
-    E2D2_ERR_TIMEOUT = 8      /* a bounded device-side wait gave up (see e2d2_last_device_error) */
+    E2D2_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up (see e2d2_last_device_error) */
+    E2D2_ERR_DEVICE_CHECK = 9 /* debug library: a device-side bounds check failed              */
 } e2d2_status;
 
 typedef struct {
@@ -174,6 +175,9 @@ E2D2_API e2d2_status e2d2_attn_decoder_sample(const void* q_blk, const void* k_c
  * over split_ctas CTAs, whose fp32 partials the last CTA to finish a unit merges in CTA order.
  *   kernel: 0 = the generic kernel, 16/32/64 = the kernel with keys on the tensor-memory lanes
  *   and that many packed query columns (head_dim 128 and G*S <= 64).
+ * The environment variable E2D2_SPLITS=n (read once per process) sets the split phase's CTA count
+ * to n, clamped to [split_units, min(grid, split_units * tiles_per_unit)], in this plan and in the
+ * calls alike: a test knob for split-count independence.
  * Returns E2D2_ERR_INVALID_ARG for a NULL plan, bad dims, S <= 0, P < 0 or num_sms <= 0.
  */
 typedef struct {
@@ -283,9 +287,24 @@ E2D2_API const char* e2d2_status_string(e2d2_status status);
 
 /*
  * Synchronises `stream`, then reads and clears the device error word of the current device:
- * E2D2_OK, or E2D2_ERR_TIMEOUT if a bounded device-side wait gave up since the last read.
+ * E2D2_OK; E2D2_ERR_DEVICE_CHECK if, in the debug library (built with E2D2_DEBUG, loaded by the
+ * Python binding when the environment variable E2D2_DEBUG=1), a device-side bounds check on a
+ * TMA coordinate or a work-unit index failed; else E2D2_ERR_TIMEOUT if a bounded device-side wait
+ * gave up since the last read.  After either, outputs of the affected calls are undefined and
+ * sampling workspaces must be zero-filled again.
  */
 E2D2_API e2d2_status e2d2_last_device_error(cudaStream_t stream);
+
+/*
+ * Test hook for the failure path, not for production use.  On the current device, pipeline waits
+ * of later launches give up after wait_limit_ns (default 2 s) and every kernel's load producer
+ * first sleeps for producer_delay_ns (default 0), so that a test can make the bounded waits run
+ * out without any fault: the kernels then unwind (waits that guard freeing tensor memory or copies
+ * in flight keep the 2 s limit), return, and e2d2_last_device_error() reports E2D2_ERR_TIMEOUT.
+ * (0, 0) restores the defaults.  Synchronous; returns E2D2_ERR_CUDA if the device is unusable.
+ */
+E2D2_API e2d2_status e2d2_debug_set_wait_test(unsigned long long wait_limit_ns,
+                                              unsigned long long producer_delay_ns);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 E2D2_API int e2d2_version(void);

@@ -174,3 +174,17 @@ def test_ragged_sample_argument_errors(lib):
     assert f(P16, P16, P16, 64, P16, P16, P16, P16, None, dims, 16, P16, ws - 1, None) == 6   # small workspace
     assert f(P16, P16, P16, -1, P16, P16, P16, P16, None, dims, 16, P16, ws, None) == 1       # capacity < 0
 
+
+def test_debug_library_exports_every_declared_symbol():
+    """The E2D2_DEBUG build (device-side bounds checks) has the same C ABI."""
+    dbg = _lib.load(build.build(debug=True))
+    for name in header_functions():
+        assert hasattr(dbg, name), name
+    dbg.e2d2_status_string.restype = ctypes.c_char_p
+    assert dbg.e2d2_status_string(9) == b"E2D2_ERR_DEVICE_CHECK"
+
+
+def test_status_strings_cover_every_status(lib):
+    for code, name in _lib.STATUS.items():
+        assert lib.e2d2_status_string(code).decode() == name
+

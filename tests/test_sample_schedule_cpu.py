@@ -220,3 +220,41 @@ def test_ragged_plan_clamps_and_refuses():
     big = (_lib.ctypes.c_int * 257)()
     assert lib.e2d2_attn_decoder_sample_ragged_plan(_lib.Dims(257, 4, 2, 128, 0.0), 16, big, 64, 148, ref) == 3
     assert lib.e2d2_attn_decoder_sample_ragged_plan(good, 16, arr, 64, 148, ref) == 0
+
+
+_OVERRIDE = r"""
+import sys
+sys.path.insert(0, {root!r})
+from block_discrete_diffusion_tcgen05_b200 import attn
+for args in ((4, 32, 8, 128, 16, 2000, 148), (32, 16, 8, 128, 16, 2048, 148), (2, 8, 2, 64, 40, 5000, 13)):
+    print(repr(attn.sample_plan(*args)))
+"""
+
+
+@pytest.mark.parametrize("splits", ["1", "7", "32", "100", "1000"])
+def test_split_override_plans_stay_valid(splits):
+    """E2D2_SPLITS=n (read once per process) sets the split phase's CTA count, clamped to what the
+    schedule supports; every overridden plan still takes each tile once with correct merges."""
+    import os
+    import subprocess
+    import sys
+    from pathlib import Path
+
+    root = Path(__file__).resolve().parents[1]
+    res = subprocess.run([sys.executable, "-c", _OVERRIDE.format(root=str(root))], capture_output=True, text=True,
+                         env=dict(os.environ, E2D2_SPLITS=splits), timeout=300)
+    assert res.returncode == 0, res.stderr
+    for line in res.stdout.splitlines():
+        plan = eval(line)
+        R, Tu = plan["split_units"], plan["tiles_per_unit"]
+        if R:
+            want = max(R, min(int(splits), min(148, 256)))
+            assert plan["split_ctas"] == min(want, R * Tu, max(plan["grid"], R)), plan
+        taken, partial_ctas = walk(plan)
+        assert (taken == 1).all()
+        T = R * Tu
+        for u, ctas in partial_ctas.items():
+            if ctas:
+                c_first = owner_cta(u * Tu, T, plan["split_ctas"])
+                c_last = owner_cta(u * Tu + Tu - 1, T, plan["split_ctas"])
+                assert ctas == set(range(c_first, c_last + 1))
