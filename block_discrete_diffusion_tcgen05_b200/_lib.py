@@ -24,7 +24,7 @@ EXPORTS = ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
            "e2d2_attn_train_backward_workspace", "e2d2_attn_encoder_backward",
            "e2d2_attn_decoder_train_backward", "e2d2_attn_decoder_sample_plan",
            "e2d2_attn_decoder_sample_ragged", "e2d2_attn_decoder_sample_ragged_plan",
-           "e2d2_debug_set_wait_test")
+           "e2d2_debug_set_wait_test", "e2d2_kv_cache_append_ragged")
 
 # E2D2_SAMPLE_NOALLOC_MAX_BYTES of include/e2d2_attn.h
 SAMPLE_NOALLOC_MAX_BYTES = 32 << 20
@@ -49,7 +49,7 @@ class RaggedPlan(ctypes.Structure):
     """e2d2_ragged_plan."""
 
     _fields_ = [("kernel", ctypes.c_int), ("units", ctypes.c_int), ("units_per_entry", ctypes.c_int),
-                ("total_tiles", ctypes.c_longlong), ("grid", ctypes.c_int)]
+                ("total_tiles", ctypes.c_longlong), ("grid", ctypes.c_int), ("stream_ctas", ctypes.c_int)]
 
 
 class E2D2Error(RuntimeError):
@@ -83,6 +83,8 @@ def load(path: Path | str | None = None):
     lib.e2d2_attn_decoder_sample.argtypes = [vp, vp, vp, ci, ci, vp, vp, vp, fp, Dims, ci, vp,
                                              ctypes.c_size_t, st]
     lib.e2d2_kv_cache_append.argtypes = [vp, vp, ci, ci, vp, vp, ci, Dims, st]
+    lib.e2d2_kv_cache_append_ragged.argtypes = [vp, vp, ci, vp, vp, vp, ci, Dims, st]
+    lib.e2d2_kv_cache_append_ragged.restype = ctypes.c_int
     lib.e2d2_attn_encoder_block_step.argtypes = [vp, vp, vp, ci, ci, vp, vp, vp, fp, Dims, ci, vp,
                                                  ctypes.c_size_t, st]
     lib.e2d2_attn_decoder_sample_noalloc.argtypes = [vp, vp, vp, ci, ci, vp, vp, vp, fp, Dims, ci, st]

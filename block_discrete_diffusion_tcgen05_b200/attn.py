@@ -335,6 +335,25 @@ def kv_cache_append(k_cache, v_cache, P: int, k_new, v_new):
     return P + S_new
 
 
+@_device_guard
+def kv_cache_append_ragged(k_cache, v_cache, P, k_new, v_new):
+    """Writes k_new/v_new [B,Hkv,S_new,d] into rows P[b]..P[b]+S_new-1 of entry b's caches, P a
+    CUDA int32 tensor [B] (not advanced: the caller adds S_new when the block is final)."""
+    lib = _lib.load()
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (k_new, "k_new"), (v_new, "v_new")):
+        _need(t, n)
+    _need(P, "P", dtype=torch.int32, ndim=1)
+    B, Hkv, cap, d = k_cache.shape
+    S_new = k_new.shape[2]
+    if k_new.shape != (B, Hkv, S_new, d) or v_new.shape != k_new.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if P.shape != (B,):
+        raise ValueError("P must be [B]")
+    st = lib.e2d2_kv_cache_append_ragged(k_cache.data_ptr(), v_cache.data_ptr(), cap, P.data_ptr(), k_new.data_ptr(),
+                                         v_new.data_ptr(), S_new, _dims(B, Hkv, Hkv, d, None), _stream(k_cache))
+    _lib.check(st, "e2d2_kv_cache_append_ragged")
+
+
 def last_device_error(device=None) -> int:
     lib = _lib.load()
     return int(lib.e2d2_last_device_error(torch.cuda.current_stream(device).cuda_stream))

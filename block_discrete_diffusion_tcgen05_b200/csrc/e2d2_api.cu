@@ -693,17 +693,24 @@ e2d2_status e2d2_attn_decoder_sample_ragged_plan(e2d2_dims dims, int S, const in
     plan->units_per_entry = upe;
     plan->total_tiles = total;
     plan->grid = num_sms < kSampleMaxCtas ? num_sms : kSampleMaxCtas;
+    long long g = total / kMinRaggedTiles;
+    if (g < plan->units) g = plan->units;
+    if (g > plan->grid) g = plan->grid;
+    if (g > total) g = total;
+    plan->stream_ctas = static_cast<int>(g);
     return E2D2_OK;
 }
 
-e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int P, const void* k_new,
-                                 const void* v_new, int S_new, e2d2_dims dims, cudaStream_t stream) {
+namespace {
+e2d2_status append_call(void* k_cache, void* v_cache, int capacity, int P, const int* P_dev, const void* k_new,
+                        const void* v_new, int S_new, const e2d2_dims& dims, cudaStream_t stream) {
     if (!k_cache || !v_cache || !k_new || !v_new) return E2D2_ERR_INVALID_ARG;
     e2d2_status s = check_dims(dims);
     if (s != E2D2_OK) return s;
     if (P < 0 || S_new < 0 || capacity < 0) return E2D2_ERR_INVALID_ARG;
     if (static_cast<long long>(P) + S_new > capacity) return E2D2_ERR_CAPACITY;
-    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new))
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new) ||
+        (reinterpret_cast<uintptr_t>(P_dev) & 3u))
         return E2D2_ERR_ALIGNMENT;
     if (S_new == 0) return E2D2_OK;
     DeviceInfo* di = nullptr;
@@ -719,12 +726,27 @@ e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int
     a.S_new = S_new;
     a.vec_per_row = dims.head_dim / 8;
     a.units = dims.batch * dims.kv_heads;
+    a.P_dev = P_dev;
+    a.kv_heads = dims.kv_heads;
     const long long total = static_cast<long long>(a.units) * S_new * a.vec_per_row;
     long long blocks = (total + 255) / 256;
     const long long cap_blocks = static_cast<long long>(di->sms) * 8;
     if (blocks > cap_blocks) blocks = cap_blocks;
     kv_append_kernel<<<dim3(static_cast<unsigned>(blocks), 2), 256, 0, stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+}
+}  // namespace
+
+e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int P, const void* k_new,
+                                 const void* v_new, int S_new, e2d2_dims dims, cudaStream_t stream) {
+    return append_call(k_cache, v_cache, capacity, P, nullptr, k_new, v_new, S_new, dims, stream);
+}
+
+e2d2_status e2d2_kv_cache_append_ragged(void* k_cache, void* v_cache, int capacity, const int* P_dev,
+                                        const void* k_new, const void* v_new, int S_new, e2d2_dims dims,
+                                        cudaStream_t stream) {
+    if (!P_dev) return E2D2_ERR_INVALID_ARG;
+    return append_call(k_cache, v_cache, capacity, 0, P_dev, k_new, v_new, S_new, dims, stream);
 }
 
 e2d2_status e2d2_last_device_error(cudaStream_t stream) {

@@ -119,6 +119,7 @@ struct alignas(64) FmhaParams {
 };
 
 constexpr int kRaggedMaxBatch = 256;  // entries of a ragged sampling call (one per thread of the prefix scan)
+constexpr int kMinRaggedTiles = 6;    // tiles per CTA the ragged split aims for
 
 __host__ __device__ __forceinline__ int ragged_clamp(int P, int capacity) {
     return P < 0 ? 0 : (P > capacity ? capacity : P);
@@ -290,9 +291,16 @@ struct Scheduler {
         if (MODE == kDecoderSample) {
             const int c = static_cast<int>(blockIdx.x);
             if (p.P_dev != nullptr) {
-                // every CTA of the stream gets at least one tile: CTAs past the tile count stay idle
+                // CTAs of the stream: one per unit at least, more while every CTA keeps about
+                // kMinRaggedTiles tiles (a partial costs more than streaming a few tiles), never
+                // more than the grid or the tile count (every CTA of the stream gets a tile)
                 total = rg_pre[p.batch];
-                sgrid = total < static_cast<long long>(gridDim.x) ? static_cast<int>(total) : static_cast<int>(gridDim.x);
+                const long long units = static_cast<long long>(p.batch) * p.rg_units_per_entry;
+                long long g = total / kMinRaggedTiles;
+                if (g < units) g = units;
+                if (g > gridDim.x) g = gridDim.x;
+                if (g > total) g = total;
+                sgrid = static_cast<int>(g);
                 pos = c < sgrid ? range_begin(c, total, sgrid) : 0;
                 end = c < sgrid ? range_begin(c + 1, total, sgrid) : 0;
             } else {

@@ -241,7 +241,7 @@ E2D2_API e2d2_status e2d2_attn_encoder_block_step(const void* q_blk, void* k_cac
  *   Other arguments, layouts and the workspace as for e2d2_attn_decoder_sample; batch <= 256
  *   (E2D2_ERR_SHAPE otherwise); a NULL P_dev is E2D2_ERR_INVALID_ARG.
  *   Work split: the key tiles of every (entry, kv head, query tile) unit form one stream cut into
- *   equal contiguous ranges over min(SMs, 256, tiles) CTAs (entry b's units take
+ *   equal contiguous ranges over up to min(SMs, 256) CTAs (entry b's units take
  *   ceil(S/128) + ceil(P_dev[b]/128) tiles each); partials of units that straddle CTAs are merged
  *   as in the single-prefix call.
  */
@@ -256,8 +256,9 @@ E2D2_API e2d2_status e2d2_attn_decoder_sample_ragged(const void* q_blk, const vo
  *   kernel: as in e2d2_sample_plan; units = batch * units_per_entry; total_tiles = the length of
  *   the stream (sum over entries of units_per_entry * (ceil(S/128) + ceil(P/128)), P clamped to
  *   [0, capacity]); grid = CTAs launched = min(num_sms, 256).  The stream is cut over
- *   G = min(grid, total_tiles) CTAs, CTA c < G taking stream tiles [c * total / G, (c + 1) * total / G)
- *   (so each at least one); CTAs c >= G take nothing.
+ *   stream_ctas = min(grid, total_tiles, max(units, total_tiles / 6)) CTAs (at least one per unit,
+ *   about six tiles each beyond that, at least one tile each), CTA c < stream_ctas taking stream
+ *   tiles [c * total / stream_ctas, (c + 1) * total / stream_ctas); the other CTAs take nothing.
  * Returns E2D2_ERR_INVALID_ARG for NULL pointers, bad dims, S <= 0, capacity < 0 or num_sms <= 0,
  * E2D2_ERR_SHAPE for batch > 256.
  */
@@ -267,6 +268,7 @@ typedef struct {
     int units_per_entry;
     long long total_tiles;
     int grid;
+    int stream_ctas;
 } e2d2_ragged_plan;
 
 E2D2_API e2d2_status e2d2_attn_decoder_sample_ragged_plan(e2d2_dims dims, int S, const int* P_host, int capacity,
@@ -281,6 +283,19 @@ E2D2_API e2d2_status e2d2_attn_decoder_sample_ragged_plan(e2d2_dims dims, int S,
 E2D2_API e2d2_status e2d2_kv_cache_append(void* k_cache, void* v_cache, int capacity, int P,
                                  const void* k_new, const void* v_new, int S_new, e2d2_dims dims,
                                  cudaStream_t stream);
+
+/*
+ * KV-cache append with ragged lengths: as e2d2_kv_cache_append, but batch entry b's new rows go
+ * to rows P_dev[b]..P_dev[b]+S_new-1 of its own caches (P_dev: DEVICE array of batch ints,
+ * 4-byte aligned, read by the kernel; each value clamped to [0, capacity]).  Rows that would land
+ * at or past capacity are not written (keep P_dev[b] + S_new <= capacity).  The lengths stay with
+ * the caller, on the device: the call does not advance P_dev.  A NULL P_dev is
+ * E2D2_ERR_INVALID_ARG.  With P_dev on the device, a sequence of sampling and append calls can be
+ * captured once in a CUDA graph and replayed for every block.
+ */
+E2D2_API e2d2_status e2d2_kv_cache_append_ragged(void* k_cache, void* v_cache, int capacity, const int* P_dev,
+                                                 const void* k_new, const void* v_new, int S_new, e2d2_dims dims,
+                                                 cudaStream_t stream);
 
 /* Human-readable name of a status code (static string). */
 E2D2_API const char* e2d2_status_string(e2d2_status status);

@@ -188,3 +188,15 @@ def test_status_strings_cover_every_status(lib):
     for code, name in _lib.STATUS.items():
         assert lib.e2d2_status_string(code).decode() == name
 
+
+def test_ragged_append_argument_errors(lib):
+    f = lib.e2d2_kv_cache_append_ragged
+    dims = _lib.Dims(2, 2, 2, 128, 0.0)
+    # (k_cache, v_cache, capacity, P_dev, k_new, v_new, S_new, dims, stream)
+    assert f(P16, P16, 64, None, P16, P16, 16, dims, None) == 1        # P is required
+    assert f(P16, P16, 64, P16 + 2, P16, P16, 16, dims, None) == 4     # misaligned P
+    assert f(P16, P16, 64, P16, P16 + 8, P16, 16, dims, None) == 4     # misaligned rows
+    assert f(P16, P16, 8, P16, P16, P16, 16, dims, None) == 5          # S_new > capacity
+    assert f(P16, P16, 64, P16, P16, P16, -1, dims, None) == 1
+    assert f(P16, P16, 64, P16, P16, P16, 0, dims, None) == 0          # nothing to append
+

@@ -80,3 +80,29 @@ def test_ragged_sampling_workload_size_sampled_entries(oracle):
                                                     kb[0].f32[sl], vb[0].f32[sl])
         H.compare(out[sl], lse[sl], ref_o, ref_l, f"ragged sampling size entry {b} P {P[b]}")
     assert attn.last_device_error() == 0
+
+
+def test_ragged_append_is_bitwise_per_entry(oracle):
+    """e2d2_kv_cache_append_ragged: entry b's new rows land at rows P[b].. of its own caches, bit
+    for bit (the oracle's append per entry); rows that would pass the capacity are not written; all
+    other rows keep their bits."""
+    from block_discrete_diffusion_tcgen05_b200 import synth
+
+    B, Hkv, cap, d, S = 4, 2, 100, 128, 16
+    P = [0, 84, 37, 90]   # the last entry's rows 100..105 fall past the capacity
+    kc, vc = (synth.normal_bf16((B, Hkv, cap, d), 2100 + t) for t in range(2))
+    kn, vn = (synth.normal_bf16((B, Hkv, S, d), 2102 + t) for t in range(2))
+    kd, vd = synth.to_torch(kc, "cuda"), synth.to_torch(vc, "cuda")
+    attn.kv_cache_append_ragged(kd, vd, torch.tensor(P, dtype=torch.int32, device="cuda"),
+                                synth.to_torch(kn, "cuda"), synth.to_torch(vn, "cuda"))
+    torch.cuda.synchronize()
+    got_k = kd.cpu().view(torch.int16).numpy().view(np.uint16)
+    got_v = vd.cpu().view(torch.int16).numpy().view(np.uint16)
+    for b, pb in enumerate(P):
+        kb, vb = kc.bits[b:b + 1].copy(), vc.bits[b:b + 1].copy()
+        n = min(S, cap - pb)
+        if n == S:
+            oracle.kv_append(kb, vb, pb, kn.bits[b:b + 1], vn.bits[b:b + 1])
+        else:
+            kb[:, :, pb:pb + n], vb[:, :, pb:pb + n] = kn.bits[b:b + 1, :, :n], vn.bits[b:b + 1, :, :n]
+        assert np.array_equal(got_k[b:b + 1], kb) and np.array_equal(got_v[b:b + 1], vb), f"entry {b}"

@@ -135,6 +135,10 @@ def test_sample_workspace_holds_two_slots_per_cta():
 # entry b's units taking ceil(S/128) + ceil(P[b]/128) tiles each, cut into equal contiguous
 # ranges over all launched CTAs.
 # ---------------------------------------------------------------------------------------------
+def ragged_stream_ctas(T, units, grid):
+    return min(grid, T, max(units, T // 6))
+
+
 def ragged_walk(P, S, upe, cap, grid):
     """The schedule as the kernels walk it: per-entry prefix, binary search for a tile's entry,
     unit = entry's units in order, the stream cut over min(grid, tiles) CTAs.  Returns (taken per
@@ -142,7 +146,7 @@ def ragged_walk(P, S, upe, cap, grid):
     per_entry = [upe * (-(-S // 128) + -(-min(max(p, 0), cap) // 128)) for p in P]
     pre = np.concatenate([[0], np.cumsum(per_entry)]).astype(np.int64)
     T = int(pre[-1])
-    grid = min(grid, T)   # CTAs past the tile count take nothing
+    grid = ragged_stream_ctas(T, len(P) * upe, grid)   # the stream's CTAs; the others take nothing
     taken = np.zeros(T, dtype=np.int64)
     writers = {}
     for c in range(grid):
@@ -192,7 +196,7 @@ def test_ragged_plan_covers_every_tile_once(B, Hq, Hkv, d, S, cap, P, sms):
     assert plan["units_per_entry"] == Hkv * qtiles and plan["units"] == B * Hkv * qtiles
     assert plan["grid"] == min(sms, MAX_CTAS)
     taken, writers, pre, T, G = ragged_walk(P, S, plan["units_per_entry"], cap, plan["grid"])
-    assert plan["total_tiles"] == T
+    assert plan["total_tiles"] == T and plan["stream_ctas"] == G
     assert (taken == 1).all(), "a key tile taken twice or never"
     for u, ctas in writers.items():
         b, Tu = u // plan["units_per_entry"], None
