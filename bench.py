@@ -321,18 +321,39 @@ def run_workload_set(torch, attn, workloads, dev, peaks):
         for kc, vc in caches:
             attn.kv_cache_append(kc, vc, P, kn, vn)
 
-    for n in range(4):  # warm-up on the first blocks
-        block(16 * n)
+    # The loop as a serving engine runs it: prefix lengths on the device, one block (16 steps x 8
+    # sampling calls, 8 appends, the length update) captured once in a CUDA graph and replayed for
+    # every block, so no host work sits between the launches.
+    P_dev = torch.zeros(B, dtype=torch.int32, device=dev)
+
+    def block_dev():
+        for _ in range(steps_pb):
+            for kc, vc in caches:
+                attn.decoder_sample_ragged(qb, kc, vc, P_dev, kb, vb, workspace=ws, out=out, lse=lse)
+        for kc, vc in caches:
+            attn.kv_cache_append_ragged(kc, vc, P_dev, kn, vn)
+        P_dev.add_(Sb)
+
+    block_dev()  # first launches configure the kernels (not capturable)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        block_dev()
+    P_dev.zero_()
+    for _ in range(3):  # warm-up on the first blocks
+        graph.replay()
+    P_dev.zero_()
     torch.cuda.synchronize()
     quarters = 4
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(quarters + 1)]
     ev[0].record()
     for qi in range(quarters):
         for n in range(qi * nblocks // quarters, (qi + 1) * nblocks // quarters):
-            block(16 * n)
+            graph.replay()
         ev[qi + 1].record()
     torch.cuda.synchronize()
     q_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(quarters)]
+    del graph
     calls = steps_pb * layers
 
     def loop_bytes(n0, n1):
@@ -350,10 +371,26 @@ def run_workload_set(torch, attn, workloads, dev, peaks):
                         "us_per_sample_call": q_ms[qi] * 1e3 / ((n1 - n0) * calls)})
     total_ms = sum(q_ms)
     by = loop_bytes(0, nblocks)
+    # the first quarter again with eager launches from Python (host-bound), for comparison
+    for n in range(2):
+        block(16 * n)
+    torch.cuda.synchronize()
+    n_eager = nblocks // quarters
+    ev[0].record()
+    for n in range(n_eager):
+        block(16 * n)
+    ev[1].record()
+    torch.cuda.synchronize()
+    eager_ms = ev[0].elapsed_time(ev[1])
     res["long_sample_loop"] = {
         "workload": w["name"], "blocks": nblocks, "sample_calls": nblocks * calls, "appends": nblocks * layers,
         "ms_per_loop": total_ms, "gbs": by / (total_ms * 1e-3) / 1e9, "frac_hbm": by / (total_ms * 1e-3) / 1e9 / hbm,
-        "by_prefix_quarter": buckets, "launch": "eager (one Python call per kernel)"}
+        "by_prefix_quarter": buckets,
+        "launch": "CUDA graph of one block (128 ragged sampling calls, 8 ragged appends, length update) "
+                  "replayed per block; prefix lengths on the device",
+        "eager_first_quarter": {"P": [0, 16 * (n_eager - 1)], "ms": eager_ms,
+                                "us_per_sample_call": eager_ms * 1e3 / (n_eager * calls),
+                                "launch": "eager single-prefix calls from Python"}}
     del caches
     torch.cuda.empty_cache()
     return res
