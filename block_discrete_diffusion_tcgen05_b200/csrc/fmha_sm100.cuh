@@ -22,9 +22,13 @@
 //     P  = exp2(S*c - m)  softmax warpgroup, written back over S as bf16  -> TMEM
 //     O += P V            tcgen05.mma, A = P (TMEM), B = V (smem, MN-major) -> TMEM
 // Train calls take two 128-row query tiles per work item (one per softmax warpgroup) against
-// one shared K/V stream, and the MMA warp issues P.V(A, j-1), S(A, j), P.V(B, j-1), S(B, j):
-// while one warpgroup computes exponentials the other waits for its tensor-core work, so
-// the exponential unit and the tensor core stay busy (ping-pong).  The sampling call (shapes the
+// one shared K/V stream.  At head_dim <= 64 the S of both query tiles rotate through three TMEM
+// buffers (S number n in buffer n % 3): S(n) is issued as soon as P.V(n-3) has freed its buffer,
+// so a warpgroup's next S is ready when it finishes the current P, and neither warpgroup waits
+// for the tensor core; the P.V are issued in order as their P arrive, and at the end of an item
+// all of them at once (the epilogue waits for the last).  At head_dim 128 (no TMEM for a third
+// buffer) the MMA warp issues P.V(A, j-1), S(A, j), P.V(B, j-1), S(B, j), one S buffer per query
+// tile.  The sampling call (shapes the
 // keys-on-lanes kernel of fmha_keyrow_sm100.cuh does not take) uses one query tile holding all
 // G*S packed rows of a kv head, with S double-buffered in TMEM instead.
 // Each thread owns one query row (its TMEM lane) and all 128 key columns of a tile, read from
@@ -174,9 +178,20 @@ struct Cfg {
     static constexpr bool SAMPLE = (MODE == kDecoderSample);
     static constexpr int NQ = SAMPLE ? 1 : 2;                 // query tiles per work item
     static constexpr int NSB = SAMPLE ? 2 : 1;                // S buffers per query tile
-    static constexpr int NOB = (D <= 64) ? 2 : 1;             // O accumulator sets per query tile
+    // Train calls at d <= 64 rotate three S buffers over both query tiles: S number n (counted
+    // over the item sequence, both tiles interleaved) lives in buffer n % 3, so a query tile's
+    // next S is computed while its softmax still works on the current one.  At d = 128 the two
+    // O accumulators leave room for two S buffers only (one per query tile, NSB = 1).
+    static constexpr bool ROT = !SAMPLE && D <= 64;
+    static constexpr int NSBUF = ROT ? 3 : NQ * NSB;          // S buffers in TMEM, 128 columns each
+    // s_full barriers: per S buffer, and with rotating buffers per (query tile, buffer), so that a
+    // barrier's phases are one softmax warpgroup's S in that buffer, which it consumes in order.
+    static constexpr int NSFULL = ROT ? NQ * 3 : NQ * NSB;
+    static constexpr int O_COL = ROT ? 384 : 256;             // first TMEM column of the O sets
+    static constexpr int NOB = ROT ? (D <= 32 ? 2 : 1) : (D <= 64 ? 2 : 1);  // O sets per query tile
+    static_assert(O_COL + NOB * NQ * D <= 512, "TMEM columns");
     static constexpr int QBUF = (D == 128) ? 1 : 2;           // Q buffer sets (double-buffered)
-    static constexpr int NST = SAMPLE ? (D == 128 ? 3 : (D == 64 ? 6 : 8)) : (D == 128 ? 2 : (D == 64 ? 3 : 6));
+    static constexpr int NST = SAMPLE ? (D == 128 ? 3 : (D == 64 ? 6 : 8)) : (D == 128 ? 2 : (D == 64 ? 4 : 6));
     static constexpr int RB = (D * 2 < 128) ? D * 2 : 128;  // bytes per smem row of one chunk
     static constexpr int NCH = D * 2 / RB;                   // column chunks per tile
     static constexpr uint32_t SWZ = (RB == 128) ? 2u : 4u;   // 128-byte / 64-byte swizzle
@@ -198,8 +213,8 @@ struct Smem {
     static constexpr int O_BYTES = C::STAGE_O ? C::NQ * C::TILE_BYTES : 0;
     static constexpr int OFF_BAR = OFF_O + O_BYTES;
     // barriers: k_full[NST], v_full[NST], kv_empty[NST], q_full[QBUF], q_empty[QBUF],
-    // s_full[NQ*NSB], p_full[NQ*NSB], pv_done[NQ], o_free[NOB*NQ], mma_drain, softmax_done
-    static constexpr int NBAR = 3 * C::NST + 2 * C::QBUF + 2 * C::NQ * C::NSB + C::NQ + C::NOB * C::NQ + 2;
+    // s_full[NSFULL], p_full[NSBUF], pv_done[NQ], o_free[NOB*NQ], mma_drain, softmax_done
+    static constexpr int NBAR = 3 * C::NST + 2 * C::QBUF + C::NSFULL + C::NSBUF + C::NQ + C::NOB * C::NQ + 2;
     static constexpr int OFF_MISC = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;
     // sampling: ragged prefix table pre[kRaggedMaxBatch + 1] and the scan's 8 warp sums
     static constexpr int OFF_RG = OFF_MISC + 64;
@@ -503,9 +518,10 @@ __device__ __forceinline__ uint32_t p_col(uint32_t ks) { return ks * 8; }
 struct PendingPV {
     bool have;
     bool first;        // first tile of its item: overwrite O, wait for the O buffer to be free
+    int q;             // query tile
     uint32_t st;       // K/V stage
     uint32_t round;    // stage round (v_full parity)
-    uint32_t qt;       // per-query-tile tile counter (p_full parity)
+    uint32_t qt;       // S buffer use: per-query-tile tile counter, or (rotating buffers) S number
     uint32_t qi;       // per-query-tile item counter (o_free parity, O buffer)
     uint32_t nk;       // keys in the tile (multiple of 16)
 };
@@ -518,16 +534,17 @@ __device__ __forceinline__ bool issue_pv(int q, const PendingPV& pv, uint64_t* p
                                          uint64_t* v_full, uint64_t* kv_empty, uint64_t* pv_done,
                                          volatile int* abort_flag, unsigned int* err, uint32_t tmem_base,
                                          uint32_t sV, uint64_t vdesc, uint32_t idesc_pv, int D, bool leader) {
-    const uint32_t sbuf = pv.qt % C::NSB;
-    if (!wait_bar_warp(&p_full[q * C::NSB + sbuf], (pv.qt / C::NSB) & 1, abort_flag, err)) return false;
+    const uint32_t sb = C::ROT ? pv.qt % 3 : q * C::NSB + pv.qt % C::NSB;
+    const uint32_t sph = C::ROT ? (pv.qt / 3) & 1 : (pv.qt / C::NSB) & 1;
+    if (!wait_bar_warp(&p_full[sb], sph, abort_flag, err)) return false;
     const uint32_t ob = pv.qi % C::NOB;
     if (pv.first && !wait_bar_warp(&o_free[ob * C::NQ + q], ((pv.qi / C::NOB) & 1) ^ 1, abort_flag, err))
         return false;
     if (!wait_bar_warp(&v_full[pv.st], pv.round & 1, abort_flag, err)) return false;
     ptx::tc_fence_after();
     if (leader) {
-        const uint32_t a_tmem = tmem_base + (q * C::NSB + sbuf) * 128;
-        const uint32_t d_tmem = tmem_base + 256 + (ob * C::NQ + q) * D;
+        const uint32_t a_tmem = tmem_base + sb * 128;
+        const uint32_t d_tmem = tmem_base + C::O_COL + (ob * C::NQ + q) * D;
         const uint32_t v_base = sV + pv.st * C::TILE_BYTES;
         for (uint32_t ks = 0; ks < pv.nk / 16; ++ks)
             ptx::mma_ts(d_tmem, a_tmem + p_col(ks), vdesc | ((v_base + ks * 16 * C::RB) >> 4), idesc_pv,
@@ -587,45 +604,52 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v, float scale) {
     return w;
 }
 
-// Loads the 128 S columns of this thread's row (one TMEM round trip), applies the row's key
-// interval [cmin, cmax) (tile-relative) and sets chunks without any allowed key in the warp to
-// -inf.  The loads are unconditional so that s has a single definition (no spills).  Returns the
-// chunks in which every row of the warp has all 32 keys (no -inf there).
-__device__ __forceinline__ uint32_t load_s_row(uint32_t s_tmem, uint32_t live, int cmin, int cmax, float (&s)[128]) {
+// Loads the 128 S columns of this thread's row (one TMEM round trip, eight 16-column loads),
+// applies the row's key interval [cmin, cmax) (tile-relative) and sets chunks without any allowed
+// key in the warp (live bit clear) to -inf.  The loads are unconditional so that s has a single
+// definition (no spills).  Returns the row maximum.
+__device__ __forceinline__ float load_s_row(uint32_t s_tmem, uint32_t live, int cmin, int cmax, float (&s)[128]) {
     uint32_t raw[128];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) ptx::tmem_ld32(s_tmem + 32 * a, &raw[32 * a]);
+    for (int h = 0; h < 8; ++h) ptx::tmem_ld16(s_tmem + 16 * h, *reinterpret_cast<uint32_t(*)[16]>(&raw[16 * h]));
     ptx::tmem_wait_ld();
     ptx::reg_fence<128>(raw);
 #pragma unroll
     for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c]);
-    uint32_t whole_bits = 0;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
         if (!(live & (1u << a))) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) s[32 * a + c] = -INFINITY;
-        } else {
-            const bool whole = (cmin <= 32 * a) && (cmax >= 32 * a + 32);
-            if (!__all_sync(0xffffffffu, whole)) {
+        } else if (!__all_sync(0xffffffffu, cmin <= 32 * a && cmax >= 32 * a + 32)) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int col = 32 * a + c;
-                    s[32 * a + c] = (col >= cmin && col < cmax) ? s[32 * a + c] : -INFINITY;
-                }
-            } else {
-                whole_bits |= 1u << a;
+            for (int c = 0; c < 32; ++c) {
+                const int col = 32 * a + c;
+                s[col] = (col >= cmin && col < cmax) ? s[col] : -INFINITY;
             }
         }
     }
-    return whole_bits;
+    // maximum as a tree: eight independent chains over 16 columns each, then 8 -> 3 -> 1
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = s[j];
+#pragma unroll
+    for (int c = 8; c < 120; c += 16)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = ptx::fmax3(acc[j], s[c + j], s[c + 8 + j]);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = fmaxf(acc[j], s[120 + j]);
+    return ptx::fmax3(ptx::fmax3(acc[0], acc[1], acc[2]), ptx::fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
 }
 
 // P = exp2(s * sl2 + neg_m) for the live chunks, packed to bf16 and stored over S (keys 32a..
 // 32a+31 -> columns 16a..16a+15); dead chunks below nchunks store zeros.  Returns the row sum.
-__device__ __forceinline__ float exp_store_row(uint32_t s_tmem, uint32_t live, uint32_t whole, int nchunks,
-                                               const float (&s)[128], float sl2, float neg_m) {
-    float sums[4] = {0.f, 0.f, 0.f, 0.f};
+// The arguments and the sums run on column pairs (packed fp32x2 FMA / add of sm_100), the
+// exponentials one by one.
+__device__ __forceinline__ float exp_store_row(uint32_t s_tmem, uint32_t live, int nchunks, const float (&s)[128],
+                                               float sl2, float neg_m) {
+    const float2 sl2v = make_float2(sl2, sl2), nm = make_float2(neg_m, neg_m);
+    float2 sums[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
         if (a < nchunks) {
@@ -633,10 +657,10 @@ __device__ __forceinline__ float exp_store_row(uint32_t s_tmem, uint32_t live, u
             if (live & (1u << a)) {
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float e0 = ptx::ex2(fmaf(s[32 * a + c], sl2, neg_m));
-                    const float e1 = ptx::ex2(fmaf(s[32 * a + c + 1], sl2, neg_m));
-                    sums[(c >> 1) & 3] += e0 + e1;
-                    pk[c / 2] = ptx::pack_bf16x2(e0, e1);
+                    const float2 x = __ffma2_rn(make_float2(s[32 * a + c], s[32 * a + c + 1]), sl2v, nm);
+                    const float2 e = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+                    sums[(c >> 1) & 1] = __fadd2_rn(sums[(c >> 1) & 1], e);
+                    pk[c / 2] = ptx::pack_bf16x2(e.x, e.y);
                 }
             } else {
 #pragma unroll
@@ -645,7 +669,8 @@ __device__ __forceinline__ float exp_store_row(uint32_t s_tmem, uint32_t live, u
             ptx::tmem_st16(s_tmem + p_col(2 * a), pk);
         }
     }
-    return (sums[0] + sums[1]) + (sums[2] + sums[3]);
+    const float2 t = __fadd2_rn(sums[0], sums[1]);
+    return t.x + t.y;
 }
 
 template <int D, int MODE>
@@ -667,9 +692,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
     uint64_t* kv_empty = bars + 2 * C::NST;                                                          \
     uint64_t* q_full = bars + 3 * C::NST;                                                            \
     uint64_t* q_empty = q_full + C::QBUF;                                                            \
-    uint64_t* s_full = q_empty + C::QBUF;  /* [q][sbuf] */                                           \
-    uint64_t* p_full = s_full + NQ * NSB;  /* [q][sbuf] */                                           \
-    uint64_t* pv_done = p_full + NQ * NSB; /* [q] */                                                 \
+    uint64_t* s_full = q_empty + C::QBUF;  /* [S buffer] or [q][S buffer] */                         \
+    uint64_t* p_full = s_full + C::NSFULL; /* [S buffer] */                                          \
+    uint64_t* pv_done = p_full + C::NSBUF; /* [q] */                                                 \
     uint64_t* o_free = pv_done + NQ;       /* [ob][q] */                                             \
     uint64_t* mma_drain = o_free + NOB * NQ;                                                         \
     uint64_t* softmax_done = mma_drain + 1; /* every softmax thread is finished with TMEM */        \
@@ -695,10 +720,8 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             ptx::mbar_init(&q_full[i], 1);
             ptx::mbar_init(&q_empty[i], 1);
         }
-        for (int i = 0; i < NQ * NSB; ++i) {
-            ptx::mbar_init(&s_full[i], 1);
-            ptx::mbar_init(&p_full[i], kSoftmaxThreads / 2);
-        }
+        for (int i = 0; i < C::NSFULL; ++i) ptx::mbar_init(&s_full[i], 1);
+        for (int i = 0; i < C::NSBUF; ++i) ptx::mbar_init(&p_full[i], kSoftmaxThreads / 2);
         for (int i = 0; i < NQ; ++i) ptx::mbar_init(&pv_done[i], 1);
         for (int i = 0; i < NOB * NQ; ++i) ptx::mbar_init(&o_free[i], kSoftmaxThreads / 2);
         ptx::mbar_init(mma_drain, 1);
@@ -836,99 +859,191 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         const uint64_t vdesc = ptx::smem_desc(0, C::CHUNK_BYTES, 8 * C::RB, C::SWZ);  // V: MN-major
         constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kBlockM, D, true);
         bool ok = true;
-        while (ok && sched.next(it)) {
-            const int qb = item_idx % C::QBUF;
-            ok = wait_bar_warp(&q_full[qb], (item_idx / C::QBUF) & 1, abort_flag, p.err);
-            if (!ok) break;
-            // A query tile that sits this item out gets its last P.V issued now.
+        if constexpr (C::ROT) {
+            // Rotating S buffers.  S number n goes to buffer n % 3, whose previous S (n - 3) is
+            // consumed by its P.V: that P.V is issued first (the tensor core runs one CTA's MMAs
+            // in order, so the P.V reads P before the new S overwrites it).  The P.V still owed
+            // are kept in issue order, at most three (f0 oldest).
+            PendingPV f0, f1, f2;
+            f0.have = f1.have = f2.have = false;
+            int nf = 0;
+            uint32_t seq = 0;
+            uint32_t qitem[NQ];
 #pragma unroll
-            for (int q = 0; q < NQ; ++q)
-                if (q >= it.nact && pend[q].have) {
-                    ok = ok && issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
+            for (int q = 0; q < NQ; ++q) qitem[q] = 0;
+            auto pop = [&]() -> bool {
+                const bool r = issue_pv<C>(f0.q, f0, p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
                                            tmem_base, sV, vdesc, idesc_pv, D, leader);
-                    pend[q].have = false;
-                }
-            if (!ok) break;
-            bool seen[NQ];
+                f0 = f1;
+                f1 = f2;
+                --nf;
+                return r;
+            };
+            while (ok && sched.next(it)) {
+                const int qb = item_idx % C::QBUF;
+                ok = wait_bar_warp(&q_full[qb], (item_idx / C::QBUF) & 1, abort_flag, p.err);
+                if (!ok) break;
+                bool seen[NQ];
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) seen[q] = false;
-            for (int t = it.t_begin; t < it.t_end && ok; ++t) {
-                const uint32_t st = kv_iter % C::NST;
-                const uint32_t round = kv_iter / C::NST;
-                // A P.V still pending on this stage (its query tile skipped the tiles since)
-                // must be issued now: the stage is reloaded only after it.
+                for (int q = 0; q < NQ; ++q) seen[q] = false;
+                for (int t = it.t_begin; t < it.t_end && ok; ++t) {
+                    const uint32_t st = kv_iter % C::NST;
+                    const uint32_t round = kv_iter / C::NST;
+                    // The stage is reloaded only after the P.V that still reads its old V.
+                    while (ok && ((nf > 0 && f0.st == st) || (nf > 1 && f1.st == st) || (nf > 2 && f2.st == st)))
+                        ok = pop();
+                    if (!ok) break;
+                    ok = wait_bar_warp(&k_full[st], round & 1, abort_flag, p.err);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const TileRef tr = tile_of<MODE>(p, it, t);
+                    const uint32_t idesc_qk = ptx::idesc_bf16_f32(kBlockM, tr.nk16, false);
+                    const uint32_t k_base = sK + st * C::TILE_BYTES;
+#pragma unroll
+                    for (int q = 0; q < NQ; ++q) {
+                        if (q >= it.nact || !tile_needed(it, q, t)) {
+                            if (leader) ptx::mbar_arrive(&kv_empty[st]);
+                            __syncwarp();
+                            continue;
+                        }
+                        while (ok && nf > 0 && f0.qt + 3 <= seq) ok = pop();
+                        if (!ok) break;
+                        const uint32_t sb = seq % 3;
+                        if (leader) {
+                            const uint32_t q_base = sQ + (qb * NQ + q) * C::TILE_BYTES;
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t off = (ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
+                                                     (ks % C::KSTEPS_PER_CHUNK) * 32;
+                                ptx::mma_ss(tmem_base + sb * 128, kdesc | ((q_base + off) >> 4),
+                                            kdesc | ((k_base + off) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
+                            }
+                            ptx::mma_commit(&s_full[q * 3 + sb]);
+                        }
+                        __syncwarp();
+                        PendingPV e;
+                        e.have = true;
+                        e.first = !seen[q];
+                        e.q = q;
+                        e.st = st;
+                        e.round = round;
+                        e.qt = seq;
+                        e.qi = qitem[q];
+                        e.nk = tr.nk16;
+                        if (nf == 0) f0 = e;
+                        else if (nf == 1) f1 = e;
+                        else f2 = e;
+                        ++nf;
+                        ++seq;
+                        seen[q] = true;
+                    }
+                    ++kv_iter;
+                }
 #pragma unroll
                 for (int q = 0; q < NQ; ++q)
-                    if (ok && pend[q].have && pend[q].st == st) {
-                        ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
-                                         tmem_base, sV, vdesc, idesc_pv, D, leader);
+                    if (q < it.nact) ++qitem[q];
+                if (leader) ptx::mma_commit(&q_empty[qb]);
+                __syncwarp();
+                ++item_idx;
+                // The item's last P.V go out as soon as their P is ready: the epilogues wait for
+                // them (left queued, they would wait for the next item's S).
+                while (ok && nf > 0) ok = pop();
+            }
+        } else {
+            while (ok && sched.next(it)) {
+                const int qb = item_idx % C::QBUF;
+                ok = wait_bar_warp(&q_full[qb], (item_idx / C::QBUF) & 1, abort_flag, p.err);
+                if (!ok) break;
+                // A query tile that sits this item out gets its last P.V issued now.
+    #pragma unroll
+                for (int q = 0; q < NQ; ++q)
+                    if (q >= it.nact && pend[q].have) {
+                        ok = ok && issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
+                                               tmem_base, sV, vdesc, idesc_pv, D, leader);
                         pend[q].have = false;
                     }
                 if (!ok) break;
-                ok = wait_bar_warp(&k_full[st], round & 1, abort_flag, p.err);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const TileRef tr = tile_of<MODE>(p, it, t);
-                const uint32_t idesc_qk = ptx::idesc_bf16_f32(kBlockM, tr.nk16, false);
-                const uint32_t k_base = sK + st * C::TILE_BYTES;
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    if (q >= it.nact || !tile_needed(it, q, t)) {
-                        // This query tile does not use the stage: its kv_empty share is free now.
-                        if (leader) ptx::mbar_arrive(&kv_empty[st]);
-                        __syncwarp();
-                        continue;
-                    }
-                    const uint32_t sbuf = qtile[q] % NSB;
-                    // With one S buffer per query tile, the pending P.V (reading P over S) must be
-                    // issued before S is overwritten; with two, S first keeps the tensor core busy.
-                    if (NSB == 1 && pend[q].have) {
-                        ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
-                                         tmem_base, sV, vdesc, idesc_pv, D, leader);
-                        if (!ok) break;
-                    }
-                    if (leader) {
-                        const uint32_t q_base = sQ + (qb * NQ + q) * C::TILE_BYTES;
-#pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t off = (ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
-                                                 (ks % C::KSTEPS_PER_CHUNK) * 32;
-                            ptx::mma_ss(tmem_base + (q * NSB + sbuf) * 128, kdesc | ((q_base + off) >> 4),
-                                        kdesc | ((k_base + off) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
+                bool seen[NQ];
+    #pragma unroll
+                for (int q = 0; q < NQ; ++q) seen[q] = false;
+                for (int t = it.t_begin; t < it.t_end && ok; ++t) {
+                    const uint32_t st = kv_iter % C::NST;
+                    const uint32_t round = kv_iter / C::NST;
+                    // A P.V still pending on this stage (its query tile skipped the tiles since)
+                    // must be issued now: the stage is reloaded only after it.
+    #pragma unroll
+                    for (int q = 0; q < NQ; ++q)
+                        if (ok && pend[q].have && pend[q].st == st) {
+                            ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
+                                             tmem_base, sV, vdesc, idesc_pv, D, leader);
+                            pend[q].have = false;
                         }
-                        ptx::mma_commit(&s_full[q * NSB + sbuf]);
+                    if (!ok) break;
+                    ok = wait_bar_warp(&k_full[st], round & 1, abort_flag, p.err);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const TileRef tr = tile_of<MODE>(p, it, t);
+                    const uint32_t idesc_qk = ptx::idesc_bf16_f32(kBlockM, tr.nk16, false);
+                    const uint32_t k_base = sK + st * C::TILE_BYTES;
+    #pragma unroll
+                    for (int q = 0; q < NQ; ++q) {
+                        if (q >= it.nact || !tile_needed(it, q, t)) {
+                            // This query tile does not use the stage: its kv_empty share is free now.
+                            if (leader) ptx::mbar_arrive(&kv_empty[st]);
+                            __syncwarp();
+                            continue;
+                        }
+                        const uint32_t sbuf = qtile[q] % NSB;
+                        // With one S buffer per query tile, the pending P.V (reading P over S) must be
+                        // issued before S is overwritten; with two, S first keeps the tensor core busy.
+                        if (NSB == 1 && pend[q].have) {
+                            ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
+                                             tmem_base, sV, vdesc, idesc_pv, D, leader);
+                            if (!ok) break;
+                        }
+                        if (leader) {
+                            const uint32_t q_base = sQ + (qb * NQ + q) * C::TILE_BYTES;
+    #pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t off = (ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
+                                                     (ks % C::KSTEPS_PER_CHUNK) * 32;
+                                ptx::mma_ss(tmem_base + (q * NSB + sbuf) * 128, kdesc | ((q_base + off) >> 4),
+                                            kdesc | ((k_base + off) >> 4), idesc_qk, ks > 0 ? 1u : 0u);
+                            }
+                            ptx::mma_commit(&s_full[q * NSB + sbuf]);
+                        }
+                        __syncwarp();
+                        if (NSB == 2 && pend[q].have) {
+                            ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
+                                             tmem_base, sV, vdesc, idesc_pv, D, leader);
+                            if (!ok) break;
+                        }
+                        pend[q].have = true;
+                        pend[q].first = !seen[q];
+                        seen[q] = true;
+                        pend[q].st = st;
+                        pend[q].round = round;
+                        pend[q].qt = qtile[q];
+                        pend[q].qi = qitem[q];
+                        pend[q].nk = tr.nk16;
+                        ++qtile[q];
                     }
-                    __syncwarp();
-                    if (NSB == 2 && pend[q].have) {
-                        ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
-                                         tmem_base, sV, vdesc, idesc_pv, D, leader);
-                        if (!ok) break;
-                    }
-                    pend[q].have = true;
-                    pend[q].first = !seen[q];
-                    seen[q] = true;
-                    pend[q].st = st;
-                    pend[q].round = round;
-                    pend[q].qt = qtile[q];
-                    pend[q].qi = qitem[q];
-                    pend[q].nk = tr.nk16;
-                    ++qtile[q];
+                    ++kv_iter;
                 }
-                ++kv_iter;
+    #pragma unroll
+                for (int q = 0; q < NQ; ++q)
+                    if (q < it.nact) ++qitem[q];
+                // Q of this item is free once every QK^T issued so far has completed.
+                if (leader) ptx::mma_commit(&q_empty[qb]);
+                __syncwarp();
+                ++item_idx;
             }
-#pragma unroll
+    #pragma unroll
             for (int q = 0; q < NQ; ++q)
-                if (q < it.nact) ++qitem[q];
-            // Q of this item is free once every QK^T issued so far has completed.
-            if (leader) ptx::mma_commit(&q_empty[qb]);
-            __syncwarp();
-            ++item_idx;
+                if (ok && pend[q].have)
+                    ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err, tmem_base,
+                                     sV, vdesc, idesc_pv, D, leader);
         }
-#pragma unroll
-        for (int q = 0; q < NQ; ++q)
-            if (ok && pend[q].have)
-                ok = issue_pv<C>(q, pend[q], p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err, tmem_base,
-                                 sV, vdesc, idesc_pv, D, leader);
         // Drain: every MMA issued by this warp completes, and every softmax thread is done with
         // TMEM, before TMEM is released.
         if (leader) ptx::mma_commit(mma_drain);
@@ -964,8 +1079,15 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             Scheduler<MODE> sched(p, rg_pre);
             Item it;
             uint32_t qtile = 0, qitem = 0;
+            uint32_t seq = 0;     // rotating S buffers: S numbers issued so far (both query tiles)
+            uint32_t s_par = 0;   // rotating S buffers: bit b = parity of this tile's next S in buffer b
             while (sched.next(it)) {
-                if (q >= it.nact) continue;  // no valid row in this query tile: nothing to do
+                if (q >= it.nact) {
+                    // No valid row in this query tile: nothing to do but count the other's S.
+                    if (C::ROT)
+                        for (int t = it.t_begin; t < it.t_end; ++t) seq += tile_needed(it, 0, t) ? 1u : 0u;
+                    continue;
+                }
                 // Per-row key intervals [lo, hi) for source 0 and source 1 (empty for padded rows).
                 int lo0, hi0, lo1, hi1;
                 bool row_valid;
@@ -998,12 +1120,22 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                 }
                 float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of this row
                 const uint32_t ob = qitem % NOB;
-                const uint32_t o_tmem = tmem_base + lane_off + 256 + (ob * NQ + q) * D;
+                const uint32_t o_tmem = tmem_base + lane_off + C::O_COL + (ob * NQ + q) * D;
                 bool first = true;
                 for (int t = it.t_begin; t < it.t_end; ++t) {
+                    uint32_t my_seq = 0;
+                    if (C::ROT) {
+                        // the MMA warp numbers the S of a key tile query tile 0 first
+                        const bool n0 = tile_needed(it, 0, t);
+                        const bool n1 = it.nact > 1 && tile_needed(it, 1, t);
+                        my_seq = seq + ((q == 1 && n0) ? 1u : 0u);
+                        seq += (n0 ? 1u : 0u) + (n1 ? 1u : 0u);
+                    }
                     if (!tile_needed(it, q, t)) continue;
-                    const uint32_t sbuf = qtile % NSB;
-                    wait_bar_warp(&s_full[q * NSB + sbuf], (qtile / NSB) & 1, abort_flag, p.err);
+                    const uint32_t sbuf = C::ROT ? my_seq % 3 : q * NSB + qtile % NSB;
+                    const uint32_t sph = C::ROT ? (s_par >> sbuf) & 1u : (qtile / NSB) & 1;
+                    if (C::ROT) s_par ^= 1u << sbuf;
+                    wait_bar_warp(&s_full[C::ROT ? q * 3 + sbuf : sbuf], sph, abort_flag, p.err);
                     ptx::tc_fence_after();
                     const TileRef tr = tile_of<MODE>(p, it, t);
                     const int k0 = tr.kt * kBlockN;
@@ -1012,7 +1144,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     const int cmin = lo - k0;
                     const int cmax = min(hi - k0, tr.nk16);
                     const int nchunks = (tr.nk16 + 31) / 32;
-                    const uint32_t s_tmem = tmem_base + lane_off + (q * NSB + sbuf) * 128;
+                    const uint32_t s_tmem = tmem_base + lane_off + sbuf * 128;
                     // live: some row of the warp has an allowed key in the 32-column chunk.
                     uint32_t live = 0;
 #pragma unroll
@@ -1021,15 +1153,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         if (__any_sync(0xffffffffu, mine)) live |= 1u << a;
                     }
                     float s[128];
-                    const uint32_t whole = load_s_row(s_tmem, live, cmin, cmax, s);
-                    float cmx[4];
-#pragma unroll
-                    for (int a = 0; a < 4; ++a) {
-                        cmx[a] = -INFINITY;
-#pragma unroll
-                        for (int c = 0; c < 32; c += 2) cmx[a] = ptx::fmax3(cmx[a], s[32 * a + c], s[32 * a + c + 1]);
-                    }
-                    const float mx = ptx::fmax3(cmx[0], cmx[1], fmaxf(cmx[2], cmx[3]));
+                    const float mx = load_s_row(s_tmem, live, cmin, cmax, s);
                     const float m_new = fmaxf(m, mx * sl2);
                     bool rescale = false;
                     float alpha = 1.f;
@@ -1040,7 +1164,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         l *= alpha;
                     }
                     const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                    l += exp_store_row(s_tmem, live, whole, nchunks, s, sl2, neg_m);
+                    l += exp_store_row(s_tmem, live, nchunks, s, sl2, neg_m);
                     if (!first) {
                         // O may only be touched once the previous P.V has landed.
                         wait_bar_warp(&pv_done[q], (qtile - 1) & 1, abort_flag, p.err);
@@ -1067,7 +1191,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     }
                     ptx::tmem_wait_st();
                     ptx::tc_fence_before();
-                    ptx::mbar_arrive(&p_full[q * NSB + sbuf]);
+                    ptx::mbar_arrive(&p_full[sbuf]);
                     ++qtile;
                     first = false;
                 }
