@@ -22,7 +22,7 @@ EXPORTS = ("e2d2_attn_encoder_blockcausal", "e2d2_attn_decoder_train",
            "e2d2_kv_cache_append", "e2d2_status_string", "e2d2_last_device_error", "e2d2_version",
            "e2d2_attn_decoder_sample_noalloc", "e2d2_attn_encoder_block_step",
            "e2d2_attn_train_backward_workspace", "e2d2_attn_encoder_backward",
-           "e2d2_attn_decoder_train_backward", "e2d2_attn_decoder_sample_plan",
+           "e2d2_attn_decoder_train_backward", "e2d2_attn_decoder_sample_plan", "e2d2_attn_train_order",
            "e2d2_attn_decoder_sample_ragged", "e2d2_attn_decoder_sample_ragged_plan",
            "e2d2_debug_set_wait_test", "e2d2_kv_cache_append_ragged")
 
@@ -97,6 +97,9 @@ def load(path: Path | str | None = None):
                                                      Dims, ci, ci, vp, ctypes.c_size_t, st]
     lib.e2d2_attn_decoder_sample_plan.argtypes = [Dims, ci, ci, ci, ctypes.POINTER(SamplePlan)]
     lib.e2d2_attn_decoder_sample_plan.restype = ctypes.c_int
+    pi = ctypes.POINTER(ctypes.c_int)
+    lib.e2d2_attn_train_order.argtypes = [ci, Dims, ci, ci, ci, pi, pi, pi, pi]
+    lib.e2d2_attn_train_order.restype = ctypes.c_int
     lib.e2d2_attn_decoder_sample_ragged.argtypes = [vp, vp, vp, ci, vp, vp, vp, vp, fp, Dims, ci, vp,
                                                     ctypes.c_size_t, st]
     lib.e2d2_attn_decoder_sample_ragged.restype = ctypes.c_int

@@ -214,6 +214,21 @@ def sample_plan(batch, q_heads, kv_heads, head_dim, S, P, num_sms) -> dict:
     return {name: getattr(plan, name) for name, _ in _lib.SamplePlan._fields_}
 
 
+def train_order(decoder: bool, batch, q_heads, kv_heads, head_dim, L, S, num_sms) -> dict:
+    """Work order of a train call on a GPU with num_sms SMs (no GPU needed): the CTA of each work
+    item (pairs of 128-row query tiles), the grid, and whether the balanced order is used."""
+    lib = _lib.load()
+    items, grid, bal = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    st = lib.e2d2_attn_train_order(int(bool(decoder)), _dims(batch, q_heads, kv_heads, head_dim, None), L, S,
+                                   num_sms, None, ctypes.byref(items), ctypes.byref(grid), ctypes.byref(bal))
+    _lib.check(st, "e2d2_attn_train_order")
+    cta = (ctypes.c_int * items.value)()
+    st = lib.e2d2_attn_train_order(int(bool(decoder)), _dims(batch, q_heads, kv_heads, head_dim, None), L, S,
+                                   num_sms, cta, None, None, None)
+    _lib.check(st, "e2d2_attn_train_order")
+    return {"items": items.value, "grid": grid.value, "balanced": bool(bal.value), "cta_of_item": list(cta)}
+
+
 @_device_guard
 def sample_workspace(q_blk: torch.Tensor, k_cache: torch.Tensor) -> torch.Tensor:
     """A zero-filled workspace for decoder_sample with these shapes."""

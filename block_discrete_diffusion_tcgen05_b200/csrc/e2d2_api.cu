@@ -8,7 +8,11 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <queue>
+#include <utility>
+#include <vector>
 
 #include "attn_bwd_sm100.cuh"
 #include "e2d2_attn.h"
@@ -116,7 +120,8 @@ bool map_2d(CUtensorMap* m, const void* base, int D, long long rows, int box_row
 }
 
 template <int D, int MODE>
-e2d2_status launch_fmha(const FmhaParams& prm, int grid, cudaStream_t st) {
+e2d2_status launch_fmha(const FmhaParams& prm, int grid, cudaStream_t st,
+                        const typename OrderOf<MODE>::type& ord = typename OrderOf<MODE>::type{}) {
     using SM = Smem<D, MODE>;
     static_assert(SM::ALLOC <= 232448, "shared memory budget");
     auto kern = fmha_sm100_kernel<D, MODE>;
@@ -130,7 +135,7 @@ e2d2_status launch_fmha(const FmhaParams& prm, int grid, cudaStream_t st) {
             return E2D2_ERR_CUDA;
         configured_dev = dev;
     }
-    kern<<<grid, kThreads, smem, st>>>(prm);
+    kern<<<grid, kThreads, smem, st>>>(prm, ord);
     return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
 }
 
@@ -153,13 +158,102 @@ e2d2_status launch_keyrow(const FmhaParams& prm, int grid, cudaStream_t st) {
 }
 
 template <int MODE>
-e2d2_status dispatch_fmha(int D, const FmhaParams& prm, int grid, cudaStream_t st) {
+e2d2_status dispatch_fmha(int D, const FmhaParams& prm, int grid, cudaStream_t st,
+                          const typename OrderOf<MODE>::type& ord = typename OrderOf<MODE>::type{}) {
     switch (D) {
-        case 32: return launch_fmha<32, MODE>(prm, grid, st);
-        case 64: return launch_fmha<64, MODE>(prm, grid, st);
-        case 128: return launch_fmha<128, MODE>(prm, grid, st);
+        case 32: return launch_fmha<32, MODE>(prm, grid, st, ord);
+        case 64: return launch_fmha<64, MODE>(prm, grid, st, ord);
+        case 128: return launch_fmha<128, MODE>(prm, grid, st, ord);
         default: return E2D2_ERR_UNSUPPORTED;
     }
+}
+
+// Work of train item k in tile steps: the key tiles of its stream (as the kernel's scheduler
+// derives them), plus one for the epilogue and the next item's start.
+int train_item_cost(int mode, int B, int Hq, int L, int S, int num_qtiles, int k) {
+    const int BH = B * Hq;
+    const int qp = num_qtiles - 1 - k / BH;
+    const int r0 = qp * 2 * kBlockM;
+    const int nact = (r0 + kBlockM < L) ? 2 : 1;
+    int a1 = 1 << 30, e1 = 0, n0 = 0;
+    for (int q = 0; q < nact; ++q) {
+        const int rq = r0 + q * kBlockM;
+        const int rl = (L < rq + kBlockM ? L : rq + kBlockM) - 1;
+        const int blk_end = (rl / S + 1) * S < L ? (rl / S + 1) * S : L;
+        int qa1, qe1, qn0;
+        if (mode == kEncoder) {
+            qa1 = 0;
+            qe1 = 0;
+            qn0 = (blk_end + kBlockN - 1) / kBlockN;
+        } else {
+            qa1 = ((rq / S) * S) / kBlockN;
+            qe1 = (blk_end + kBlockN - 1) / kBlockN;
+            qn0 = ((rl / S) * S + kBlockN - 1) / kBlockN;
+        }
+        if (qe1 > qa1) {
+            a1 = a1 < qa1 ? a1 : qa1;
+            e1 = e1 > qe1 ? e1 : qe1;
+        }
+        n0 = n0 > qn0 ? n0 : qn0;
+    }
+    if (e1 == 0) a1 = 0;
+    return (e1 - a1) + n0 + 1;
+}
+
+// Longest processing time first: items by decreasing cost (ties by index), each to the CTA with
+// the least work so far (ties by CTA index).  Fills `ord` (enabled = 0 if it does not fit).
+// Cached per shape: the table is a pure function of it.
+void train_item_order(int mode, int B, int Hq, int L, int S, int num_qtiles, int num_items, int grid, ItemOrder* ord) {
+    ord->enabled = 0;
+    if (num_items > kOrderMaxItems || grid > kOrderMaxCtas || grid <= 0) return;
+    struct Key {
+        int mode, B, Hq, L, S, grid;
+        bool operator==(const Key& o) const {
+            return mode == o.mode && B == o.B && Hq == o.Hq && L == o.L && S == o.S && grid == o.grid;
+        }
+    };
+    struct Entry {
+        Key key;
+        ItemOrder ord;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;  // a few shapes; oldest dropped first
+    const Key key{mode, B, Hq, L, S, grid};
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const Entry& e : cache)
+            if (e.key == key) {
+                *ord = e.ord;
+                return;
+            }
+    }
+    std::vector<int> cost(num_items), idx(num_items);
+    for (int k = 0; k < num_items; ++k) {
+        cost[k] = train_item_cost(mode, B, Hq, L, S, num_qtiles, k);
+        idx[k] = k;
+    }
+    std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+    using Load = std::pair<long long, int>;  // (work so far, CTA)
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int c = 0; c < grid; ++c) heap.push({0, c});
+    std::vector<std::vector<int>> per(grid);
+    for (int k : idx) {
+        Load t = heap.top();
+        heap.pop();
+        per[t.second].push_back(k);
+        t.first += cost[k];
+        heap.push(t);
+    }
+    int pos = 0;
+    for (int c = 0; c < grid; ++c) {
+        ord->first[c] = static_cast<uint16_t>(pos);
+        for (int k : per[c]) ord->item[pos++] = static_cast<uint16_t>(k);
+    }
+    ord->first[grid] = static_cast<uint16_t>(pos);
+    ord->enabled = 1;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() >= 8) cache.erase(cache.begin());
+    cache.push_back({key, *ord});
 }
 
 constexpr long long kMaxI32 = 0x7fffffffLL;
@@ -210,8 +304,10 @@ e2d2_status train_common(int mode, const void* q, const void* k0, const void* v0
     prm.num_qtiles = (L + 2 * kBlockM - 1) / (2 * kBlockM);  // work items take pairs of query tiles
     prm.num_items = static_cast<int>(BHq * prm.num_qtiles);
     const int grid = prm.num_items < di->sms ? prm.num_items : di->sms;
-    return mode == kEncoder ? dispatch_fmha<kEncoder>(D, prm, grid, st)
-                            : dispatch_fmha<kDecoderTrain>(D, prm, grid, st);
+    ItemOrder ord;
+    train_item_order(mode, dm.batch, dm.q_heads, L, S, prm.num_qtiles, prm.num_items, grid, &ord);
+    return mode == kEncoder ? dispatch_fmha<kEncoder>(D, prm, grid, st, ord)
+                            : dispatch_fmha<kDecoderTrain>(D, prm, grid, st, ord);
 }
 
 // Backward of the train calls: two launches of attn_bwd_sm100_kernel on the stream, rows-Q
@@ -647,6 +743,33 @@ e2d2_status e2d2_attn_decoder_sample_plan(e2d2_dims dims, int S, int P, int num_
     plan->split_ctas = pl.split_ctas;
     plan->whole_units = pl.whole_units;
     plan->grid = static_cast<int>(pl.grid);
+    return E2D2_OK;
+}
+
+e2d2_status e2d2_attn_train_order(int decoder, e2d2_dims dims, int L, int S, int num_sms, int* cta_of_item,
+                                  int* items_out, int* grid_out, int* balanced_out) {
+    e2d2_status s = check_dims(dims);
+    if (s != E2D2_OK) return s;
+    if (L <= 0 || S <= 0 || num_sms <= 0) return E2D2_ERR_INVALID_ARG;
+    s = check_train_shape(dims, L, S);
+    if (s != E2D2_OK) return s;
+    const int mode = decoder ? kDecoderTrain : kEncoder;
+    const int num_qtiles = (L + 2 * kBlockM - 1) / (2 * kBlockM);
+    const long long items = static_cast<long long>(dims.batch) * dims.q_heads * num_qtiles;
+    const int grid = static_cast<int>(items < num_sms ? items : num_sms);
+    ItemOrder ord;
+    train_item_order(mode, dims.batch, dims.q_heads, L, S, num_qtiles, static_cast<int>(items), grid, &ord);
+    if (cta_of_item) {
+        if (ord.enabled) {
+            for (int c = 0; c < grid; ++c)
+                for (int j = ord.first[c]; j < ord.first[c + 1]; ++j) cta_of_item[ord.item[j]] = c;
+        } else {
+            for (long long k = 0; k < items; ++k) cta_of_item[k] = static_cast<int>(k % grid);
+        }
+    }
+    if (items_out) *items_out = static_cast<int>(items);
+    if (grid_out) *grid_out = grid;
+    if (balanced_out) *balanced_out = ord.enabled;
     return E2D2_OK;
 }
 

@@ -125,6 +125,29 @@ struct alignas(64) FmhaParams {
 constexpr int kRaggedMaxBatch = 256;  // entries of a ragged sampling call (one per thread of the prefix scan)
 constexpr int kMinRaggedTiles = 6;    // tiles per CTA the ragged split aims for
 
+// Train calls: an explicit order of the work items, computed on the host (longest processing
+// time first: each item, longest first, goes to the CTA with the least work so far).  CTA c takes
+// items item[first[c]] .. item[first[c + 1] - 1] in that order.  Without it (enabled = 0: more
+// items or CTAs than the table holds) CTA c takes items c, c + grid, c + 2 grid, ...
+constexpr int kOrderMaxCtas = 160;
+constexpr int kOrderMaxItems = 1152;
+struct ItemOrder {
+    int enabled;
+    uint16_t first[kOrderMaxCtas + 1];
+    uint16_t item[kOrderMaxItems];
+};
+struct NoOrder {
+    int enabled;
+};
+template <int MODE>
+struct OrderOf {
+    using type = ItemOrder;
+};
+template <>
+struct OrderOf<kDecoderSample> {
+    using type = NoOrder;
+};
+
 __host__ __device__ __forceinline__ int ragged_clamp(int P, int capacity) {
     return P < 0 ? 0 : (P > capacity ? capacity : P);
 }
@@ -299,10 +322,18 @@ struct Scheduler {
     long long pos, end;  // sample: tile range of this CTA
     long long total;     // sample: tiles of the split stream
     int sgrid;           // sample: CTAs the split stream is cut over
-    int k;               // train: next item index
+    int k;               // train: next item index (or next position in the item order)
+    int k_end;           // train, item order: end of this CTA's positions
+    const ItemOrder* ord;
 
-    __device__ Scheduler(const FmhaParams& prm, const int* pre = nullptr) : p(prm), rg_pre(pre) {
+    __device__ Scheduler(const FmhaParams& prm, const int* pre = nullptr, const ItemOrder* order = nullptr)
+        : p(prm), rg_pre(pre), ord(order) {
         k = blockIdx.x;
+        k_end = 0;
+        if (MODE != kDecoderSample && ord != nullptr && ord->enabled) {
+            k = ord->first[blockIdx.x];
+            k_end = ord->first[blockIdx.x + 1];
+        }
         if (MODE == kDecoderSample) {
             const int c = static_cast<int>(blockIdx.x);
             if (p.P_dev != nullptr) {
@@ -394,11 +425,18 @@ struct Scheduler {
             if (pos < end) pos = seg_end;
             return true;
         } else {
-            if (k >= p.num_items) return false;
+            int kk;
+            if (ord != nullptr && ord->enabled) {
+                if (k >= k_end) return false;
+                kk = ord->item[k++];
+            } else {
+                if (k >= p.num_items) return false;
+                kk = k;
+                k += gridDim.x;
+            }
             const int BH = p.batch * p.q_heads;
-            const int qp = p.num_qtiles - 1 - k / BH;  // pairs of query tiles, longest rows first
-            const int bh = k % BH;
-            k += gridDim.x;
+            const int qp = p.num_qtiles - 1 - kk / BH;  // pairs of query tiles, longest rows first
+            const int bh = kk % BH;
             const int b = bh / p.q_heads, h = bh % p.q_heads;
             const int L = p.L, S = p.S;
             it.q_z = bh;
@@ -673,8 +711,18 @@ __device__ __forceinline__ float exp_store_row(uint32_t s_tmem, uint32_t live, i
     return t.x + t.y;
 }
 
+template <int MODE>
+__device__ __forceinline__ const ItemOrder* order_ptr(const ItemOrder& o) {
+    return &o;
+}
+template <int MODE>
+__device__ __forceinline__ const ItemOrder* order_ptr(const NoOrder&) {
+    return nullptr;
+}
+
 template <int D, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_constant__ FmhaParams p) {
+__global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_constant__ FmhaParams p,
+                                                                  const __grid_constant__ typename OrderOf<MODE>::type ord) {
     using C = Cfg<D, MODE>;
     using SM = Smem<D, MODE>;
     constexpr int NQ = C::NQ, NSB = C::NSB, NOB = C::NOB;
@@ -763,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         }
         __syncwarp();
         test_producer_delay();
-        Scheduler<MODE> sched(p, rg_pre);
+        Scheduler<MODE> sched(p, rg_pre, order_ptr<MODE>(ord));
         Item it;
         uint32_t kv_iter = 0, item_idx = 0;
         bool ok = true;
@@ -844,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         // The whole warp walks the schedule, so descriptors and TMEM addresses are warp-uniform;
         // one elected lane issues tcgen05.mma / tcgen05.commit.
         const bool leader = ptx::elect_one();
-        Scheduler<MODE> sched(p, rg_pre);
+        Scheduler<MODE> sched(p, rg_pre, order_ptr<MODE>(ord));
         Item it;
         uint32_t kv_iter = 0, item_idx = 0;
         uint32_t qtile[NQ], qitem[NQ];
@@ -1057,7 +1105,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         ptx::setmaxnreg_dec<kRegsControl>();
         // Warps 2-3: the cache write of an encoder block step (sampling calls only), else idle.
         if (MODE == kDecoderSample && p.app_dst_k != nullptr) {
-            Scheduler<MODE> sched(p, rg_pre);
+            Scheduler<MODE> sched(p, rg_pre, order_ptr<MODE>(ord));
             Item it;
             while (sched.next(it))
                 if (it.t_begin == 0 && it.q_row0 == 0) append_block_rows(p, D, it.kv_z, threadIdx.x - 64, 64);
@@ -1076,7 +1124,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         const uint32_t wg_bar = 1 + q;               // named barrier of this warpgroup
         const float sl2 = p.scale_log2;
         if (q < NQ) {
-            Scheduler<MODE> sched(p, rg_pre);
+            Scheduler<MODE> sched(p, rg_pre, order_ptr<MODE>(ord));
             Item it;
             uint32_t qtile = 0, qitem = 0;
             uint32_t seq = 0;     // rotating S buffers: S numbers issued so far (both query tiles)

@@ -194,6 +194,23 @@ E2D2_API e2d2_status e2d2_attn_decoder_sample_plan(e2d2_dims dims, int S, int P,
                                                    e2d2_sample_plan* plan);
 
 /*
+ * Work order of a train call (host only, no GPU needed): which CTA takes each work item of
+ * e2d2_attn_encoder_blockcausal (decoder = 0) or e2d2_attn_decoder_train (decoder = 1) on a
+ * device with num_sms SMs.  A work item is a pair of 128-row query tiles of one (batch, head):
+ * item k covers rows 256 * (n_pairs - 1 - k / (batch * q_heads)) .. of head k mod (batch * q_heads),
+ * n_pairs = ceil(L / 256), so items = batch * q_heads * n_pairs.  The call's grid is
+ * min(items, num_sms).  Items are placed longest processing time first: by decreasing key-tile
+ * count (plus one for the epilogue), each on the CTA with the least work so far; with more than
+ * 1152 items or 160 CTAs the order is round robin instead (item k on CTA k mod grid).
+ *   cta_of_item: host array of `items` ints, written with the CTA of each item (may be NULL);
+ *   *items_out, *grid_out: written when non-NULL; *balanced_out: 1 if the balanced order is used.
+ * The CTA runs its items in the order listed.  Returns E2D2_ERR_INVALID_ARG for bad dims, L <= 0,
+ * S <= 0 or num_sms <= 0.
+ */
+E2D2_API e2d2_status e2d2_attn_train_order(int decoder, e2d2_dims dims, int L, int S, int num_sms, int* cta_of_item,
+                                           int* items_out, int* grid_out, int* balanced_out);
+
+/*
  * Sampling step that allocates nothing: same arguments and result as e2d2_attn_decoder_sample
  * minus the workspace.  The paper has no counterpart; this exists for callers that cannot
  * allocate device memory (an engine that gives all of HBM to its own pool and no allocator to
