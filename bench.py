@@ -58,6 +58,8 @@ KERNEL_SOURCES = {
     "decoder_train": ("fmha_sm100.cuh", "ptx_sm100.cuh"),
     "decoder_sample": ("fmha_keyrow_sm100.cuh", "fmha_sm100.cuh", "ptx_sm100.cuh"),
     "kv_append": ("kv_append.cuh",),
+    "encoder_backward": ("attn_bwd_sm100.cuh", "ptx_sm100.cuh"),
+    "decoder_backward": ("attn_bwd_sm100.cuh", "ptx_sm100.cuh"),
 }
 
 
@@ -68,6 +70,15 @@ def kernel_source_hash(kernel: str) -> str:
     for name in KERNEL_SOURCES[kernel]:
         h.update((ROOT / "block_discrete_diffusion_tcgen05_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()[:16]
+
+
+def bwd_bytes(shape, decoder: bool) -> int:
+    """Algorithmic HBM bytes of one backward call of a train pass."""
+    n_q = shape.batch * shape.q_heads * shape.L * shape.head_dim * 2
+    n_kv = shape.batch * shape.kv_heads * shape.L * shape.head_dim * 2
+    sets = 2 if decoder else 1
+    lse = shape.batch * shape.q_heads * shape.L * 4
+    return 3 * n_q + 2 * sets * n_kv + lse + n_q + 2 * sets * n_kv
 
 
 def traffic_for(kernel: str):
@@ -268,7 +279,11 @@ def run_workload_set(torch, attn, workloads, dev, peaks):
         "frac_tensor": 2 * fl_b / ((enc_ms + dec_ms) * 1e-3) / 1e12 / tc,
         # the two launches issue eight products of 2 d FLOPs per pair (S and dP twice, p K and u K,
         # p^T dO and ds^T Q) against the five of the definition
-        "issued_mma_flops_per_useful": 8 / 5}
+        "issued_mma_flops_per_useful": 8 / 5,
+        # DRAM bytes of one call (both launches) from the committed ncu capture, and the
+        # algorithmic bytes: q, o, dout, every K/V set read, lse; dq and every dK/dV set written
+        "traffic": {"encoder": traffic_for("encoder_backward"), "decoder": traffic_for("decoder_backward")},
+        "algorithmic_bytes": {"encoder": bwd_bytes(tr, decoder=False), "decoder": bwd_bytes(tr, decoder=True)}}
     # ---- one BD3LM layer against one E2D2 encoder / decoder layer (same shapes, same kernels):
     # BD3LM's 2L-token attention = a decoder-train call on the noised rows + an encoder call on the
     # clean rows; the FLOPs table puts it at twice an E2D2 layer.  L2 flushed before every call.
