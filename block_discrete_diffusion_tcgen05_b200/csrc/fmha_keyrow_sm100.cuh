@@ -463,28 +463,30 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                         wait_bar_warp(&pv_done[sb ^ 1], ((tc - 1) >> 1) & 1, abort_flag, p.err);
                         ptx::tc_fence_after();
                     }
+                    // Every column in one branch-free block (per-column branches made each column
+                    // a dependent chain of its own): the new max where the vote moved it, the factor
+                    // 2^(m_old - m_new) (0 for a column's first keys, 1 where nothing moved).
+                    float fac[NH];
 #pragma unroll
-                    for (int c0 = 0; c0 < NH; c0 += 8) {
-                        if (((E >> c0) & 0xffu) == 0) continue;
-                        uint32_t o[8];
-                        if (rescale_o) {
+                    for (int j = 0; j < NH; ++j) {
+                        const float tm = fmaxf(fmaxf(cm[j], cm[NH + j]), fmaxf(cm[2 * NH + j], cm[3 * NH + j]));
+                        const float mn = ((E >> j) & 1u) ? tm : m_run[j];
+                        fac[j] = ptx::ex2(mn == m_run[j] ? 0.f : m_run[j] - mn);
+                        m_run[j] = mn;
+                        l_part[j] *= fac[j];
+                    }
+                    if (rescale_o) {
+#pragma unroll
+                        for (int c0 = 0; c0 < NH; c0 += 8) {
+                            if (((E >> c0) & 0xffu) == 0) continue;
+                            uint32_t o[8];
                             ptx::tmem_ld8(o_tmem + c0, o);
                             ptx::tmem_wait_ld();
                             ptx::reg_fence<8>(o);
-                        }
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int j = c0 + i;
-                            float a = 1.f;
-                            if ((E >> j) & 1u) {
-                                const float tm = fmaxf(fmaxf(cm[j], cm[NH + j]), fmaxf(cm[2 * NH + j], cm[3 * NH + j]));
-                                a = ptx::ex2(m_run[j] - tm);  // 0 for the first tile (m_run = -inf)
-                                m_run[j] = tm;
-                                l_part[j] *= a;
-                            }
-                            if (rescale_o) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+                            for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fac[c0 + i]);
+                            ptx::tmem_st8(o_tmem + c0, o);
                         }
-                        if (rescale_o) ptx::tmem_st8(o_tmem + c0, o);
                     }
                     if (rescale_o) ptx::tmem_wait_st();
                 }
@@ -492,8 +494,11 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 uint32_t pk[NH / 2];
 #pragma unroll
                 for (int j = 0; j < NH; j += 2) {
-                    const float e0 = (colbase + j < rows) ? ptx::ex2(x[j] - m_run[j]) : 0.f;
-                    const float e1 = (colbase + j + 1 < rows) ? ptx::ex2(x[j + 1] - m_run[j + 1]) : 0.f;
+                    // computed unconditionally, then selected (no per-column branch); a padded
+                    // column (x = m = -inf) gives NaN here and 0 after the select
+                    float e0 = ptx::ex2(x[j] - m_run[j]), e1 = ptx::ex2(x[j + 1] - m_run[j + 1]);
+                    e0 = (colbase + j < rows) ? e0 : 0.f;
+                    e1 = (colbase + j + 1 < rows) ? e1 : 0.f;
                     l_part[j] += e0;
                     l_part[j + 1] += e1;
                     pk[j / 2] = ptx::pack_bf16x2(e0, e1);
