@@ -65,9 +65,15 @@ struct KrCfg {
     static constexpr int KV_CHUNK = kBlockN * 128;                // K/V: one 64-column chunk of 128 keys
     static constexpr int KV_BYTES = 2 * KV_CHUNK;
     static constexpr int P_BYTES = kBlockN * PRB;
-    // Ring stages (shared memory: 2 Q + 2 P^T + NK K + NV V tiles + 16 KB staging within 227 KB)
+    // Ring stages (shared memory: QB Q + 2 P^T + NK K + NV V tiles + the epilogue staging within
+    // 227 KB).  A V stage is held from its load until the P.V of its tile has run (after the
+    // softmax), so the V ring bounds how far the loads run ahead: three stages.  At N = 64 that
+    // takes Q single-buffered (the next unit's Q is loaded once the last S^T of the current one
+    // has read it) and an 8 KB staging buffer.
     static constexpr int NK = 2;
-    static constexpr int NV = (N == 64) ? 2 : 3;
+    static constexpr int NV = 3;
+    static constexpr int QB = (N == 64) ? 1 : 2;
+    static constexpr int STG_BYTES = (N == 64) ? 8192 : 16384;
     // TMEM: S^T buffers at columns 0 and N, O^T buffers at 2N and 3N.
     static constexpr uint32_t TMEM_COLS = (4 * N <= 64) ? 64u : ((4 * N <= 128) ? 128u : 256u);
 };
@@ -75,12 +81,12 @@ struct KrCfg {
 template <int N>
 struct KrSmem {
     using C = KrCfg<N>;
-    static constexpr int OFF_Q = 0;                               // [2][2 chunks][N][128 B]
-    static constexpr int OFF_P = OFF_Q + 2 * C::Q_BYTES;          // [2][128 keys][PRB]
+    static constexpr int OFF_Q = 0;                               // [QB][2 chunks][N][128 B]
+    static constexpr int OFF_P = OFF_Q + C::QB * C::Q_BYTES;      // [2][128 keys][PRB]
     static constexpr int OFF_K = OFF_P + 2 * C::P_BYTES;          // [NK][2 chunks][128][128 B]
     static constexpr int OFF_V = OFF_K + C::NK * C::KV_BYTES;     // [NV][2 chunks][128][128 B]
-    static constexpr int OFF_STG = OFF_V + C::NV * C::KV_BYTES;   // epilogue staging, 16 KB
-    static constexpr int STG_BYTES = 16384;
+    static constexpr int OFF_STG = OFF_V + C::NV * C::KV_BYTES;   // epilogue staging
+    static constexpr int STG_BYTES = C::STG_BYTES;
     static constexpr int OFF_BAR = OFF_STG + STG_BYTES;
     // q_full[2], q_empty[2], k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2],
     // s_free[2], p_full[2], pv_done[2], o_full[2], o_free[2], l_ready[2], l_free[2], qk_drain,
@@ -254,8 +260,8 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         bool ok = true;
         while (ok && sched.next(it)) {
             if (is_k) {
-                const int qb = item_idx & 1;
-                ok = wait_bar_warp(&q_empty[qb], ((item_idx >> 1) & 1) ^ 1, abort_flag, p.err);
+                const int qb = item_idx % C::QB;
+                ok = wait_bar_warp(&q_empty[qb], ((item_idx / C::QB) & 1) ^ 1, abort_flag, p.err);
                 if (!ok) break;
                 if (leader) {
                     ptx::mbar_arrive_expect_tx(&q_full[qb], C::Q_BYTES);
@@ -290,8 +296,8 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         for (uint32_t i = iter > static_cast<uint32_t>(NS) ? iter - NS : 0u; i < iter; ++i)
             wait_bar_warp(&full[i % NS], (i / NS) & 1u, &no_abort, p.err, true);
         if (is_k)
-            for (uint32_t i = item_idx > 2u ? item_idx - 2u : 0u; i < item_idx; ++i)
-                wait_bar_warp(&q_full[i & 1], (i >> 1) & 1u, &no_abort, p.err, true);
+            for (uint32_t i = item_idx > static_cast<uint32_t>(C::QB) ? item_idx - C::QB : 0u; i < item_idx; ++i)
+                wait_bar_warp(&q_full[i % C::QB], (i / C::QB) & 1u, &no_abort, p.err, true);
     } else if (warp == 1) {
         ptx::setmaxnreg_dec<kKrRegsControl>();
         E2D2_KR_POINTERS
@@ -306,8 +312,8 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         uint32_t kit = 0, item_idx = 0, tc = 0;
         bool ok = true;
         while (ok && sched.next(it)) {
-            const uint32_t qb = item_idx & 1;
-            ok = wait_bar_warp(&q_full[qb], (item_idx >> 1) & 1, abort_flag, p.err);
+            const uint32_t qb = item_idx % C::QB;
+            ok = wait_bar_warp(&q_full[qb], (item_idx / C::QB) & 1, abort_flag, p.err);
             for (int t = it.t_begin; t < it.t_end && ok; ++t) {
                 const uint32_t sb = tc & 1;
                 const uint32_t kst = kit % C::NK;
@@ -463,28 +469,29 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                         wait_bar_warp(&pv_done[sb ^ 1], ((tc - 1) >> 1) & 1, abort_flag, p.err);
                         ptx::tc_fence_after();
                     }
-                    // Every column in one branch-free block (per-column branches made each column
-                    // a dependent chain of its own): the new max where the vote moved it, the factor
-                    // 2^(m_old - m_new) (0 for a column's first keys, 1 where nothing moved).
-                    float fac[NH];
+                    // Eight columns at a time, each group one branch-free block (per-column branches
+                    // made each column a dependent chain of its own): the new max where the vote moved
+                    // it, the factor 2^(m_old - m_new) (0 for a column's first keys, 1 where nothing
+                    // moved), then the group's O^T columns if any of them moved.
 #pragma unroll
-                    for (int j = 0; j < NH; ++j) {
-                        const float tm = fmaxf(fmaxf(cm[j], cm[NH + j]), fmaxf(cm[2 * NH + j], cm[3 * NH + j]));
-                        const float mn = ((E >> j) & 1u) ? tm : m_run[j];
-                        fac[j] = ptx::ex2(mn == m_run[j] ? 0.f : m_run[j] - mn);
-                        m_run[j] = mn;
-                        l_part[j] *= fac[j];
-                    }
-                    if (rescale_o) {
+                    for (int c0 = 0; c0 < NH; c0 += 8) {
+                        float fac[8];
 #pragma unroll
-                        for (int c0 = 0; c0 < NH; c0 += 8) {
-                            if (((E >> c0) & 0xffu) == 0) continue;
+                        for (int i = 0; i < 8; ++i) {
+                            const int j = c0 + i;
+                            const float tm = fmaxf(fmaxf(cm[j], cm[NH + j]), fmaxf(cm[2 * NH + j], cm[3 * NH + j]));
+                            const float mn = ((E >> j) & 1u) ? tm : m_run[j];
+                            fac[i] = ptx::ex2(mn == m_run[j] ? 0.f : m_run[j] - mn);
+                            m_run[j] = mn;
+                            l_part[j] *= fac[i];
+                        }
+                        if (rescale_o && ((E >> c0) & 0xffu) != 0) {
                             uint32_t o[8];
                             ptx::tmem_ld8(o_tmem + c0, o);
                             ptx::tmem_wait_ld();
                             ptx::reg_fence<8>(o);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fac[c0 + i]);
+                            for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fac[i]);
                             ptx::tmem_st8(o_tmem + c0, o);
                         }
                     }
@@ -494,11 +501,8 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 uint32_t pk[NH / 2];
 #pragma unroll
                 for (int j = 0; j < NH; j += 2) {
-                    // computed unconditionally, then selected (no per-column branch); a padded
-                    // column (x = m = -inf) gives NaN here and 0 after the select
-                    float e0 = ptx::ex2(x[j] - m_run[j]), e1 = ptx::ex2(x[j + 1] - m_run[j + 1]);
-                    e0 = (colbase + j < rows) ? e0 : 0.f;
-                    e1 = (colbase + j + 1 < rows) ? e1 : 0.f;
+                    const float e0 = (colbase + j < rows) ? ptx::ex2(x[j] - m_run[j]) : 0.f;
+                    const float e1 = (colbase + j + 1 < rows) ? ptx::ex2(x[j + 1] - m_run[j + 1]) : 0.f;
                     l_part[j] += e0;
                     l_part[j + 1] += e1;
                     pk[j / 2] = ptx::pack_bf16x2(e0, e1);
@@ -610,7 +614,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
             // columns over the 128 threads, branch-free; padding columns are staged but not copied)
             // and write each pass with one bulk copy.
             const int ncols = whole ? rows : cap;
-            const int pass_cols = whole ? 64 : 32;  // 16 KB of bf16 / fp32 rows
+            const int pass_cols = whole ? SM::STG_BYTES / (D * 2) : SM::STG_BYTES / (D * 4);  // one staging buffer
 #pragma unroll 1
             for (int c_lo = 0; c_lo < ncols; c_lo += pass_cols) {
                 const int c_end = min(N, c_lo + pass_cols);
