@@ -123,7 +123,7 @@ struct alignas(64) FmhaParams {
 };
 
 constexpr int kRaggedMaxBatch = 256;  // entries of a ragged sampling call (one per thread of the prefix scan)
-constexpr int kMinRaggedTiles = 6;    // tiles per CTA the ragged split aims for
+constexpr int kMinRaggedTiles = 3;    // tiles per CTA the ragged split aims for
 
 // Train calls: an explicit order of the work items, computed on the host (longest processing
 // time first: each item, longest first, goes to the CTA with the least work so far).  CTA c takes

@@ -273,8 +273,8 @@ E2D2_API e2d2_status e2d2_attn_decoder_sample_ragged(const void* q_blk, const vo
  *   kernel: as in e2d2_sample_plan; units = batch * units_per_entry; total_tiles = the length of
  *   the stream (sum over entries of units_per_entry * (ceil(S/128) + ceil(P/128)), P clamped to
  *   [0, capacity]); grid = CTAs launched = min(num_sms, 256).  The stream is cut over
- *   stream_ctas = min(grid, total_tiles, max(units, total_tiles / 6)) CTAs (at least one per unit,
- *   about six tiles each beyond that, at least one tile each), CTA c < stream_ctas taking stream
+ *   stream_ctas = min(grid, total_tiles, max(units, total_tiles / 3)) CTAs (at least one per unit,
+ *   about three tiles each beyond that, at least one tile each), CTA c < stream_ctas taking stream
  *   tiles [c * total / stream_ctas, (c + 1) * total / stream_ctas); the other CTAs take nothing.
  * Returns E2D2_ERR_INVALID_ARG for NULL pointers, bad dims, S <= 0, capacity < 0 or num_sms <= 0,
  * E2D2_ERR_SHAPE for batch > 256.

@@ -135,8 +135,11 @@ def test_sample_workspace_holds_two_slots_per_cta():
 # entry b's units taking ceil(S/128) + ceil(P[b]/128) tiles each, cut into equal contiguous
 # ranges over all launched CTAs.
 # ---------------------------------------------------------------------------------------------
+RAGGED_MIN_TILES = 3   # tiles per CTA the ragged split aims for (kMinRaggedTiles)
+
+
 def ragged_stream_ctas(T, units, grid):
-    return min(grid, T, max(units, T // 6))
+    return min(grid, T, max(units, T // RAGGED_MIN_TILES))
 
 
 def ragged_walk(P, S, upe, cap, grid):
