@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
+    ptx::griddep_launch_dependents();  // the next kernel may launch; it waits for this one's end
 #define E2D2_BWD_SMEM_POINTERS                                                                       \
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &      \
                                                ~static_cast<uintptr_t>(1023));                       \
@@ -446,6 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             ptx::tmem_alloc(tmem_holder, kTmemCols);
             ptx::tmem_relinquish();
         }
+        ptx::griddep_wait();  // inputs (and the workspace) after the previous kernel has finished
         ptx::tc_fence_before();
         __syncthreads();
         ptx::tc_fence_after();

@@ -119,6 +119,24 @@ bool map_2d(CUtensorMap* m, const void* base, int D, long long rows, int box_row
     return r == CUDA_SUCCESS;
 }
 
+// Every kernel goes out with programmatic stream serialization: it may launch while the previous
+// kernel on the stream is still running (its CTAs do their setup on free SMs) and waits for that
+// kernel's completion (griddepcontrol.wait) before it reads or writes anything the caller owns.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <int D, int MODE>
 e2d2_status launch_fmha(const FmhaParams& prm, int grid, cudaStream_t st,
                         const typename OrderOf<MODE>::type& ord = typename OrderOf<MODE>::type{}) {
@@ -135,8 +153,7 @@ e2d2_status launch_fmha(const FmhaParams& prm, int grid, cudaStream_t st,
             return E2D2_ERR_CUDA;
         configured_dev = dev;
     }
-    kern<<<grid, kThreads, smem, st>>>(prm, ord);
-    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, prm, ord) == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
 }
 
 template <int N>
@@ -153,8 +170,7 @@ e2d2_status launch_keyrow(const FmhaParams& prm, int grid, cudaStream_t st) {
             return E2D2_ERR_CUDA;
         configured_dev = dev;
     }
-    kern<<<grid, kKrThreads, smem, st>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+    return launch_pdl(kern, dim3(grid), dim3(kKrThreads), smem, st, prm) == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
 }
 
 template <int MODE>
@@ -334,8 +350,7 @@ e2d2_status launch_bwd(const BwdTcParams& prm, int grid, cudaStream_t st) {
             return E2D2_ERR_CUDA;
         configured_dev = dev;
     }
-    kern<<<grid, kThreads, smem, st>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, prm) == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
 }
 
 template <int SIDE>
@@ -855,8 +870,9 @@ e2d2_status append_call(void* k_cache, void* v_cache, int capacity, int P, const
     long long blocks = (total + 255) / 256;
     const long long cap_blocks = static_cast<long long>(di->sms) * 8;
     if (blocks > cap_blocks) blocks = cap_blocks;
-    kv_append_kernel<<<dim3(static_cast<unsigned>(blocks), 2), 256, 0, stream>>>(a);
-    return cudaGetLastError() == cudaSuccess ? E2D2_OK : E2D2_ERR_CUDA;
+    return launch_pdl(kv_append_kernel, dim3(static_cast<unsigned>(blocks), 2), dim3(256), 0, stream, a) == cudaSuccess
+               ? E2D2_OK
+               : E2D2_ERR_CUDA;
 }
 }  // namespace
 

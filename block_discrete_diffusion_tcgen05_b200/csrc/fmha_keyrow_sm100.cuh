@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
+    ptx::griddep_launch_dependents();  // the next kernel may launch; it waits for this one's end
 #define E2D2_KR_POINTERS                                                                              \
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &       \
                                                ~static_cast<uintptr_t>(1023));                        \
@@ -224,6 +225,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         ptx::tmem_alloc(tmem_holder, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
+    ptx::griddep_wait();  // inputs are read after the previous kernel on the stream has finished
     if (p.P_dev != nullptr) ragged_prefix(p, rg_pre, rg_pre + kRaggedMaxBatch + 1);
     ptx::tc_fence_before();
     __syncthreads();

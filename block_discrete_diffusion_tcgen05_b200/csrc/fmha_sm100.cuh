@@ -729,6 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
+    ptx::griddep_launch_dependents();  // the next kernel may launch; it waits for this one's end
     // All shared-memory pointers derive from `smem`; the roles recompute them after setmaxnreg
     // so that nothing but smem/tmem_base lives across the register-budget change.
 #define E2D2_SMEM_POINTERS                                                                           \
@@ -781,6 +782,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         ptx::tmem_alloc(tmem_holder, kTmemCols);
         ptx::tmem_relinquish();
     }
+    // Everything above touches only this CTA's resources; inputs are read after the previous
+    // kernel on the stream has finished (programmatic dependent launch).
+    ptx::griddep_wait();
     if (MODE == kDecoderSample && p.P_dev != nullptr) ragged_prefix(p, rg_pre, rg_pre + kRaggedMaxBatch + 1);
     ptx::tc_fence_before();
     __syncthreads();

@@ -7,6 +7,8 @@
 
 #include <cstdint>
 
+#include "ptx_sm100.cuh"
+
 namespace e2d2 {
 
 struct AppendParams {
@@ -20,6 +22,8 @@ struct AppendParams {
 };
 
 __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams a) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();  // the previous kernel may still read the cache or write the new rows
     const int which = blockIdx.y;
     uint4* __restrict__ dst = a.cache[which];
     const uint4* __restrict__ src = a.src[which];
