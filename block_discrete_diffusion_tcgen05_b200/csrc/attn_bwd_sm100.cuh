@@ -117,8 +117,8 @@ struct BwdSmem {
     static constexpr int OFF_BAR = OFF_STG + 2 * C::ROW_TILE;
     // row_full[RBUF], row_empty[RBUF], col_full[NST], col_empty[NST], s_full[NSET], p_full[NSET],
     // set_free[NSET], acc_full[NACC], acc_free[NACC], rowd_full[2], rowd_empty[2], out_full,
-    // out_empty, acc_issued, mma_drain, acc_drain, softmax_done
-    static constexpr int NBAR = 2 * C::RBUF + 2 * C::NST + 3 * C::NSET + 2 * C::NACC + 4 + 3 + 3;
+    // out_empty, acc_issued, mma_drain, acc_drain, softmax_done, usum_ready[2], stg_free
+    static constexpr int NBAR = 2 * C::RBUF + 2 * C::NST + 3 * C::NSET + 2 * C::NACC + 4 + 3 + 3 + 3;
     static constexpr int OFF_MISC = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
@@ -401,12 +401,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
     uint64_t* mma_drain = acc_issued + 1;                                                            \
     uint64_t* acc_drain = mma_drain + 1;                                                             \
     uint64_t* softmax_done = acc_drain + 1;                                                          \
+    uint64_t* usum_ready = softmax_done + 1; /* rows-Q: [2] the early warpgroup's sum of u is in */  \
+    uint64_t* stg_free = usum_ready + 2;     /* rows-Q: the last gradient store has read the stage */\
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);                        \
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::OFF_MISC + 8);             \
     (void)row_full; (void)row_empty; (void)col_full; (void)col_empty; (void)s_full; (void)p_full;    \
     (void)acc_full; (void)acc_free; (void)mma_drain; (void)softmax_done; (void)tmem_holder;          \
     (void)set_free; (void)acc_drain; (void)rowd_full; (void)rowd_empty; (void)out_full;              \
-    (void)out_empty; (void)acc_issued;                                                               \
+    (void)out_empty; (void)acc_issued; (void)usum_ready; (void)stg_free;                             \
     (void)abort_flag;
     uint32_t tmem_base;
     {
@@ -440,6 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             ptx::mbar_init(mma_drain, 1);
             ptx::mbar_init(acc_drain, 1);
             ptx::mbar_init(softmax_done, kSoftmaxThreads);
+            ptx::mbar_init(&usum_ready[0], 128);
+            ptx::mbar_init(&usum_ready[1], 128);
+            ptx::mbar_init(stg_free, 1);
             *abort_flag = 0;
             ptx::fence_mbar_init();
         }
@@ -781,7 +786,61 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             const uint32_t acc = tmem_base + lane_off + ACC0 + ab * 2 * D;
             const int wtid = threadIdx.x - 128 - 128 * w;  // 0..127 within the warpgroup
             constexpr int UNITS_PER_CHUNK = C::RB / 16;
-            if (SIDE == kBwdRowsQ) {
+            if (SIDE == kBwdRowsQ && NACC == 1) {
+                // Only the warpgroup that took the item's last sub-tile runs the epilogue; the other
+                // hands over its sum of u and goes on with the next item (whose first sub-tile is
+                // its own).  One accumulator set: the next item's accumulations wait for acc_free,
+                // so neither warpgroup gets more than one item ahead of the epilogue, and the two
+                // usum_ready slots and the one stage cannot be reused before they are read.
+                const int par = iw & 1;
+                const int w_late = static_cast<int>((n - 1u) & 1u);  // n: one past the item's last sub-tile
+                if (w != w_late) {
+                    xch[(par * 2 + w) * kBwdRows + lrow] = usum;
+                    ptx::mbar_arrive(&usum_ready[par]);
+                } else {
+                    uint8_t* stage = smem + SM::OFF_STG;
+                    wait_bar_warp(&usum_ready[par], (iw >> 1) & 1u, abort_flag, p.err);
+                    // D_i - c_i = the sum of u over both warpgroups' sub-tiles.
+                    const float du = usum + xch[(par * 2 + (1 - w)) * kBwdRows + lrow];
+                    // the previous item's store (by either warpgroup) has finished reading the stage
+                    wait_bar_warp(stg_free, (iw & 1u) ^ 1u, abort_flag, p.err);
+                    wait_bar_warp(&acc_full[ab], (iw / NACC) & 1u, abort_flag, p.err);
+                    ptx::tc_fence_after();
+                    constexpr int CW = D < 32 ? D : 32;
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += CW) {
+                        float y[CW], x[CW];
+                        load_tmem_cols<CW>(acc + c0, y);
+                        load_tmem_cols<CW>(acc + D + c0, x);
+#pragma unroll
+                        for (int c = 0; c < CW; ++c) x[c] = fmaf(-du, y[c], x[c]);
+#pragma unroll
+                        for (int g = 0; g < CW / 8; ++g) {
+                            const int unit = (c0 + 8 * g) / 8;
+                            *reinterpret_cast<uint4*>(stage + (unit / UNITS_PER_CHUNK) * C::ROW_CHUNK +
+                                                      swz_offset<C::RB>(lrow, unit % UNITS_PER_CHUNK)) =
+                                pack8_bf16(&x[8 * g], p.scale);
+                        }
+                    }
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive_cnt(&acc_free[ab], 2);  // both warpgroups' share
+                    {
+                        const size_t r = static_cast<size_t>(it.row_z) * p.Lpad + row;
+                        p.ws_nl2[r] = valid ? nl2_row : -INFINITY;
+                        p.ws_D[r] = valid ? -(c_row + du) : 0.f;
+                    }
+                    ptx::fence_proxy_async_smem();
+                    ptx::named_barrier_sync(2 + w, 128);
+                    if (wtid == 0) {
+                        for (int ch = 0; ch < C::NCH; ++ch)
+                            ptx::tma_store_3d(&p.tm_ga[0], stage + ch * C::ROW_CHUNK, ch * (C::RB / 2), it.row0,
+                                              it.row_z);
+                        ptx::tma_store_commit();
+                        ptx::tma_store_wait_read_all();
+                        ptx::mbar_arrive(stg_free);
+                    }
+                }
+            } else if (SIDE == kBwdRowsQ) {
                 uint8_t* stage = smem + SM::OFF_STG;
                 // the previous item's store has finished reading the stage
                 if (w == 0 && wtid == 0) ptx::tma_store_wait_read_all();
@@ -859,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_sm100_kernel(const __gri
             ++iw;
         }
         // every issued store has completed before the CTA exits
-        if (threadIdx.x == 128 || (SIDE == kBwdRowsKV && threadIdx.x == 256)) ptx::tma_store_wait_all();
+        if (threadIdx.x == 128 || threadIdx.x == 256) ptx::tma_store_wait_all();
         ptx::tc_fence_before();
         ptx::mbar_arrive(softmax_done);
     }
