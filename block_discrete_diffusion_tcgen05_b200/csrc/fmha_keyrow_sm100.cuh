@@ -97,11 +97,20 @@ struct KrSmem {
     static constexpr int OFF_LRED = OFF_CMAX + 2 * 2 * 4 * C::NH * 4;  // float [2 ob][2 wg][4 warps][NH]
     static constexpr int OFF_MROW = OFF_LRED + 2 * 2 * 4 * C::NH * 4;  // float [2 ob][N]
     static constexpr int OFF_MISC = OFF_MROW + 2 * N * 4;
-    // + per-column scale of the epilogue, then the ragged prefix table (+ 8 scan sums)
-    static constexpr int OFF_RG = ((OFF_MISC + 64 + N * 4 + 15) / 16) * 16;
+    // + per-column scale of the epilogue [2][N], then the ragged prefix table (+ 8 scan sums)
+    static constexpr int OFF_RG = ((OFF_MISC + 64 + 2 * N * 4 + 15) / 16) * 16;
     static constexpr int BYTES = OFF_RG + (kRaggedMaxBatch + 1 + 8) * 4;
     static constexpr int ALLOC = ((BYTES + 1023) / 1024) * 1024 + 1024;  // + alignment slack
 };
+
+// Position (in 16-byte chunks) of chunk c of a partial-slot column row of 128 floats: inside each
+// quarter of the row (eight chunks) the chunk index is XORed with the quarter and the column's
+// parity, so the eight threads of a merge quarter-warp (two columns x four quarters) read eight
+// different bank groups.  A warp's publish of 32 consecutive values still covers one 128-byte
+// segment.
+__device__ __forceinline__ int slot_chunk(int c, int col) {
+    return (c & ~7) | ((c & 7) ^ ((c >> 3) & 3) ^ ((col & 1) << 2));
+}
 
 // Reduces v[0..NH) over the 32 lanes of the warp with `op`, halving the columns a lane keeps at
 // each exchange (NH/2 + NH/4 + ... shuffles instead of 5 per column).  Returns the result for
@@ -560,7 +569,6 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         E2D2_KR_POINTERS
         // -------------------------------------------------------------- epilogue warpgroup
         // Thread = head-dim row d = 32*w + lane of O^T (its TMEM lane); all N columns, EG at a time.
-        constexpr int EG = 8;
         const int w = warp & 3;
         const int d = 32 * w + lane;
         const int wtid = threadIdx.x - 384;
@@ -570,7 +578,6 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
         __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
         const float* mrow_all = reinterpret_cast<const float*>(smem + SM::OFF_MROW);
         const float* lred_all = reinterpret_cast<const float*>(smem + SM::OFF_LRED);
-        uint8_t* stg = smem + SM::OFF_STG;
         Scheduler<kDecoderSample> sched(p, rg_pre);
         Item it;
         uint32_t item_idx = 0;
@@ -596,7 +603,9 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
             float* slot = whole ? nullptr : slot_of(blockIdx.x);
             const float* mrow = mrow_all + ob * N;
             // Per column, once: the normaliser (whole unit) and the LSE, or the slot's m and l.
-            float* colscale = reinterpret_cast<float*>(smem + SM::OFF_MISC + 64);
+            // (double-buffered by unit parity: a thread still scaling this unit's columns cannot
+            // meet the next unit's writes, which come after the next unit's barrier)
+            float* colscale = reinterpret_cast<float*>(smem + SM::OFF_MISC + 64) + ob * N;
             if (wtid < N) {
                 const int col = wtid;
                 const float* lr = lred_all + (ob * 2 + col / NH) * 4 * NH + col % NH;
@@ -611,61 +620,42 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                     slot[cap * D + cap + col] = l;
                 }
             }
-            // The unit's rows (whole: bf16 output rows out_row0.., split: the fp32 [col][D] part of
-            // the slot) are contiguous in global memory: stage them in shared memory (a pass of
-            // columns over the 128 threads, branch-free; padding columns are staged but not copied)
-            // and write each pass with one bulk copy.
-            const int ncols = whole ? rows : cap;
-            const int pass_cols = whole ? SM::STG_BYTES / (D * 2) : SM::STG_BYTES / (D * 4);  // one staging buffer
-#pragma unroll 1
-            for (int c_lo = 0; c_lo < ncols; c_lo += pass_cols) {
-                const int c_end = min(N, c_lo + pass_cols);
-                if (wtid == 0) ptx::tma_store_wait_read_all();  // staging buffer free again
-                ptx::named_barrier_sync(3, 128);                // (and colscale written)
-#pragma unroll 1
-                for (int c0 = c_lo; c0 < c_end; c0 += EG) {
-                    uint32_t raw[EG];
-                    ptx::tmem_ld8(tmem_base + lane_off + 2 * N + ob * N + c0, raw);
-                    ptx::tmem_wait_ld();
-                    ptx::reg_fence<EG>(raw);
-                    const float4 s0 = *reinterpret_cast<const float4*>(colscale + c0);
-                    const float4 s1 = *reinterpret_cast<const float4*>(colscale + c0 + 4);
-                    const float sc[EG] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-                    if (whole) {
-                        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(stg) + (c0 - c_lo) * D + d;
+            // O^T of the unit into registers (this thread's head-dim row, every column), then the
+            // buffer is free for the next unit's products.
+            constexpr int LW = N < 32 ? N : 32;  // columns per TMEM load
+            uint32_t raw[N];
 #pragma unroll
-                        for (int j = 0; j < EG; ++j) st[j * D] = __float2bfloat16_rn(__uint_as_float(raw[j]) * sc[j]);
-                    } else {
-                        float* st = reinterpret_cast<float*>(stg) + (c0 - c_lo) * D + d;
-#pragma unroll
-                        for (int j = 0; j < EG; ++j) st[j * D] = __uint_as_float(raw[j]);
-                    }
-                }
-                ptx::fence_proxy_async_smem();
-                ptx::named_barrier_sync(3, 128);
-                if (wtid == 0) {
-                    const int c_hi = min(ncols, c_lo + pass_cols);
-                    if (whole)
-                        ptx::bulk_store_s2g(outp + static_cast<size_t>(it.out_row0 + c_lo) * D, stg,
-                                            static_cast<uint32_t>(c_hi - c_lo) * D * 2);
-                    else
-                        ptx::bulk_store_s2g(slot + static_cast<size_t>(c_lo) * D, stg,
-                                            static_cast<uint32_t>(c_hi - c_lo) * D * 4);
-                    ptx::tma_store_commit();
-                }
+            for (int c0 = 0; c0 < N; c0 += LW) {
+                const uint32_t ta = tmem_base + lane_off + 2 * N + ob * N + c0;
+                if constexpr (LW == 32) ptx::tmem_ld32(ta, raw + c0);
+                else ptx::tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(raw + c0));
             }
-            // O^T and the column statistics of this buffer are consumed.
+            ptx::tmem_wait_ld();
+            ptx::reg_fence<N>(raw);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&o_free[ob]);
+            ptx::named_barrier_sync(3, 128);  // colscale written, column statistics read
             ptx::mbar_arrive(&l_free[ob]);
+            // The unit's rows (whole: bf16 output rows out_row0.., split: the fp32 [col][D] part of
+            // the slot) go straight from registers to global memory: for each column a warp writes
+            // 32 consecutive head-dim values (one 128-byte segment of the slot).
+            if (whole) {
+                __nv_bfloat16* dst = outp + static_cast<size_t>(it.out_row0) * D + d;
+#pragma unroll
+                for (int c = 0; c < N; ++c)
+                    if (c < rows)
+                        dst[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(raw[c]) * colscale[c]);
+            } else {
+                const int off0 = slot_chunk(d >> 2, 0) * 4 + (d & 3), off1 = slot_chunk(d >> 2, 1) * 4 + (d & 3);
+#pragma unroll
+                for (int c = 0; c < N; ++c)
+                    if (c < cap) slot[static_cast<size_t>(c) * D + ((c & 1) ? off1 : off0)] = __uint_as_float(raw[c]);
+            }
             if (!whole) {
-                // Release: the slot's bulk copies have landed (wait_group 0) and are ordered before
-                // generic accesses; the barrier orders the other threads' m/l stores before one
-                // thread's fence and ticket.  The last CTA of the unit gets ticket c_last - c_first.
+                // Release: the barrier orders every thread's slot stores before one thread's fence
+                // and ticket.  The last CTA of the unit gets ticket c_last - c_first.
                 ptx::named_barrier_sync(3, 128);
                 if (wtid == 0) {
-                    ptx::tma_store_wait_all();
-                    ptx::fence_proxy_async_global();
                     __threadfence();
                     const int ticket = atomicAdd(&p.ws_tickets[c_first], 1);
                     const int last = (ticket == c_last - c_first) ? 1 : 0;
@@ -676,9 +666,8 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 const int is_last = *bcast;
                 ptx::named_barrier_sync(3, 128);
                 // In the CTA's last unit every K/V, Q and P^T buffer is free (the producers are done
-                // and every product of the unit has landed), and so is the staging buffer (this
-                // CTA's slot copies completed before the ticket): the partial slots are then copied
-                // in with one bulk copy each, all in flight at once, and merged from shared memory.
+                // and every product of the unit has landed): the partial slots are then copied in
+                // with one bulk copy each, all in flight at once, and merged from shared memory.
                 const int nparts = c_last - c_first + 1;
                 const uint32_t slot_bytes = static_cast<uint32_t>(p.slot_floats) * 4u;
                 Scheduler<kDecoderSample> peek = sched;
@@ -686,96 +675,82 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 const bool in_smem = is_last && !peek.next(next_it) &&
                                      static_cast<uint32_t>(nparts) * slot_bytes <=
                                          static_cast<uint32_t>(SM::OFF_STG + SM::STG_BYTES - SM::OFF_Q);
+                bool go = is_last;
+                const uint8_t* region = smem + SM::OFF_Q;
                 if (in_smem) {
                     __threadfence();
-                    uint8_t* region = smem + SM::OFF_Q;
                     if (wtid == 0) {
                         ptx::fence_proxy_async_global();
                         ptx::mbar_arrive_expect_tx(merge_full, static_cast<uint32_t>(nparts) * slot_bytes);
                         for (int c = c_first; c <= c_last; ++c)
-                            ptx::bulk_load_g2s(region + (c - c_first) * slot_bytes, slot_of(c), slot_bytes, merge_full);
+                            ptx::bulk_load_g2s(smem + SM::OFF_Q + (c - c_first) * slot_bytes, slot_of(c), slot_bytes,
+                                               merge_full);
                     }
                     // If the copies never landed (bounded wait gave up: error word set), the
                     // slots are not merged and out / lse are left untouched.
-                    const bool landed = wait_bar_warp(merge_full, 0, abort_flag, p.err);
-                    const int dq = (wtid & 3) * 32;
-#pragma unroll 1
-                    for (int col = wtid >> 2; landed && col < cap; col += 32) {
-                        float mm = -INFINITY, ll = 0.f, acc[32];
+                    go = wait_bar_warp(merge_full, 0, abort_flag, p.err);
+                } else if (is_last) {
+                    __threadfence();
+                }
+                // Online merge over the partials in CTA order (the result does not depend on which
+                // CTA merges).  Thread = (column, 32 head-dim values): the eight 16-byte loads of one
+                // partial are independent; the slot's chunk swizzle spreads the eight threads of a
+                // quarter-warp over all 32 banks.
+                const int q4 = wtid & 3;
+                // One partial of the merge: m, l and this thread's 32 values of column col.
+                auto merge_one = [&](float& mm, float& ll, float (&acc)[32], float mc, float lc, const float4 (&v)[8]) {
+                    const float mn = fmaxf(mm, mc);
+                    const float wa = (mm == -INFINITY) ? 0.f : ptx::ex2(mm - mn);
+                    const float wb = (mc == -INFINITY) ? 0.f : ptx::ex2(mc - mn);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+                    for (int i = 0; i < 8; ++i) {
+                        acc[4 * i + 0] = acc[4 * i + 0] * wa + v[i].x * wb;
+                        acc[4 * i + 1] = acc[4 * i + 1] * wa + v[i].y * wb;
+                        acc[4 * i + 2] = acc[4 * i + 2] * wa + v[i].z * wb;
+                        acc[4 * i + 3] = acc[4 * i + 3] * wa + v[i].w * wb;
+                    }
+                    ll = ll * wa + lc * wb;
+                    mm = mn;
+                };
+#pragma unroll 1
+                for (int col = wtid >> 2; go && col < cap; col += 32) {
+                    float mm = -INFINITY, ll = 0.f, acc[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+                    const int sw = q4 ^ ((col & 1) << 2);
+                    if (in_smem) {
 #pragma unroll 1
                         for (int c = 0; c < nparts; ++c) {
                             const float* sl = reinterpret_cast<const float*>(region + c * slot_bytes);
-                            const float mc = sl[cap * D + col];
-                            const float lc = sl[cap * D + cap + col];
-                            const float4* so = reinterpret_cast<const float4*>(sl + col * D + dq);
-                            const float mn = fmaxf(mm, mc);
-                            const float wa = (mm == -INFINITY) ? 0.f : ptx::ex2(mm - mn);
-                            const float wb = (mc == -INFINITY) ? 0.f : ptx::ex2(mc - mn);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const float4 v = so[i];
-                                acc[4 * i + 0] = acc[4 * i + 0] * wa + v.x * wb;
-                                acc[4 * i + 1] = acc[4 * i + 1] * wa + v.y * wb;
-                                acc[4 * i + 2] = acc[4 * i + 2] * wa + v.z * wb;
-                                acc[4 * i + 3] = acc[4 * i + 3] * wa + v.w * wb;
-                            }
-                            ll = ll * wa + lc * wb;
-                            mm = mn;
-                        }
-                        const float inv = ll > 0.f ? 1.f / ll : 0.f;
-                        uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + col) * D + dq);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = pack8_bf16(&acc[8 * i], inv);
-                        if (p.lse != nullptr && dq == 0)
-                            p.lse[it.out_row0 + col] = ll > 0.f ? (mm + __log2f(ll)) * 0.69314718055994531f : -INFINITY;
-                    }
-                } else if (is_last) {
-                    __threadfence();
-                    // Online merge over the partials in CTA order (the result does not depend on
-                    // which CTA merges).  Thread = (column, 32 head-dim values): the ten loads of
-                    // one partial are independent, and two partials are in flight at a time.
-                    const int dq = (wtid & 3) * 32;
-#pragma unroll 1
-                    for (int col = wtid >> 2; col < cap; col += 32) {
-                        float mm = -INFINITY, ll = 0.f, acc[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-#pragma unroll 2
-                        for (int c = c_first; c <= c_last; ++c) {
-                            const float* sl = slot_of(c);
-                            const float mc = __ldcg(sl + cap * D + col);
-                            const float lc = __ldcg(sl + cap * D + cap + col);
-                            const float4* so = reinterpret_cast<const float4*>(sl + static_cast<size_t>(col) * D + dq);
+                            const float4* row = reinterpret_cast<const float4*>(sl + col * D) + 8 * q4;
                             float4 v[8];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) v[i] = __ldcg(so + i);
-                            const float mn = fmaxf(mm, mc);
-                            const float wa = (mm == -INFINITY) ? 0.f : ptx::ex2(mm - mn);
-                            const float wb = (mc == -INFINITY) ? 0.f : ptx::ex2(mc - mn);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                acc[4 * i + 0] = acc[4 * i + 0] * wa + v[i].x * wb;
-                                acc[4 * i + 1] = acc[4 * i + 1] * wa + v[i].y * wb;
-                                acc[4 * i + 2] = acc[4 * i + 2] * wa + v[i].z * wb;
-                                acc[4 * i + 3] = acc[4 * i + 3] * wa + v[i].w * wb;
-                            }
-                            ll = ll * wa + lc * wb;
-                            mm = mn;
+                            for (int i = 0; i < 8; ++i) v[i] = row[i ^ sw];
+                            merge_one(mm, ll, acc, sl[cap * D + col], sl[cap * D + cap + col], v);
                         }
-                        const float inv = ll > 0.f ? 1.f / ll : 0.f;
-                        uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + col) * D + dq);
+                    } else {
+                        // two partials in flight
+#pragma unroll 2
+                        for (int c = 0; c < nparts; ++c) {
+                            const float* sl = slot_of(c_first + c);
+                            const float4* row =
+                                reinterpret_cast<const float4*>(sl + static_cast<size_t>(col) * D) + 8 * q4;
+                            float4 v[8];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = pack8_bf16(&acc[8 * i], inv);
-                        if (p.lse != nullptr && dq == 0)
-                            p.lse[it.out_row0 + col] = ll > 0.f ? (mm + __log2f(ll)) * 0.69314718055994531f : -INFINITY;
+                            for (int i = 0; i < 8; ++i) v[i] = __ldcg(row + (i ^ sw));
+                            merge_one(mm, ll, acc, __ldcg(sl + cap * D + col), __ldcg(sl + cap * D + cap + col), v);
+                        }
                     }
+                    const float inv = ll > 0.f ? 1.f / ll : 0.f;
+                    uint4* dst = reinterpret_cast<uint4*>(outp + static_cast<size_t>(it.out_row0 + col) * D + 32 * q4);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) dst[i] = pack8_bf16(&acc[8 * i], inv);
+                    if (p.lse != nullptr && q4 == 0)
+                        p.lse[it.out_row0 + col] = ll > 0.f ? (mm + __log2f(ll)) * 0.69314718055994531f : -INFINITY;
                 }
             }
             ++item_idx;
         }
-        if (wtid == 0) ptx::tma_store_wait_all();  // the staging buffer is read before the CTA exits
         ptx::tc_fence_before();
         ptx::mbar_arrive(tmem_done);
     }
