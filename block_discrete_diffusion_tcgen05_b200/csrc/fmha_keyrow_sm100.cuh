@@ -634,17 +634,36 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
             ptx::reg_fence<N>(raw);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&o_free[ob]);
+            if (wtid == 0) ptx::tma_store_wait_read_all();  // the last unit's output has left the staging buffer
             ptx::named_barrier_sync(3, 128);  // colscale written, column statistics read
             ptx::mbar_arrive(&l_free[ob]);
             // The unit's rows (whole: bf16 output rows out_row0.., split: the fp32 [col][D] part of
             // the slot) go straight from registers to global memory: for each column a warp writes
             // 32 consecutive head-dim values (one 128-byte segment of the slot).
             if (whole) {
-                __nv_bfloat16* dst = outp + static_cast<size_t>(it.out_row0) * D + d;
+                // bf16 rows staged in shared memory (a pass of columns per staging buffer) and
+                // written with one bulk copy per pass
+                constexpr int PASS = SM::STG_BYTES / (D * 2);
+                __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(smem + SM::OFF_STG) + d;
 #pragma unroll
-                for (int c = 0; c < N; ++c)
-                    if (c < rows)
-                        dst[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(raw[c]) * colscale[c]);
+                for (int c_lo = 0; c_lo < N; c_lo += PASS) {
+                    if (c_lo >= rows) break;
+                    if (c_lo > 0) {
+                        if (wtid == 0) ptx::tma_store_wait_read_all();  // the previous pass has been read
+                        ptx::named_barrier_sync(3, 128);
+                    }
+#pragma unroll
+                    for (int c = c_lo; c < c_lo + PASS && c < N; ++c)
+                        st[(c - c_lo) * D] = __float2bfloat16_rn(__uint_as_float(raw[c]) * colscale[c]);
+                    ptx::fence_proxy_async_smem();
+                    ptx::named_barrier_sync(3, 128);
+                    if (wtid == 0) {
+                        const int c_hi = min(rows, c_lo + PASS);
+                        ptx::bulk_store_s2g(outp + static_cast<size_t>(it.out_row0 + c_lo) * D,
+                                            smem + SM::OFF_STG, static_cast<uint32_t>(c_hi - c_lo) * D * 2);
+                        ptx::tma_store_commit();
+                    }
+                }
             } else {
                 const int off0 = slot_chunk(d >> 2, 0) * 4 + (d & 3), off1 = slot_chunk(d >> 2, 1) * 4 + (d & 3);
 #pragma unroll
@@ -751,6 +770,7 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
             }
             ++item_idx;
         }
+        if (wtid == 0) ptx::tma_store_wait_all();  // the staging buffer is read before the CTA exits
         ptx::tc_fence_before();
         ptx::mbar_arrive(tmem_done);
     }
