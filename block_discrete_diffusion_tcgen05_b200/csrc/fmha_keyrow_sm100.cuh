@@ -286,6 +286,10 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
             for (int t = it.t_begin; t < it.t_end; ++t) {
                 const int st = iter % NS;
                 ok = wait_bar_warp(&empty[st], ((iter / NS) & 1) ^ 1, abort_flag, p.err);
+                // The first V loads wait for the first K tile: at launch every CTA asks for its
+                // tiles at once, and Q + K0 (the first product's operands) land sooner without
+                // three V tiles competing for the same DRAM bandwidth.
+                if (ok && !is_k && iter == 0) ok = wait_bar_warp(&k_full[0], 0, abort_flag, p.err);
                 if (!ok) break;
                 const TileRef tr = tile_of<kDecoderSample>(p, it, t);
                 // debug builds: the tile starts inside its source and the kv unit exists
