@@ -124,6 +124,13 @@ struct alignas(64) FmhaParams {
 
 constexpr int kRaggedMaxBatch = 256;  // entries of a ragged sampling call (one per thread of the prefix scan)
 constexpr int kMinRaggedTiles = 3;    // tiles per CTA the ragged split aims for
+// P.V completions of a query tile go round a ring of this many barriers (P.V number j to barrier
+// j % kPvRing).  A softmax warp waits for the previous P.V only when it rescales O; with one
+// barrier, skipped waits could leave it two phases behind and a parity wait would pass early.
+// When the softmax works on tile t, every P.V of that query tile up to t - 3 has completed (the
+// S it reads was issued after them, and the tensor core runs in order) and P.V t + k cannot
+// complete before tile t + k's P exists, so a ring of four keeps each wait unambiguous.
+constexpr int kPvRing = 4;
 
 // Train calls: an explicit order of the work items, computed on the host (longest processing
 // time first: each item, longest first, goes to the CTA with the least work so far).  CTA c takes
@@ -236,8 +243,8 @@ struct Smem {
     static constexpr int O_BYTES = C::STAGE_O ? C::NQ * C::TILE_BYTES : 0;
     static constexpr int OFF_BAR = OFF_O + O_BYTES;
     // barriers: k_full[NST], v_full[NST], kv_empty[NST], q_full[QBUF], q_empty[QBUF],
-    // s_full[NSFULL], p_full[NSBUF], pv_done[NQ], o_free[NOB*NQ], mma_drain, softmax_done
-    static constexpr int NBAR = 3 * C::NST + 2 * C::QBUF + C::NSFULL + C::NSBUF + C::NQ + C::NOB * C::NQ + 2;
+    // s_full[NSFULL], p_full[NSBUF], pv_done[NQ][kPvRing], o_free[NOB*NQ], mma_drain, softmax_done
+    static constexpr int NBAR = 3 * C::NST + 2 * C::QBUF + C::NSFULL + C::NSBUF + C::NQ * kPvRing + C::NOB * C::NQ + 2;
     static constexpr int OFF_MISC = ((OFF_BAR + NBAR * 8 + 15) / 16) * 16;
     // sampling: ragged prefix table pre[kRaggedMaxBatch + 1] and the scan's 8 warp sums
     static constexpr int OFF_RG = OFF_MISC + 64;
@@ -562,6 +569,7 @@ struct PendingPV {
     uint32_t qt;       // S buffer use: per-query-tile tile counter, or (rotating buffers) S number
     uint32_t qi;       // per-query-tile item counter (o_free parity, O buffer)
     uint32_t nk;       // keys in the tile (multiple of 16)
+    uint32_t pvn;      // P.V number of its query tile (pv_done ring slot pvn % kPvRing)
 };
 
 // Issues O[q] (+)= P[q] . V[st] (A = P from TMEM, B = V MN-major in shared memory) once the
@@ -587,7 +595,7 @@ __device__ __forceinline__ bool issue_pv(int q, const PendingPV& pv, uint64_t* p
         for (uint32_t ks = 0; ks < pv.nk / 16; ++ks)
             ptx::mma_ts(d_tmem, a_tmem + p_col(ks), vdesc | ((v_base + ks * 16 * C::RB) >> 4), idesc_pv,
                         (pv.first && ks == 0) ? 0u : 1u);
-        ptx::mma_commit(&pv_done[q]);
+        ptx::mma_commit(&pv_done[q * kPvRing + pv.pvn % kPvRing]);
         ptx::mma_commit(&kv_empty[pv.st]);
     }
     __syncwarp();
@@ -743,8 +751,8 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
     uint64_t* q_empty = q_full + C::QBUF;                                                            \
     uint64_t* s_full = q_empty + C::QBUF;  /* [S buffer] or [q][S buffer] */                         \
     uint64_t* p_full = s_full + C::NSFULL; /* [S buffer] */                                          \
-    uint64_t* pv_done = p_full + C::NSBUF; /* [q] */                                                 \
-    uint64_t* o_free = pv_done + NQ;       /* [ob][q] */                                             \
+    uint64_t* pv_done = p_full + C::NSBUF; /* [q][kPvRing] */                                        \
+    uint64_t* o_free = pv_done + NQ * kPvRing; /* [ob][q] */                                         \
     uint64_t* mma_drain = o_free + NOB * NQ;                                                         \
     uint64_t* softmax_done = mma_drain + 1; /* every softmax thread is finished with TMEM */        \
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM::OFF_MISC);                        \
@@ -771,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
         }
         for (int i = 0; i < C::NSFULL; ++i) ptx::mbar_init(&s_full[i], 1);
         for (int i = 0; i < C::NSBUF; ++i) ptx::mbar_init(&p_full[i], kSoftmaxThreads / 2);
-        for (int i = 0; i < NQ; ++i) ptx::mbar_init(&pv_done[i], 1);
+        for (int i = 0; i < NQ * kPvRing; ++i) ptx::mbar_init(&pv_done[i], 1);
         for (int i = 0; i < NOB * NQ; ++i) ptx::mbar_init(&o_free[i], kSoftmaxThreads / 2);
         ptx::mbar_init(mma_drain, 1);
         ptx::mbar_init(softmax_done, kSoftmaxThreads);
@@ -920,9 +928,9 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
             f0.have = f1.have = f2.have = false;
             int nf = 0;
             uint32_t seq = 0;
-            uint32_t qitem[NQ];
+            uint32_t qitem[NQ], qpv[NQ];
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) qitem[q] = 0;
+            for (int q = 0; q < NQ; ++q) qitem[q] = qpv[q] = 0;
             auto pop = [&]() -> bool {
                 const bool r = issue_pv<C>(f0.q, f0, p_full, o_free, v_full, kv_empty, pv_done, abort_flag, p.err,
                                            tmem_base, sV, vdesc, idesc_pv, D, leader);
@@ -982,6 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         e.qt = seq;
                         e.qi = qitem[q];
                         e.nk = tr.nk16;
+                        e.pvn = qpv[q]++;
                         if (nf == 0) f0 = e;
                         else if (nf == 1) f1 = e;
                         else f2 = e;
@@ -1078,6 +1087,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                         pend[q].qt = qtile[q];
                         pend[q].qi = qitem[q];
                         pend[q].nk = tr.nk16;
+                        pend[q].pvn = qtile[q];
                         ++qtile[q];
                     }
                     ++kv_iter;
@@ -1217,12 +1227,14 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     }
                     const float neg_m = (m == -INFINITY) ? 0.f : -m;
                     l += exp_store_row(s_tmem, live, nchunks, s, sl2, neg_m);
-                    if (!first) {
-                        // O may only be touched once the previous P.V has landed.
-                        wait_bar_warp(&pv_done[q], (qtile - 1) & 1, abort_flag, p.err);
+                    // tcgen05.ld/st are warp-collective: the warp rescales if any row needs it, and O may
+                    // only be touched once the previous P.V has landed (without a rescale there is
+                    // nothing to wait for: see kPvRing).
+                    if (!first && __any_sync(0xffffffffu, rescale)) {
+                        wait_bar_warp(&pv_done[q * kPvRing + (qtile - 1) % kPvRing], ((qtile - 1) / kPvRing) & 1,
+                                      abort_flag, p.err);
                         ptx::tc_fence_after();
-                        // tcgen05.ld/st are warp-collective: the warp rescales if any row needs it.
-                        if (__any_sync(0xffffffffu, rescale)) rescale_tmem_cols<D>(o_tmem, rescale ? alpha : 1.f);
+                        rescale_tmem_cols<D>(o_tmem, rescale ? alpha : 1.f);
                     }
                     if (MODE == kDecoderSample && p.P_dev != nullptr && tr.src == 0 && it.P - k0 < tr.nk16) {
                         // Ragged prefix: cache rows at or past P[b] in this tile may hold anything (NaN
@@ -1248,7 +1260,8 @@ __global__ void __launch_bounds__(kThreads, 1) fmha_sm100_kernel(const __grid_co
                     first = false;
                 }
                 // ------------------------------------------------------------ epilogue
-                wait_bar_warp(&pv_done[q], (qtile - 1) & 1, abort_flag, p.err);
+                wait_bar_warp(&pv_done[q * kPvRing + (qtile - 1) % kPvRing], ((qtile - 1) / kPvRing) & 1, abort_flag,
+                              p.err);
                 ptx::tc_fence_after();
                 const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
                 const float lse_val = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;

@@ -1,7 +1,9 @@
 """Protocol walk of the train kernels' pipeline at head_dim <= 64 (fmha_sm100.cuh: three rotating
 S buffers), modelled in Python: one CTA's TMA producer, the MMA warp with its queue of owed P.V
 (S(n) issued only after P.V(n-3); the queue drained at the end of each item), an in-order tensor
-pipe whose commits land later, and the two softmax warpgroups, over random interleavings.  Every
+pipe whose commits land later, and the two softmax warpgroups, over random interleavings.  A
+softmax warp waits for the previous P.V only when it rescales O (random per tile here); the P.V
+completions of a query tile go round a ring of four barriers, so those waits stay unambiguous.  Every
 mbarrier wait is checked for phase aliasing (a parity wait is only correct while the barrier is
 at the awaited phase or one past it), every S for overwriting a P that no P.V has consumed, the
 S numbering of the MMA warp against the softmax side's, and the whole for deadlock.  Item
@@ -53,7 +55,7 @@ class Bar:
         s.arr += 1
         if s.arr == s.count: s.arr = 0; s.ph += 1
 
-def run(mode, L, S, B, H, grid, c, NST, QBUF, NOB, rng):
+def run(mode, L, S, B, H, grid, c, NST, QBUF, NOB, rng, ring=4):
     its = list(items(mode, L, S, B, H, grid, c))
     if not its: return 0
     bars = {}
@@ -65,7 +67,8 @@ def run(mode, L, S, B, H, grid, c, NST, QBUF, NOB, rng):
     for i in range(3): bar(('p_full', i), 1)
     for i in range(6): bar(('s_full', i))
     for i in range(2): bar(('tok', i))
-    for q in range(2): bar(('pv_done', q))
+    for q in range(2):
+        for j in range(ring): bar(('pv_done', q, j))
     for i in range(NOB * 2): bar(('o_free', i), 1)
     tensor = []      # in-order queue of pending completions: list of bar names (commit) ; loads
     loads = []       # async TMA loads: bar names (any order)
@@ -84,7 +87,7 @@ def run(mode, L, S, B, H, grid, c, NST, QBUF, NOB, rng):
                 loads.append(('k_full', st)); loads.append(('v_full', st))
                 kv += 1
     def mma():
-        kv = 0; seq = 0; fifo = []; qitem = [0, 0]
+        kv = 0; seq = 0; fifo = []; qitem = [0, 0]; qpv = [0, 0]
         def pop():
             e = fifo.pop(0)
             sb = e['seq'] % 3
@@ -93,7 +96,7 @@ def run(mode, L, S, B, H, grid, c, NST, QBUF, NOB, rng):
             if e['first'] and e['qi'] // NOB > 0: yield W(('o_free', ob * 2 + e['q']), e['qi'] // NOB - 1)
             yield W(('v_full', e['st']), e['round'])
             state['pv_issued'].add(e['seq'])
-            tensor.append(('pv_done', e['q'])); tensor.append(('kv_empty', e['st']))
+            tensor.append(('pv_done', e['q'], e['pvn'] % ring)); tensor.append(('kv_empty', e['st']))
         for ii, it in enumerate(its):
             qb = ii % QBUF
             yield W(('q_full', qb), ii // QBUF)
@@ -111,7 +114,8 @@ def run(mode, L, S, B, H, grid, c, NST, QBUF, NOB, rng):
                     if seq >= 3: assert seq - 3 in state['pv_issued'], ('S over unconsumed P', seq)
                     state['s_issued'][(ii, t, q)] = seq
                     tensor.append(('s_full', q * 3 + seq % 3))
-                    fifo.append(dict(q=q, seq=seq, st=st, round=rd, first=not seen[q], qi=qitem[q]))
+                    fifo.append(dict(q=q, seq=seq, st=st, round=rd, first=not seen[q], qi=qitem[q], pvn=qpv[q]))
+                    qpv[q] += 1
                     assert len(fifo) <= 3
                     seq += 1; seen[q] = True
                 kv += 1
@@ -134,10 +138,12 @@ def run(mode, L, S, B, H, grid, c, NST, QBUF, NOB, rng):
                 state['soft_seq'][(ii, t, q)] = my
                 yield W(('s_full', q * 3 + my % 3), scnt[my % 3]); scnt[my % 3] += 1
 
-                if not first: yield W(('pv_done', q), qtile - 1)
+                # the warp waits for the previous P.V only when it rescales O (random here)
+                if not first and rng.random() < 0.3:
+                    yield W(('pv_done', q, (qtile - 1) % ring), (qtile - 1) // ring)
                 bars[('p_full', my % 3)].arrive()
                 qtile += 1; first = False
-            yield W(('pv_done', q), qtile - 1)
+            yield W(('pv_done', q, (qtile - 1) % ring), (qtile - 1) // ring)
             bars[('o_free', ob * 2 + q)].arrive()
             qitem += 1
     procs = {'prod': producer(), 'mma': mma(), 's0': softmax(0), 's1': softmax(1)}
@@ -181,6 +187,19 @@ CASES = [(mode, L, S, nob, grid, c)
          for nob in (1, 2)
          for grid in (1, 3)
          for c in range(grid)]
+
+
+def test_single_pv_done_barrier_with_skipped_waits_is_caught():
+    """Planted mistake: one P.V completion barrier per query tile while the softmax skips the wait
+    on tiles without a rescale; the walk must report a wait that a parity check would pass early."""
+    rng = random.Random(5)
+    caught = 0
+    for m, L, S, nob, grid, c in CASES[::7]:
+        try:
+            run(m, L, S, 1, 2, grid, c, 4, 2, nob, rng, ring=1)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
 
 
 @pytest.mark.parametrize("mode", [0, 1])
