@@ -641,9 +641,9 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
             if (wtid == 0) ptx::tma_store_wait_read_all();  // the last unit's output has left the staging buffer
             ptx::named_barrier_sync(3, 128);  // colscale written, column statistics read
             ptx::mbar_arrive(&l_free[ob]);
-            // The unit's rows (whole: bf16 output rows out_row0.., split: the fp32 [col][D] part of
-            // the slot) go straight from registers to global memory: for each column a warp writes
-            // 32 consecutive head-dim values (one 128-byte segment of the slot).
+            // The unit's rows: a whole unit's bf16 output rows out_row0.. go through the staging
+            // buffer; a split unit's fp32 [col][D] partial goes straight from registers to its slot
+            // (for each column a warp writes 32 consecutive head-dim values, one 128-byte segment).
             if (whole) {
                 // bf16 rows staged in shared memory (a pass of columns per staging buffer) and
                 // written with one bulk copy per pass
@@ -689,8 +689,10 @@ __global__ void __launch_bounds__(kKrThreads, 1) fmha_keyrow_kernel(const __grid
                 const int is_last = *bcast;
                 ptx::named_barrier_sync(3, 128);
                 // In the CTA's last unit every K/V, Q and P^T buffer is free (the producers are done
-                // and every product of the unit has landed): the partial slots are then copied in
-                // with one bulk copy each, all in flight at once, and merged from shared memory.
+                // and every product of the unit has landed), and so is the staging buffer (an earlier
+                // unit's output store finished reading it before this unit's first barrier): the
+                // partial slots are then copied in with one bulk copy each, all in flight at once, and
+                // merged from shared memory.
                 const int nparts = c_last - c_first + 1;
                 const uint32_t slot_bytes = static_cast<uint32_t>(p.slot_floats) * 4u;
                 Scheduler<kDecoderSample> peek = sched;
