@@ -94,7 +94,8 @@ def traffic_for(kernel: str):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons (nvidia-smi) while the timed region runs."""
+    """Samples SM clock and throttle reasons while the timed region runs: NVML reads (read-only)
+    every 10 ms when NVML loads, else nvidia-smi queries."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -106,16 +107,40 @@ class ClockSampler:
         self._stop = threading.Event()
         self._thr = None
 
+    def _nvml_handle(self):
+        """NVML handle of the device (read-only queries), or None when NVML is not usable."""
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+        except Exception:
+            return None
+
     def _run(self):
+        nv = self._nvml_handle()
+        bits = (8, 64, 32, 4)  # hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
         while not self._stop.is_set():
             try:
+                if nv is not None:
+                    # NVML reads take microseconds, so the timed region gets many samples; the row
+                    # has the layout of the nvidia-smi query below
+                    m, h = nv
+                    sm = m.nvmlDeviceGetClockInfo(h, m.NVML_CLOCK_SM)
+                    mx = m.nvmlDeviceGetMaxClockInfo(h, m.NVML_CLOCK_SM)
+                    pw = m.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    r = m.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append([str(self.index), str(sm), str(mx), f"{pw:.1f}", hex(r)] +
+                                        ["Active" if r & b else "Not Active" for b in bits])
+                    self._stop.wait(0.01)
+                    continue
                 out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
                                       "--format=csv,noheader,nounits"], capture_output=True, text=True,
                                      timeout=5).stdout.strip()
                 if out:
                     self.samples.append([x.strip() for x in out.split(",")])
             except Exception:
-                pass
+                nv = None
             self._stop.wait(0.05)
 
     def __enter__(self):
